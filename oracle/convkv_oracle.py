@@ -1,0 +1,369 @@
+"""fp64 CPU oracle for the ConvKV Memory attention step.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The product path (the
+C-ABI library and its Python binding) never calls it and has no CPU fallback.
+It shares no code with the CUDA path; the only common dependency is the seeded
+input generator, which holds none of the method's arithmetic.
+
+What it computes, and where that is stated:
+
+* SoulX-LiveAct blog walk-through (gongshangzheng.github.io/paper-liveact.html),
+  section "ConvKV Memory": recent KV is kept exact, older KV is compressed by a
+  lightweight 1D convolution into a fixed-length long-term memory; the context
+  is [long-term memory | short-term memory | current block]; cached KV is
+  append-only; compression starts with the third generated block.
+* Same page, section "Streaming Pipeline": the conv runs once between blocks,
+  and the KV footprint is constant for any stream length.
+* Same page, section "Neighbor Forcing": block-wise causal mask -- the current
+  block sees all history and all of itself (no mask inside the attended set).
+* digi.china.com press article (third technical paragraph): old KV is rolled
+  into a fixed-length representation at a fixed compression ratio, and RoPE
+  Reset re-aligns the position encoding.
+* aiboss88.com summary, section "SoulX-LiveActの技術的原理", ConvKV Memory
+  bullet: the 1D convolution compresses at 5:1 and the RoPE position encoding
+  is reset.
+* Model card (hf.xjtesla.cn/Soul-AILab/LiveAct), "Command Line Arguments"
+  table, ``--fp8_kv_cache``: the KV cache is stored in FP8 and dequantised to
+  BF16 on use.
+
+Readings taken where the pages are silent (each listed in the design notes):
+W counts past-block frames only and eviction happens at append time in
+groups of 5 until the window holds at most W frames; the memory is a FIFO of
+C slots (oldest dropped); the conv is a per-head cross-correlation over the 5
+evicted frames (tap j = j-th oldest frame), no bias, applied to un-rotated K
+and V; compressed slots are stored in the cache's storage type (bf16 rounded
+to nearest even, or e4m3 with a per-(head, slot) fp32 scale); RoPE time
+indices restart at 0 over [memory | window | current], one index per memory
+slot, spatial (row, column) indices are kept; RoPE rotates adjacent pairs of
+each axis segment [t | h | w] with frequency theta^(-2i/d_axis); softmax scale
+is 1/sqrt(D).  In the fp8 variant the current block is attended in bf16 and is
+quantised when it joins the window.
+
+Parity status: every function below is pinned by tests under ``tests/`` that
+check it against closed forms, library routines or hand-derived tables (no
+function is left unpinned).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+# Partition codes of a key frame in the attended sequence.
+PART_MEMORY, PART_WINDOW, PART_CURRENT = 0, 1, 2
+EVICT = 5          # frames per eviction group = conv kernel = conv stride (5:1)
+E4M3_MAX = 448.0   # largest finite e4m3 value
+
+
+# --------------------------------------------------------------------------
+# bf16 / e4m3 storage rounding
+# --------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even).
+
+    The cache stores K/V in bf16; a compressed slot is stored in the same type.
+    Done on the exact binary expansion: bf16 keeps 8 significant bits, so the
+    value is rounded at the bit below the 8th significant bit.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    m, e = np.frexp(x[nz])              # x = m * 2^e, 0.5 <= |m| < 1
+    q = np.round(m * 256.0)              # 8 significant bits, numpy rounds half to even
+    out[nz] = np.ldexp(q / 256.0, e)
+    return out
+
+
+def e4m3_rne_satfinite(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest e4m3 value (ties to even), saturating to +-448.
+
+    e4m3 (OCP FP8): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; normal
+    numbers 2^-6 .. 448, subnormals are multiples of 2^-9.  A value with
+    exponent e (|x| in [2^e, 2^(e+1))) has quantum 2^(e-3); below 2^-6 the
+    quantum is 2^-9.  Values beyond 448 saturate to 448.
+    """
+    x = np.asarray(x32, dtype=np.float32).astype(np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))   # a = m * 2^ex, 0.5 <= m < 1
+    e = np.maximum(ex.astype(np.float64) - 1.0, -6.0)
+    quantum = np.exp2(e - 3.0)
+    q = np.round(a / quantum) * quantum   # exact: a and quantum are dyadic
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(a > 0, np.copysign(q, x), 0.0 * x)
+
+
+def fp8_quantize(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-head e4m3 quantisation of one frame or slot x[T, H, D].
+
+    scale = amax / 448 in fp32 (1 if amax == 0); code = e4m3(fp32(x) / scale)
+    with the fp32 divide rounded to nearest.  Returns (dequantised values
+    code * scale in float64, scales[H] as float32).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    x32 = x.astype(np.float32)
+    amax = np.abs(x32).max(axis=(0, 2))                      # [H], fp32
+    scale = np.where(amax == 0, np.float32(1.0), (amax / np.float32(E4M3_MAX)).astype(np.float32))
+    scale = scale.astype(np.float32)
+    y = (x32 / scale[None, :, None]).astype(np.float32)      # IEEE fp32 divide
+    code = e4m3_rne_satfinite(y)
+    return code * scale.astype(np.float64)[None, :, None], scale
+
+
+# --------------------------------------------------------------------------
+# RoPE with reset positions
+# --------------------------------------------------------------------------
+
+def rope_split(D: int) -> Tuple[int, int, int]:
+    """Channel split (time, row, column) of head_dim D: 44/42/42 for D=128.
+
+    Row and column each get 2*floor(D/6) channels, time gets the rest.
+    """
+    dh = 2 * (D // 6)
+    return D - 2 * dh, dh, dh
+
+
+def rope_rotate(x: np.ndarray, t: np.ndarray, y: np.ndarray, xc: np.ndarray,
+                split: Tuple[int, int, int], theta: float) -> np.ndarray:
+    """Rotate x[..., D] by 3D RoPE at positions (t, y, xc) (broadcast over x[..., 0]).
+
+    Channels [0, d_t) use the time index, [d_t, d_t+d_h) the row index and the
+    rest the column index.  Inside an axis segment of width d, pair i (channels
+    2i, 2i+1 of the segment) turns by angle pos * theta^(-2i/d):
+    (a, b) -> (a cos - b sin, a sin + b cos).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    start = 0
+    for width, pos in zip(split, (t, y, xc)):
+        i = np.arange(width // 2, dtype=np.float64)
+        freq = theta ** (-2.0 * i / width)
+        ang = np.asarray(pos, dtype=np.float64)[..., None] * freq
+        c, s = np.cos(ang), np.sin(ang)
+        a = x[..., start:start + width:2]
+        b = x[..., start + 1:start + width:2]
+        out[..., start:start + width:2] = a * c - b * s
+        out[..., start + 1:start + width:2] = a * s + b * c
+        start += width
+    return out
+
+
+# --------------------------------------------------------------------------
+# 1D conv compression of one eviction group
+# --------------------------------------------------------------------------
+
+def conv_compress(group: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Compress 5 frames group[5, T, H, D] into one slot [T, H, D].
+
+    out[s, h, o] = sum_j sum_i w[h, o, i, j] * group[j, s, h, i]
+    (per-head channel mixing, kernel 5 = stride 5 over time, no padding,
+    no bias, tap j = j-th oldest frame).
+    """
+    g = np.asarray(group, dtype=np.float64)
+    wf = np.asarray(w, dtype=np.float64)
+    assert g.shape[0] == EVICT and wf.shape[-1] == EVICT
+    return np.einsum("hoij,jshi->sho", wf, g, optimize=True)
+
+
+# --------------------------------------------------------------------------
+# attention of query rows over one key/value sequence
+# --------------------------------------------------------------------------
+
+def attend_rows(q_rot: np.ndarray, k_rot: np.ndarray, v: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """softmax(q k^T / sqrt(D)) v for one head, unmasked.
+
+    q_rot[n, D], k_rot[Nk, D], v[Nk, D] -> (o[n, D], sum of the normalised
+    weights per row, which is 1 up to rounding).
+    """
+    D = q_rot.shape[-1]
+    s = (q_rot @ k_rot.T) / np.sqrt(D)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    l = p.sum(axis=1, keepdims=True)
+    p = p / l
+    return p @ v, p.sum(axis=1)
+
+
+# --------------------------------------------------------------------------
+# the streaming state of one layer / denoising step
+# --------------------------------------------------------------------------
+
+@dataclass
+class OracleConfig:
+    H: int
+    D: int
+    grid_h: int
+    grid_w: int
+    window: int            # W, past-block frames kept exact
+    mem_slots: int         # C, FIFO capacity of compressed slots
+    theta: float = 1e4
+    fp8: bool = False
+    split: Optional[Tuple[int, int, int]] = None
+
+    @property
+    def T(self) -> int:
+        return self.grid_h * self.grid_w
+
+    def rope(self) -> Tuple[int, int, int]:
+        return self.split if self.split is not None else rope_split(self.D)
+
+
+@dataclass
+class _Frame:
+    k: np.ndarray          # [T, H, D] float64 (stored values)
+    v: np.ndarray
+    index: int             # stream frame index (window/current) or slot index (memory)
+
+
+@dataclass
+class ConvEvent:
+    block: int             # 1-based block number of the append that ran it
+    first_frame: int       # stream index of the oldest evicted frame (g0)
+    slot: int              # slot index S-1 (covers frames [5*slot, 5*slot+5))
+
+
+class OracleStream:
+    """Reference state machine for one layer / denoising-step KV cache."""
+
+    def __init__(self, cfg: OracleConfig, conv_w: np.ndarray):
+        """conv_w: [2 (K, V), H, D_out, D_in, 5], float64 (exact bf16 values)."""
+        self.cfg = cfg
+        self.w = np.asarray(conv_w, dtype=np.float64)
+        self.window: List[_Frame] = []
+        self.current: List[_Frame] = []
+        self.current_q8: List[_Frame] = []   # fp8: quantised form of the current frames
+        self.memory: List[_Frame] = []
+        self.P = 0        # frames promoted into the window so far
+        self.E = 0        # frames evicted so far
+        self.S = 0        # slots produced so far
+        self.block = 0
+        self.events: List[ConvEvent] = []
+        self.mem_scales: List[np.ndarray] = []  # fp8: per-slot [2, H] scales
+        self.frame_scales = {}                  # fp8: stream frame -> [2, H] scales
+
+    # -- append ------------------------------------------------------------
+    def append(self, k: np.ndarray, v: np.ndarray) -> List[ConvEvent]:
+        """Append one block k, v[b, T, H, D] (exact input values)."""
+        cfg = self.cfg
+        self.block += 1
+        # (i) the previous current block joins the window
+        promoted = self.current_q8 if cfg.fp8 else self.current
+        self.window.extend(promoted)
+        self.P += len(promoted)
+        self.current, self.current_q8 = [], []
+        # (ii) evict the oldest 5 frames while the window holds more than W
+        new_events = []
+        while len(self.window) > cfg.window:
+            group, self.window = self.window[:EVICT], self.window[EVICT:]
+            kc = conv_compress(np.stack([f.k for f in group]), self.w[0])
+            vc = conv_compress(np.stack([f.v for f in group]), self.w[1])
+            if cfg.fp8:
+                kc, sk = fp8_quantize(kc)
+                vc, sv = fp8_quantize(vc)
+                scales = np.stack([sk, sv])
+            else:
+                kc, vc = round_to_bf16(kc), round_to_bf16(vc)
+                scales = None
+            if len(self.memory) == cfg.mem_slots:
+                self.memory.pop(0)
+                self.mem_scales.pop(0)
+            self.memory.append(_Frame(kc, vc, self.S))
+            self.mem_scales.append(scales)
+            ev = ConvEvent(self.block, group[0].index, self.S)
+            self.E += EVICT
+            self.S += 1
+            self.events.append(ev)
+            new_events.append(ev)
+        # (iii) the new block becomes the current block
+        b = k.shape[0]
+        for f in range(b):
+            idx = self.P + f
+            kf = np.asarray(k[f], dtype=np.float64)
+            vf = np.asarray(v[f], dtype=np.float64)
+            self.current.append(_Frame(kf, vf, idx))
+            if cfg.fp8:
+                kq, sk = fp8_quantize(kf)
+                vq, sv = fp8_quantize(vf)
+                self.current_q8.append(_Frame(kq, vq, idx))
+                self.frame_scales[idx] = np.stack([sk, sv])
+        return new_events
+
+    # -- layout ------------------------------------------------------------
+    def key_frames(self) -> List[Tuple[int, _Frame, int]]:
+        """(partition, frame, RoPE time index) in attended order."""
+        out = []
+        t = 0
+        for f in self.memory:
+            out.append((PART_MEMORY, f, t)); t += 1
+        for f in self.window:
+            out.append((PART_WINDOW, f, t)); t += 1
+        for f in self.current:
+            out.append((PART_CURRENT, f, t)); t += 1
+        return out
+
+    def layout(self) -> np.ndarray:
+        """int64 rows (partition, source index, RoPE time) per key frame.
+
+        source index = stream frame index for window/current frames, slot index
+        for memory slots (slot k covers stream frames [5k, 5k+5)).
+        """
+        return np.array([(p, f.index, t) for p, f, t in self.key_frames()], dtype=np.int64).reshape(-1, 3)
+
+    @property
+    def m(self) -> int:
+        return len(self.memory)
+
+    @property
+    def w_frames(self) -> int:
+        return len(self.window)
+
+    # -- attend ------------------------------------------------------------
+    def attend(self, q: np.ndarray, rows: Optional[Sequence[int]] = None, heads: Optional[Sequence[int]] = None,
+               t_offset: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+        """Attention of the current block's queries over [memory | window | current].
+
+        q: [b, T, H, D] exact query values (the block's own queries).
+        rows: query rows r in [0, b*T) to evaluate (all if None); row r is
+        token r % T of current frame r // T.
+        t_offset: added to every time index (both queries and keys); the output
+        must not depend on it (RoPE is relative).
+        Returns (o[n, H', D], weight sums[n, H']) in float64.
+        """
+        cfg = self.cfg
+        T, D = cfg.T, cfg.D
+        b = q.shape[0]
+        assert b == len(self.current), "attend() must follow the append of the same block"
+        rows = np.arange(b * T) if rows is None else np.asarray(rows, dtype=np.int64)
+        heads = list(range(cfg.H)) if heads is None else list(heads)
+        kf = self.key_frames()
+        tok = np.arange(T)
+        ky, kx = tok // cfg.grid_w, tok % cfg.grid_w
+        k_t = np.concatenate([np.full(T, t) for _, _, t in kf]) + t_offset
+        k_y = np.tile(ky, len(kf))
+        k_x = np.tile(kx, len(kf))
+        qf, qs = rows // T, rows % T
+        q_t = (self.m + self.w_frames + qf) + t_offset
+        q_y, q_x = qs // cfg.grid_w, qs % cfg.grid_w
+        split = cfg.rope()
+        o = np.zeros((len(rows), len(heads), D))
+        psum = np.zeros((len(rows), len(heads)))
+        for hi, h in enumerate(heads):
+            kh = np.concatenate([f.k[:, h, :] for _, f, _ in kf])
+            vh = np.concatenate([f.v[:, h, :] for _, f, _ in kf])
+            k_rot = rope_rotate(kh, k_t, k_y, k_x, split, cfg.theta)
+            q_rows = np.asarray(q[qf, qs, h, :], dtype=np.float64)
+            q_rot = rope_rotate(q_rows, q_t, q_y, q_x, split, cfg.theta)
+            o[:, hi, :], psum[:, hi] = attend_rows(q_rot, k_rot, vh)
+        return o, psum
+
+    def memory_slot(self, age: int) -> Tuple[np.ndarray, np.ndarray]:
+        """Stored (K, V) of the memory slot `age` positions after the oldest."""
+        f = self.memory[age]
+        return f.k, f.v
