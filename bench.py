@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Benchmark of the ConvKV Memory attention step on B200.
+
+One step = one block of the stream through the whole path: append (promote,
+evict + conv-compress, ring copy) and the fused reset-RoPE attention.  The
+workload is the 512x512 shape (H=40, D=128, 32x32 tokens, blocks of 8 frames,
+window 10, memory 8) in steady state (memory full), inputs resident in HBM.
+
+Prints one JSON line (rank 0).  With --impl reference the fp64 CPU oracle is
+timed instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ConvKV attend TFLOP/s (append+compress+attend step), latent frames/s per layer-step, % bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(Nq, Nk, D, H, S=1):
+    return 4.0 * Nq * Nk * D * H * S
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, rows: int, seed_offset: int = 0):
+    """A steady-state oracle state of workload w built directly from seeded frames
+    (memory slots, window, current block), plus the queries of the current block."""
+    import numpy as np
+    import seeded_inputs as si
+    from oracle import convkv_oracle as O
+    cfg = O.OracleConfig(H=w.heads, D=w.head_dim, grid_h=w.grid_h, grid_w=w.grid_w, window=w.window_frames,
+                         mem_slots=w.mem_slots)
+    wts = si.bf16_bits_to_f64(si.conv_weights(w.seed, 0, w.heads, w.head_dim))
+    st = O.OracleStream(cfg, wts)
+    fe = w.T * w.heads * w.head_dim
+    shape = (w.T, w.heads, w.head_dim)
+
+    def fr(tensor, f):
+        return si.bf16_bits_to_f64(si.frames(w.seed, tensor, 0, f, 1, fe)).reshape(shape)
+
+    C, W, b = w.mem_slots, 8, w.block_frames
+    st.memory = [O._Frame(O.round_to_bf16(fr(si.K, 1000 + i)), O.round_to_bf16(fr(si.V, 1000 + i)), i)
+                 for i in range(C)]
+    st.window = [O._Frame(fr(si.K, 40 + i), fr(si.V, 40 + i), 40 + i) for i in range(W)]
+    st.current = [O._Frame(fr(si.K, 48 + i), fr(si.V, 48 + i), 48 + i) for i in range(b)]
+    q = np.stack([fr(si.Q, 48 + i) for i in range(b)])
+    group = np.stack([fr(si.K, 40 + i) for i in range(5)])
+    rng = np.random.default_rng(seed_offset)
+    r = rng.choice(b * w.T, size=rows, replace=False)
+    Nk = (C + W + b) * w.T
+    return st, q, r, group, wts, Nk
+
+
+def time_oracle(w, rows: int, reps: int = 1, seed_offset: int = 0):
+    """Seconds and algorithmic FLOPs of the oracle on `rows` query rows (all heads) + one conv group."""
+    from oracle import convkv_oracle as O
+    st, q, r, group, wts, Nk = oracle_sample(w, rows, seed_offset)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        st.attend(q, rows=r)
+        O.conv_compress(group, wts[0])
+    dt = time.perf_counter() - t0
+    conv = 2.0 * w.T * 5 * w.head_dim * w.head_dim * w.heads
+    flops = reps * (attention_flops(rows, Nk, w.head_dim, w.heads) + conv)
+    return dt, flops, Nk
+
+
+def cpu_baseline(w, budget_rows: int = 256):
+    dt, flops, Nk = time_oracle(w, budget_rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{budget_rows} query rows x {w.heads} heads of one steady-state {w.name} block "
+                      f"(Nk={Nk}) + one conv group, fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 32
+    for _ in range(args.warmup):
+        time_oracle(w, rows)
+    total_dt, total_flops = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl, Nk = time_oracle(w, rows, seed_offset=i + 1)
+        total_dt += dt
+        total_flops += fl
+    value = total_flops / total_dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
+            "config": {"workload": f"{w.name} steady state, oracle sample of {rows} query rows x {w.heads} heads "
+                                   f"per step + one conv group", "Nk": Nk},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": f"{rows} query rows x {w.heads} heads + one K conv group per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        smax = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------- our path
+
+def run_ours(args, w):
+    import torch
+    import seeded_inputs as si
+    import compressed_kv_cache_convkv_b200 as ckv
+    from compressed_kv_cache_convkv_b200 import build
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if rank == 0:
+        build.build()
+        si.build(device=True)
+    if dist is not None:
+        dist.barrier()
+
+    S, H, D, T = w.num_states, w.heads, w.head_dim, w.T
+    cfg = w.config(host_io=True)
+    stream = torch.cuda.current_stream()
+    fe = T * H * D
+    # conv weights and inputs: seeded, generated on the device (each rank its own layer state)
+    weights = torch.empty((S, 2, H, D, D, 5), dtype=torch.bfloat16, device="cuda")
+    for s in range(S):
+        for kv, tid in ((0, si.WK), (1, si.WV)):
+            si.frames_device(weights[s, kv].data_ptr(), w.seed + rank, tid, s, 0, 1, H * D * D * 5,
+                             si.weight_scale(D), stream.cuda_stream)
+    h = ckv.ConvKV(cfg, weights, stream=stream)
+    b = w.block_frames
+    npool = 3
+    pool = []
+    for p in range(npool):
+        t3 = []
+        for tid in (si.Q, si.K, si.V):
+            x = torch.empty((S, b * T, H, D), dtype=torch.bfloat16, device="cuda")
+            for s in range(S):
+                si.frames_device(x[s].data_ptr(), w.seed + rank, tid, s, 100 + p * b, b, fe, 1.0, stream.cuda_stream)
+            t3.append(x)
+        pool.append(t3)
+    out = torch.empty((S, b * T, H, D), dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        q, k, v = pool[i % npool]
+        h.append(k, v)
+        return q
+
+    # fill to steady state (memory full) -- untimed
+    first = w.first_block_frames
+    q0, k0, v0 = (x[:, : first * T].contiguous() for x in pool[0])
+    h.append(k0, v0)
+    h.attend(q0)
+    while h.counters()["m"] < w.mem_slots or h.counters()["blocks"] < 8:
+        q = step(0)
+        h.attend(q, out)
+    for i in range(args.warmup):
+        q = step(i)
+        h.attend(q, out)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flops, nk_list = [], []
+    groups = 0
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = h.launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(K):
+            q = step(i)
+            c = h.counters()
+            groups += c["groups"]
+            nk = (c["m"] + c["w"] + c["b"]) * T
+            nk_list.append(nk)
+            flops.append(attention_flops(b * T, nk, D, H, S))
+            ev[i][0].record(stream)
+            h.attend(q, out)
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    launches = h.launch_count() - launches0
+    total_ms = start.elapsed_time(end)
+    att_ms = [a.elapsed_time(bb) for a, bb in ev]
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    clocks = clk.summary()
+
+    # end to end through the host-buffer entry points: pinned host q/k/v in, host out back, every step
+    qh = pool[0][0].cpu().pin_memory()
+    kh = pool[0][1].cpu().pin_memory()
+    vh = pool[0][2].cpu().pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    Ke = max(3, min(K, 10))
+    for _ in range(2):
+        h.append_host(kh, vh)
+        h.attend_host(qh, oh)
+    torch.cuda.synchronize()
+    e2e_flops = 0.0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(Ke):
+        h.append_host(kh, vh)
+        c = h.counters()
+        e2e_flops += attention_flops(b * T, (c["m"] + c["w"] + c["b"]) * T, D, H, S)
+        h.attend_host(qh, oh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert h.status() == 0, "device status reported an error"
+
+    pk, kind = peaks()
+    total_flops = sum(flops) * world
+    value = total_flops / (total_ms * 1e-3) / 1e12
+    att_avg_ms = statistics.mean(att_ms)
+    att_achieved = statistics.mean(flops) / (att_avg_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    frames_per_s = K * b * S * world / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
+        "config": {"workload": f"{w.name} steady state (memory full), one layer state per GPU",
+                   "heads": H, "head_dim": D, "tokens_per_frame": T, "block_frames": b,
+                   "window_frames": w.window_frames, "mem_slots": w.mem_slots, "states": S,
+                   "keys_per_step_avg": statistics.mean(nk_list), "state_bytes": h.state_bytes(),
+                   "l2": "inputs larger than L2 (q,k,v 252 MB/step + 671 MB K/V state vs 126 MB L2)",
+                   "parallelism": f"replicas x{world} (independent layer states, no collective)"},
+        "latent_frames_per_s_per_layer_step": frames_per_s,
+        "pct_bf16_peak": 100.0 * value / peak,
+        "kernels_ms": {"attend_avg": att_avg_ms, "append_compress_avg": (total_ms - sum(att_ms)) / K,
+                       "conv_groups_per_step": groups / K},
+        "roofline": {"bound": "tensor", "achieved": att_achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": att_achieved / peak, "traffic": None,
+                     "kernel": "attn_kernel<128>", "peak_source": f"{kind} bf16 burst (MEASURED_PEAKS.json)"},
+        "e2e": {"value": e2e_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 3 * S * b * fe * 2, "d2h_bytes_per_step": S * b * fe * 2},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    h.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="512x512")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from compressed_kv_cache_convkv_b200.configs import PRESETS
+    w = PRESETS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

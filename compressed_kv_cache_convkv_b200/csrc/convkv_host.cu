@@ -1,0 +1,497 @@
+// Host side of the ConvKV C ABI: configuration checks, the integer bookkeeping
+// of the ring window / FIFO memory (bit-exact, independent of stream length),
+// the single device arena, RoPE tables, TMA descriptors and launch order.
+//
+// Bookkeeping (SoulX-LiveAct blog walk-through, sections "ConvKV Memory" and
+// "Streaming Pipeline"; aiboss88.com summary, ConvKV bullet, for the 5:1 ratio):
+//   P  frames promoted into the window so far, E frames evicted, S slots made.
+//   append(b): P += b_prev; while P - E > W: compress frames [E, E+5) into slot
+//              S (memory position S mod C), E += 5, S += 1; the new block goes to
+//              ring slots (P + f) mod R with R = W + max(b1, b).
+//   attend:    keys = stored slots S-m .. S-1 (m = min(S, C)) at time 0..m-1,
+//              then frames E .. P+b-1 at time m + (f - E).
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/convkv.h"
+#include "convkv_internal.h"
+
+using namespace ckv;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct convkv {
+  convkv_cfg cfg{};
+  int H = 0, D = 0, T = 0, gh = 0, gw = 0, b1 = 0, bn = 0, Bmax = 0, W = 0, C = 0, R = 0, S = 0;
+  int PT = 0, PH = 0, PW = 0, tab_t_rows = 0;
+  bool dry = false, mean = false, fp8 = false, host_io = false;
+  // bookkeeping
+  int64_t P = 0, E = 0, Sn = 0, blocks = 0;
+  int bcur = 0, last_groups = 0;
+  // device memory
+  void* arena = nullptr;
+  size_t arena_bytes = 0;
+  void *ringK = nullptr, *ringV = nullptr, *memK = nullptr, *memV = nullptr, *weights = nullptr;
+  float2* tables = nullptr;
+  int* status = nullptr;
+  void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
+  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{};
+  cudaStream_t stream = nullptr;
+  int64_t launches = 0;
+  int last_cuda = 0;
+
+  int cuda_fail(cudaError_t e) {
+    last_cuda = static_cast<int>(e);
+    return CONVKV_ERR_CUDA;
+  }
+  int64_t frame_elems() const { return static_cast<int64_t>(T) * H * D; }
+  int m() const { return static_cast<int>(Sn < C ? Sn : C); }
+  int w() const { return static_cast<int>(P - E); }
+};
+
+namespace {
+
+int encode_4d(CUtensorMap* map, void* ptr, int D, int H, int64_t rows, int S) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return CONVKV_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(S)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                           static_cast<cuuint64_t>(rows) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVKV_OK : CONVKV_ERR_CUDA;
+}
+
+int encode_weights(CUtensorMap* map, void* ptr, int D, int H, int S) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return CONVKV_ERR_CUDA;
+  const cuuint64_t rows = static_cast<cuuint64_t>(2) * H * kEvict * D;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), rows, static_cast<cuuint64_t>(S)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, rows * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(D), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVKV_OK : CONVKV_ERR_CUDA;
+}
+
+int validate(const convkv_cfg* c) {
+  if (!c) return CONVKV_ERR_INVALID_ARG;
+  if (c->heads < 1 || c->head_dim < 1 || c->grid_h < 1 || c->grid_w < 1 || c->first_block_frames < 1 ||
+      c->block_frames < 1 || c->window_frames < 4 || c->mem_slots < 1 || c->num_states < 1 ||
+      !(c->rope_theta > 0.0) || c->t_offset < 0)
+    return CONVKV_ERR_INVALID_ARG;
+  if (c->evict_frames != kEvict) return CONVKV_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return CONVKV_ERR_UNSUPPORTED;
+  if (c->kv_format != CONVKV_KV_BF16 && c->kv_format != CONVKV_KV_FP8_E4M3) return CONVKV_ERR_INVALID_ARG;
+  if (c->compress_mode != CONVKV_COMPRESS_CONV && c->compress_mode != CONVKV_COMPRESS_MEAN)
+    return CONVKV_ERR_INVALID_ARG;
+  if (c->flags & ~(CONVKV_FLAG_DRY_RUN | CONVKV_FLAG_HOST_IO)) return CONVKV_ERR_INVALID_ARG;
+  const int D = c->head_dim;
+  const int dh = 2 * (D / 6);
+  const bool dflt = c->rope_t == 0 && c->rope_h == 0 && c->rope_w == 0;
+  if (!dflt && (c->rope_t != D - 2 * dh || c->rope_h != dh || c->rope_w != dh)) return CONVKV_ERR_UNSUPPORTED;
+  const int Bmax = c->first_block_frames > c->block_frames ? c->first_block_frames : c->block_frames;
+  if ((c->window_frames + Bmax) / kEvict > kMaxGroups) return CONVKV_ERR_UNSUPPORTED;
+  const int64_t T = static_cast<int64_t>(c->grid_h) * c->grid_w;
+  const int64_t R = c->window_frames + Bmax;
+  // TMA coordinates and row counts are 32-bit
+  if (T * (R > c->mem_slots ? R : c->mem_slots) > (int64_t(1) << 30) || T * Bmax > (int64_t(1) << 30))
+    return CONVKV_ERR_UNSUPPORTED;
+  const int64_t tabs = (int64_t(c->mem_slots) + c->window_frames + Bmax) * (D - 2 * dh) / 2 +
+                       (int64_t(c->grid_h) + c->grid_w) * dh / 2;
+  if (tabs * 8 > 32 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables must fit in shared memory
+  if (c->kv_format == CONVKV_KV_FP8_E4M3 && !(c->flags & CONVKV_FLAG_DRY_RUN)) return CONVKV_ERR_UNSUPPORTED;
+  if (c->compress_mode == CONVKV_COMPRESS_CONV && !(c->flags & CONVKV_FLAG_DRY_RUN) && !c->conv_weight)
+    return CONVKV_ERR_INVALID_ARG;
+  return CONVKV_OK;
+}
+
+void build_tables(const convkv* h, std::vector<float2>& out) {
+  // rows of (cos, sin) for pair i of an axis with 2*npairs channels: angle = pos * theta^(-2i/(2*npairs))
+  auto axis = [&](int rows, int npairs, int offset) {
+    for (int r = 0; r < rows; ++r)
+      for (int i = 0; i < npairs; ++i) {
+        const double freq = std::pow(h->cfg.rope_theta, -2.0 * i / (2.0 * npairs));
+        const double ang = static_cast<double>(r + offset) * freq;
+        out.push_back(make_float2(static_cast<float>(std::cos(ang)), static_cast<float>(std::sin(ang))));
+      }
+  };
+  axis(h->tab_t_rows, h->PT, h->cfg.t_offset);
+  axis(h->gh, h->PH, 0);
+  axis(h->gw, h->PW, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* convkv_strerror(int code) {
+  switch (code) {
+    case CONVKV_OK: return "ok";
+    case CONVKV_ERR_INVALID_ARG: return "invalid argument";
+    case CONVKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CONVKV_ERR_BAD_ORDER: return "call out of order";
+    case CONVKV_ERR_OOM: return "device allocation failed";
+    case CONVKV_ERR_CUDA: return "CUDA error";
+    case CONVKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    default: return "unknown error";
+  }
+}
+
+int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
+  if (!out) return CONVKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = validate(cfg);
+  if (rc) return rc;
+  convkv* h = new (std::nothrow) convkv;
+  if (!h) return CONVKV_ERR_OOM;
+  h->cfg = *cfg;
+  h->H = cfg->heads;
+  h->D = cfg->head_dim;
+  h->gh = cfg->grid_h;
+  h->gw = cfg->grid_w;
+  h->T = cfg->grid_h * cfg->grid_w;
+  h->b1 = cfg->first_block_frames;
+  h->bn = cfg->block_frames;
+  h->Bmax = h->b1 > h->bn ? h->b1 : h->bn;
+  h->W = cfg->window_frames;
+  h->C = cfg->mem_slots;
+  h->R = h->W + h->Bmax;
+  h->S = cfg->num_states;
+  h->PH = cfg->head_dim / 6;
+  h->PW = h->PH;
+  h->PT = (cfg->head_dim - 4 * h->PH) / 2;
+  h->tab_t_rows = h->C + h->W + h->Bmax;
+  h->dry = (cfg->flags & CONVKV_FLAG_DRY_RUN) != 0;
+  h->host_io = (cfg->flags & CONVKV_FLAG_HOST_IO) != 0;
+  h->mean = cfg->compress_mode == CONVKV_COMPRESS_MEAN;
+  h->fp8 = cfg->kv_format == CONVKV_KV_FP8_E4M3;
+  h->stream = static_cast<cudaStream_t>(cfg->stream);
+  h->cfg.conv_weight = nullptr;
+  if (h->dry) {
+    *out = h;
+    return CONVKV_OK;
+  }
+
+  const size_t fe = static_cast<size_t>(h->frame_elems());
+  const size_t ring_b = static_cast<size_t>(h->S) * h->R * fe * 2;
+  const size_t mem_b = static_cast<size_t>(h->S) * h->C * fe * 2;
+  const size_t w_b = h->mean ? 0 : static_cast<size_t>(h->S) * 2 * h->H * kEvict * h->D * h->D * 2;
+  std::vector<float2> tab;
+  build_tables(h, tab);
+  const size_t tab_b = tab.size() * sizeof(float2);
+  const size_t io_b = h->host_io ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_rk = take(ring_b), o_rv = take(ring_b), o_mk = take(mem_b), o_mv = take(mem_b), o_w = take(w_b),
+               o_tab = take(tab_b), o_st = take(sizeof(int)), o_q = take(io_b), o_k = take(io_b),
+               o_v = take(io_b), o_o = take(io_b);
+  h->arena_bytes = off;
+  cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
+  if (e != cudaSuccess) {
+    h->arena = nullptr;
+    delete h;
+    cudaGetLastError();
+    return CONVKV_ERR_OOM;
+  }
+  char* a = static_cast<char*>(h->arena);
+  h->ringK = a + o_rk;
+  h->ringV = a + o_rv;
+  h->memK = a + o_mk;
+  h->memV = a + o_mv;
+  h->weights = w_b ? a + o_w : nullptr;
+  h->tables = reinterpret_cast<float2*>(a + o_tab);
+  h->status = reinterpret_cast<int*>(a + o_st);
+  if (h->host_io) {
+    h->io_q = a + o_q;
+    h->io_k = a + o_k;
+    h->io_v = a + o_v;
+    h->io_out = a + o_o;
+  }
+  // zero fill: rows past a segment's end are read (then masked) and must be finite
+  if ((e = cudaMemsetAsync(h->arena, 0, h->arena_bytes, h->stream)) != cudaSuccess) goto fail_cuda;
+  if ((e = cudaMemcpyAsync(h->tables, tab.data(), tab_b, cudaMemcpyHostToDevice, h->stream)) != cudaSuccess)
+    goto fail_cuda;
+  if (w_b) {
+    if ((e = static_cast<cudaError_t>(launch_permute_weights(cfg->conv_weight, h->weights, h->S, h->H, h->D,
+                                                             h->stream))) != cudaSuccess)
+      goto fail_cuda;
+    h->launches++;
+  }
+  if ((e = cudaStreamSynchronize(h->stream)) != cudaSuccess) goto fail_cuda;
+  rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+  if (!rc) rc = encode_4d(&h->mapRingV, h->ringV, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+  if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+  if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+  if (!rc && w_b) rc = encode_weights(&h->mapW, h->weights, h->D, h->H, h->S);
+  if (rc) {
+    cudaFree(h->arena);
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return CONVKV_OK;
+fail_cuda:
+  cudaStreamSynchronize(h->stream);
+  cudaFree(h->arena);
+  delete h;
+  return CONVKV_ERR_CUDA;
+}
+
+void convkv_destroy(convkv_t* h) {
+  if (!h) return;
+  if (h->arena) {
+    cudaStreamSynchronize(h->stream);
+    cudaFree(h->arena);
+  }
+  delete h;
+}
+
+size_t convkv_state_bytes(const convkv_t* h) { return h ? h->arena_bytes : 0; }
+
+int64_t convkv_launch_count(const convkv_t* h) { return h ? h->launches : 0; }
+
+int convkv_last_cuda_error(const convkv_t* h) { return h ? h->last_cuda : 0; }
+
+int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
+  if (!h || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
+  if (!h->dry && (!k || !v)) return CONVKV_ERR_INVALID_ARG;
+  // 1. the previous current block joins the window
+  h->P += h->bcur;
+  // 2. evict groups of 5 while the window holds more than W frames
+  std::vector<std::pair<int64_t, int64_t>> groups;  // (first frame, slot index)
+  while (h->P - h->E > h->W) {
+    groups.emplace_back(h->E, h->Sn);
+    h->E += kEvict;
+    h->Sn += 1;
+  }
+  h->last_groups = static_cast<int>(groups.size());
+  // groups older than the last C of this call would be dropped by the FIFO before anyone reads them
+  const size_t first = groups.size() > static_cast<size_t>(h->C) ? groups.size() - h->C : 0;
+  h->bcur = frames;
+  h->blocks += 1;
+  if (h->dry) return CONVKV_OK;
+
+  if (groups.size() > first) {
+    ConvParams cp{};
+    cp.H = h->H;
+    cp.T = h->T;
+    cp.S = h->S;
+    cp.C = h->C;
+    cp.R = h->R;
+    cp.ngroups = static_cast<int>(groups.size() - first);
+    for (size_t g = first; g < groups.size(); ++g) {
+      ConvGroup& cg = cp.grp[g - first];
+      for (int j = 0; j < kEvict; ++j) cg.ring_slot[j] = static_cast<int>((groups[g].first + j) % h->R);
+      cg.mem_pos = static_cast<int>(groups[g].second % h->C);
+    }
+    cp.memK = h->memK;
+    cp.memV = h->memV;
+    cp.status = h->status;
+    int e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
+                    : launch_conv_bf16(h->D, cp, h->mapRingK, h->mapRingV, h->mapW, h->stream);
+    h->launches++;
+    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  }
+  // 3. the new block becomes the current block: copy into ring slots (P + f) mod R
+  AppendParams ap{};
+  ap.S = h->S;
+  ap.b = frames;
+  ap.R = h->R;
+  ap.slot0 = static_cast<int>(h->P % h->R);
+  ap.frame_elems = h->frame_elems();
+  int e = launch_append_bf16(ap, k, v, h->ringK, h->ringV, h->stream);
+  h->launches++;
+  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  return CONVKV_OK;
+}
+
+int convkv_attend(convkv_t* h, const void* q, void* out) {
+  if (!h || (!h->dry && (!q || !out))) return CONVKV_ERR_INVALID_ARG;
+  if (h->blocks < 1) return CONVKV_ERR_BAD_ORDER;
+  if (h->dry) return CONVKV_OK;
+  const int m = h->m(), w = h->w(), b = h->bcur, T = h->T;
+  AttnParams ap{};
+  ap.H = h->H;
+  ap.T = T;
+  ap.grid_w = h->gw;
+  ap.Nq = b * T;
+  ap.tq0 = m + w;
+  int tiles = 0;
+  auto add = [&](int buf, int frame0, int nframes, int t0) {
+    KeySeg& s = ap.seg[ap.nseg++];
+    s.buf = buf;
+    s.row0 = frame0 * T;
+    s.nrows = nframes * T;
+    s.t0 = t0;
+    s.tile0 = tiles;
+    tiles += (s.nrows + 127) / 128;
+  };
+  if (m > 0) {
+    const int pos0 = static_cast<int>((h->Sn - m) % h->C);
+    const int n1 = m < h->C - pos0 ? m : h->C - pos0;
+    add(1, pos0, n1, 0);
+    if (m > n1) add(1, 0, m - n1, n1);
+  }
+  {
+    const int n = w + b;
+    const int start = static_cast<int>(h->E % h->R);
+    const int n1 = n < h->R - start ? n : h->R - start;
+    add(0, start, n1, m);
+    if (n > n1) add(0, 0, n - n1, m + n1);
+  }
+  ap.ntiles = tiles;
+  ap.tab_t_rows = h->tab_t_rows;
+  ap.tab_h_rows = h->gh;
+  ap.tab_w_rows = h->gw;
+  ap.tables = h->tables;
+  ap.out = static_cast<__nv_bfloat16*>(out);
+  ap.q_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->D)));
+  ap.R = h->R;
+  ap.C = h->C;
+  ap.status = h->status;
+  CUtensorMap mq;
+  int rc = encode_4d(&mq, const_cast<void*>(q), h->D, h->H, ap.Nq, h->S);
+  if (rc) return rc;
+  CUtensorMap km[3] = {h->mapRingK, h->mapMemK, h->mapRingK};
+  CUtensorMap vm[3] = {h->mapRingV, h->mapMemV, h->mapRingV};
+  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->stream);
+  h->launches++;
+  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  return CONVKV_OK;
+}
+
+int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames) {
+  if (!h || !k_host || !v_host || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
+  if (!h->host_io || h->dry) return CONVKV_ERR_BAD_ORDER;
+  const size_t bytes = static_cast<size_t>(h->S) * frames * h->frame_elems() * 2;
+  cudaError_t e = cudaMemcpyAsync(h->io_k, k_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->io_v, v_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e);
+  return convkv_append_block(h, h->io_k, h->io_v, frames);
+}
+
+int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
+  if (!h || !q_host || !out_host) return CONVKV_ERR_INVALID_ARG;
+  if (!h->host_io || h->dry || h->blocks < 1) return CONVKV_ERR_BAD_ORDER;
+  const size_t bytes = static_cast<size_t>(h->S) * h->bcur * h->frame_elems() * 2;
+  cudaError_t e = cudaMemcpyAsync(h->io_q, q_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e);
+  int rc = convkv_attend(h, h->io_q, h->io_out);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, h->io_out, bytes, cudaMemcpyDeviceToHost, h->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e);
+  return CONVKV_OK;
+}
+
+int convkv_layout(const convkv_t* h, int32_t* rec, int cap) {
+  if (!h || (cap > 0 && !rec) || cap < 0) return CONVKV_ERR_INVALID_ARG;
+  const int m = h->m(), w = h->w(), b = h->bcur;
+  int n = 0;
+  auto put = [&](int part, int64_t src, int64_t phys, int t) {
+    if (n < cap) {
+      rec[4 * n + 0] = part;
+      rec[4 * n + 1] = static_cast<int32_t>(src);
+      rec[4 * n + 2] = static_cast<int32_t>(phys);
+      rec[4 * n + 3] = t;
+    }
+    ++n;
+  };
+  for (int i = 0; i < m; ++i) {
+    const int64_t k = h->Sn - m + i;
+    put(0, k, k % h->C, i);
+  }
+  for (int i = 0; i < w; ++i) put(1, h->E + i, (h->E + i) % h->R, m + i);
+  for (int f = 0; f < b; ++f) put(2, h->P + f, (h->P + f) % h->R, m + w + f);
+  return n;
+}
+
+int convkv_counters(const convkv_t* h, int64_t out[8]) {
+  if (!h || !out) return CONVKV_ERR_INVALID_ARG;
+  out[0] = h->P;
+  out[1] = h->E;
+  out[2] = h->Sn;
+  out[3] = h->m();
+  out[4] = h->w();
+  out[5] = h->bcur;
+  out[6] = h->blocks;
+  out[7] = h->last_groups;
+  return CONVKV_OK;
+}
+
+static int read_frame(const convkv_t* hc, const void* dev_base, int nslots, int state, int slot, void* host_dst) {
+  convkv_t* h = const_cast<convkv_t*>(hc);
+  const size_t fb = static_cast<size_t>(h->frame_elems()) * 2;
+  const char* src = static_cast<const char*>(dev_base) + (static_cast<size_t>(state) * nslots + slot) * fb;
+  cudaError_t e = cudaStreamSynchronize(h->stream);
+  if (e == cudaSuccess) e = cudaMemcpy(host_dst, src, fb, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return h->cuda_fail(e);
+  return CONVKV_OK;
+}
+
+int convkv_read_slot(const convkv_t* h, int state, int kv, int pos, void* host_dst, float* host_scales) {
+  (void)host_scales;
+  if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || pos < 0 || pos >= h->C)
+    return CONVKV_ERR_INVALID_ARG;
+  if (h->dry) return CONVKV_ERR_BAD_ORDER;
+  return read_frame(h, kv ? h->memV : h->memK, h->C, state, pos, host_dst);
+}
+
+int convkv_read_ring(const convkv_t* h, int state, int kv, int slot, void* host_dst, float* host_scales) {
+  (void)host_scales;
+  if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || slot < 0 || slot >= h->R)
+    return CONVKV_ERR_INVALID_ARG;
+  if (h->dry) return CONVKV_ERR_BAD_ORDER;
+  return read_frame(h, kv ? h->ringV : h->ringK, h->R, state, slot, host_dst);
+}
+
+int convkv_status(convkv_t* h) {
+  if (!h) return CONVKV_ERR_INVALID_ARG;
+  if (h->dry) return CONVKV_OK;
+  int st = 0;
+  cudaError_t e = cudaStreamSynchronize(h->stream);
+  if (e == cudaSuccess) e = cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && st != 0) e = cudaMemsetAsync(h->status, 0, sizeof(int), h->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e);
+  return st == kStatusOk ? CONVKV_OK : CONVKV_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Internal interface between the host library (convkv_host.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace ckv {
+
+constexpr int kEvict = 5;       // eviction group = conv kernel = conv stride (5:1)
+constexpr int kMaxSegs = 6;     // key segments of one attend (memory 2 + ring 2 + staging 1)
+constexpr int kMaxGroups = 16;  // eviction groups one append may compress
+
+// Device status word values (written by kernels, read by convkv_status()).
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 1;
+
+// One contiguous run of key rows in one buffer.
+struct KeySeg {
+  int buf;     // which K/V tensor maps: 0 ring, 1 memory, 2 fp8 current-block staging
+  int row0;    // first row (token) in that buffer, a frame boundary
+  int nrows;   // rows = frames * T
+  int t0;      // RoPE time index of the segment's first frame
+  int tile0;   // index of the segment's first 128-row key tile in the attend's tile list
+  int fp8;     // 1 if the rows are e4m3 with per-frame scales
+  int scale_slot0;  // fp8: slot index (ring slot or memory position) of the first frame
+  int scale_nslots; // fp8: slots in the scale array (R or C) for wrap-free indexing
+};
+
+struct AttnParams {
+  int H, T, grid_w, Nq;   // Nq = query rows per state (frames * T)
+  int tq0;                // RoPE time index of the current block's first frame (m + w)
+  int nseg, ntiles;
+  KeySeg seg[kMaxSegs];
+  int tab_t_rows, tab_h_rows, tab_w_rows;  // rows of the cos/sin tables
+  const float2* tables;   // [t rows][PT] ++ [grid_h][PH] ++ [grid_w][PW] (cos, sin)
+  __nv_bfloat16* out;     // [S][Nq][H][D]
+  float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
+  const float* ring_scale;  // fp8: [S][2][R][H]
+  const float* mem_scale;   // fp8: [S][2][C][H]
+  int R, C;
+  int* status;
+};
+
+struct ConvGroup {
+  int ring_slot[kEvict];  // physical ring slots of the 5 frames, oldest first
+  int mem_pos;            // destination memory position
+};
+
+struct ConvParams {
+  int H, T, S, C, R, ngroups;
+  ConvGroup grp[kMaxGroups];
+  void* memK;             // bf16 [S][C*T][H][D], or fp32 scratch in the fp8 format
+  void* memV;
+  int* status;
+};
+
+struct AppendParams {
+  int S, b, R, slot0;         // states, frames, ring frames, ring slot of frame 0
+  int64_t frame_elems;        // T * H * D
+};
+
+// Kernel launchers (return cudaError_t of the launch).
+int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
+                       cudaStream_t s);
+int launch_permute_weights(const void* src, void* dst, int S, int H, int D, cudaStream_t s);
+int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const CUtensorMap& ringV,
+                     const CUtensorMap& wmap, cudaStream_t s);
+int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s);
+int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k,
+                  const CUtensorMap* v, int S, cudaStream_t s);
+size_t attend_smem_bytes(int D, const AttnParams& p);
+size_t conv_smem_bytes(int D);
+
+}  // namespace ckv

@@ -1,0 +1,448 @@
+// Fused reset-RoPE attention of the current block over [memory | window | current].
+//
+// What it computes (SoulX-LiveAct): for each head and each query row of the
+// current block,
+//     o = sum_k softmax_k( <R(pos_q) q, R(pos_k) k> / sqrt(D) ) v_k
+// over every key of the memory slots, the window frames and the current block,
+// with no mask inside that set (blog walk-through, "Neighbor Forcing":
+// block-wise causal mask; "ConvKV Memory": the four-partition context), the
+// RoPE time index reset to run 0.. over memory, window, current (press
+// article and aiboss88.com summary: RoPE Reset), and the cached K kept
+// un-rotated, so the rotation is applied here, on the fly, tile by tile.
+//
+// CTA = one (state, head, 256 query rows) work unit, 16 warps:
+//   warp 0      TMA producer: Q (2 tiles of 128 rows), then K/V tiles of 128
+//               keys through a 2-stage ring, per key segment
+//   warp 1      tcgen05.mma issuer and TMEM owner: S_i = Q_i K^T (SS form),
+//               O_i += P_i V (P read from TMEM, TS form); tiles i = 0, 1 are
+//               interleaved so one tile's softmax overlaps the other's MMAs
+//   warps 4-7   softmax of query tile 0; warps 8-11 softmax of tile 1: one
+//               thread per query row; online softmax in fp32 registers with a
+//               lazily rescaled running max (the O rescale is only done when
+//               the max grows by more than 2^8); P written back over S as bf16,
+//               and the row sum taken over the same bf16 values the MMA uses
+//   warps 12-15 RoPE of each landed K tile, in place in shared memory
+// TMEM: S_0 | S_1 | O_0 | O_1 = 128 | 128 | D | D columns of 512.
+// Every barrier wait is bounded; on expiry the CTA raises an abort flag, skips
+// the remaining work, drains its outstanding copies and MMAs, frees TMEM and
+// records CONVKV_ERR_DEVICE_TIMEOUT in the status word.
+#include "convkv_internal.h"
+#include "sm100.cuh"
+
+namespace ckv {
+namespace {
+
+using namespace dev;
+
+template <int D>
+struct AttnCfg {
+  static constexpr int BM = 128, BN = 128, QT = 2, KST = 2, VST = 2;
+  static constexpr int NBOX = D / 64;
+  static constexpr int TILE = 128 * D * 2;     // bytes of one 128-row bf16 tile
+  static constexpr int BOX = 128 * 128;        // bytes of one 128-row x 64-channel box
+  static constexpr int PT = (D - 4 * (D / 6)) / 2;  // rotation pairs on the time axis
+  static constexpr int PH = D / 6;                  // ... on the row axis
+  static constexpr int PW = D / 6;                  // ... on the column axis
+  static constexpr int O_COL = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 512;
+  static constexpr int NBARS = 20;
+  static constexpr size_t FIXED = 1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16;
+};
+
+__device__ __forceinline__ int find_seg(const AttnParams& p, int j) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxSegs; ++i)
+    if (i < p.nseg && j >= p.seg[i].tile0) s = i;
+  return s;
+}
+
+// Rotate one 128-byte-swizzled row of a tile in place: adjacent channel pairs
+// (2i, 2i+1) of each axis segment [t | h | w] turn by the tabulated angle.
+// The swizzle permutes 16-byte chunks only, and a pair never straddles a
+// chunk, so the rotation is independent of it.
+template <int D, bool SCALE>
+__device__ __forceinline__ void rope_row(uint8_t* tile, int row, const float2* cs_t, const float2* cs_h,
+                                         const float2* cs_w, float scale) {
+  using C = AttnCfg<D>;
+  uint8_t* rowp = tile + row * 128;
+  const int sw = row & 7;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const int bx = c >> 3, cc = c & 7;
+    uint4* ptr = reinterpret_cast<uint4*>(rowp + bx * C::BOX + ((cc ^ sw) << 4));
+    const uint4 v = *ptr;
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int pi = 4 * c + q;
+      const float2 cs = pi < C::PT ? cs_t[pi] : (pi < C::PT + C::PH ? cs_h[pi - C::PT] : cs_w[pi - C::PT - C::PH]);
+      const float a = bf16lo_to_f32(w[q]), b = bf16hi_to_f32(w[q]);
+      float ra = a * cs.x - b * cs.y;
+      float rb = a * cs.y + b * cs.x;
+      if (SCALE) {
+        ra *= scale;
+        rb *= scale;
+      }
+      w[q] = pack_bf16x2(ra, rb);
+    }
+    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
+                const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
+                const __grid_constant__ CUtensorMap tmV1, const __grid_constant__ CUtensorMap tmK2,
+                const __grid_constant__ CUtensorMap tmV2, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = sQ + C::QT * C::TILE;
+  uint8_t* sV = sK + C::KST * C::TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::VST * C::TILE);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_ready = bars + 1;
+  uint64_t* k_full = bars + 2;    // [KST]
+  uint64_t* k_ready = bars + 4;   // [KST]
+  uint64_t* k_empty = bars + 6;   // [KST]
+  uint64_t* v_full = bars + 8;    // [VST]
+  uint64_t* v_empty = bars + 10;  // [VST]
+  uint64_t* s_full = bars + 12;   // [2]
+  uint64_t* p_full = bars + 14;   // [2]
+  uint64_t* o_full = bars + 16;   // [2]
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* tab = reinterpret_cast<float2*>(tmem_slot + 4);
+  const float2* tab_t = tab;
+  const float2* tab_h = tab_t + p.tab_t_rows * C::PT;
+  const float2* tab_w = tab_h + p.tab_h_rows * C::PH;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.y, state = blockIdx.z;
+  const int q_row0 = blockIdx.x * (C::QT * C::BM);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_ready, 2 * C::BM);
+    for (int i = 0; i < C::KST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_ready[i], C::BN);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < C::VST; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], C::BM);
+      mbar_init(&o_full[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  {
+    const int ntab = p.tab_t_rows * C::PT + p.tab_h_rows * C::PH + p.tab_w_rows * C::PW;
+    for (int i = threadIdx.x; i < ntab; i += blockDim.x) tab[i] = p.tables[i];
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const CUtensorMap* kmap[3] = {&tmK0, &tmK1, &tmK2};
+      const CUtensorMap* vmap[3] = {&tmV0, &tmV1, &tmV2};
+      tma_prefetch_desc(&tmQ);
+      mbar_expect_tx(q_full, C::QT * C::TILE);
+#pragma unroll
+      for (int i = 0; i < C::QT; ++i)
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sQ + i * C::TILE + bx * C::BOX, &tmQ, q_full, bx * 64, head, q_row0 + i * C::BM, state);
+      int kiss[C::KST] = {}, viss[C::VST] = {};
+      for (int j = 0; j < p.ntiles; ++j) {
+        const KeySeg& sg = p.seg[find_seg(p, j)];
+        const int row = sg.row0 + (j - sg.tile0) * C::BN;
+        const int ks = j % C::KST;
+        if (j >= C::KST && !mbar_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&k_full[ks], C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap[sg.buf], &k_full[ks], bx * 64, head, row, state);
+        ++kiss[ks];
+        const int vs = j % C::VST;
+        if (j >= C::VST && !mbar_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&v_full[vs], C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap[sg.buf], &v_full[vs], bx * 64, head, row, state);
+        ++viss[vs];
+      }
+      // drain: every issued copy must land before the CTA exits
+      volatile int no_abort = 0;
+      mbar_wait(q_full, 0, &no_abort);
+      for (int i = 0; i < C::KST; ++i)
+        if (kiss[i] > 0) mbar_wait(&k_full[i], (kiss[i] - 1) & 1, &no_abort);
+      for (int i = 0; i < C::VST; ++i)
+        if (viss[i] > 0) mbar_wait(&v_full[i], (viss[i] - 1) & 1, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, C::BN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      bool issued_any = false;
+      auto issue_s = [&](int i, int ks) {
+        const uint32_t a = q_addr + i * C::TILE, b = k_addr + ks * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+          mma_ss(tmem + i * 128, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc_qk,
+                 kk > 0);
+        }
+        issued_any = true;
+      };
+      auto issue_pv = [&](int i, int vs, bool acc) {
+        const uint32_t b = v_addr + vs * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          mma_ts(tmem + C::O_COL + i * D, tmem + i * 128 + kk * 8, sdesc_sw128(b + kk * 16 * 128, C::BOX, 1024),
+                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      do {
+        if (!mbar_wait(q_ready, 0, abort_flag)) break;
+        if (!mbar_wait(&k_ready[0], 0, abort_flag)) break;
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(&s_full[0]);
+        issue_s(1, 0);
+        tc_commit(&s_full[1]);
+        tc_commit(&k_empty[0]);
+        bool ok = true;
+        for (int j = 0; j < p.ntiles && ok; ++j) {
+          const int vs = j % C::VST;
+          if (!mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag)) { ok = false; break; }
+          const bool has_next = j + 1 < p.ntiles;
+          const int ksn = (j + 1) % C::KST;
+          for (int i = 0; i < 2; ++i) {
+            if (!mbar_wait(&p_full[i], j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(i, vs, j > 0);
+            if (i == 1) tc_commit(&v_empty[vs]);
+            if (has_next) {
+              if (i == 0) {
+                if (!mbar_wait(&k_ready[ksn], ((j + 1) / C::KST) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+              }
+              issue_s(i, ksn);
+              tc_commit(&s_full[i]);
+              if (i == 1) tc_commit(&k_empty[ksn]);
+            }
+          }
+        }
+        if (!ok) break;
+        tc_commit(&o_full[0]);
+        tc_commit(&o_full[1]);
+      } while (false);
+      if (issued_any) {
+        volatile int no_abort = 0;
+        tc_commit(drain);
+        mbar_wait(drain, 0, &no_abort);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ softmax
+    const int i = (warp - 4) >> 2;
+    const int lane_base = (warp & 3) * 32;
+    const int r = lane_base + lane;
+    const int qr = q_row0 + i * C::BM + r;
+    bool alive = mbar_wait(q_full, 0, abort_flag);
+    if (alive && qr < p.Nq) {
+      const int f = qr / p.T;
+      const int s = qr - f * p.T;
+      const int t = p.tq0 + f;
+      const int y = s / p.grid_w;
+      const int x = s - y * p.grid_w;
+      rope_row<D, true>(sQ + i * C::TILE, r, tab_t + t * C::PT, tab_h + y * C::PH, tab_w + x * C::PW, p.q_scale);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+
+    const uint32_t tS = tmem + (static_cast<uint32_t>(lane_base) << 16) + i * 128;
+    const uint32_t tO = tmem + (static_cast<uint32_t>(lane_base) << 16) + C::O_COL + i * D;
+    float m_run = -INFINITY, l_run = 0.0f;
+    for (int j = 0; j < p.ntiles; ++j) {
+      if (!mbar_wait_warp(&s_full[i], j & 1, abort_flag)) { alive = false; break; }
+      tc_fence_after();
+      const KeySeg& sg = p.seg[find_seg(p, j)];
+      const int valid = min(C::BN, sg.nrows - (j - sg.tile0) * C::BN);
+      // pass 1: row max over the valid columns
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_ld_wait();
+        if (valid >= (c + 1) * 32) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
+      }
+      const float m_new = fmaxf(m_run, mx);
+      if (j == 0) {
+        m_run = m_new;
+      } else {
+        const bool need = m_new > m_run + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          // O has no MMA in flight here: PV_i(j-1) completed before S_i(j) was committed
+          const float corr = need ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
+            tmem_st32(tO + c * 32, v);
+          }
+          if (need) {
+            l_run *= corr;
+            m_run = m_new;
+          }
+        }
+      }
+      // pass 2: P = exp2(S - m) as bf16, written over the first half of S's columns
+#pragma unroll
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+        if (valid >= (c + 1) * 32) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(__uint_as_float(v[2 * e]) - m_run);
+            const float p1 = fast_exp2(__uint_as_float(v[2 * e + 1]) - m_run);
+            pk[e] = pack_bf16x2(p0, p1);
+            l_run += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = (c * 32 + 2 * e < valid) ? fast_exp2(__uint_as_float(v[2 * e]) - m_run) : 0.0f;
+            const float p1 = (c * 32 + 2 * e + 1 < valid) ? fast_exp2(__uint_as_float(v[2 * e + 1]) - m_run) : 0.0f;
+            pk[e] = pack_bf16x2(p0, p1);
+            l_run += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
+          }
+        }
+        tmem_st16(tS + c * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[i]);
+    }
+    // epilogue: O / l -> bf16 -> out
+    if (alive && mbar_wait_warp(&o_full[i], 0, abort_flag)) {
+      tc_fence_after();
+      const float inv = 1.0f / l_run;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + ((static_cast<int64_t>(state) * p.Nq + qr) * p.H + head) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + c * 32, v);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+        if (qr < p.Nq) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[c * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ K RoPE
+    const int r = threadIdx.x - 384;
+    for (int j = 0; j < p.ntiles; ++j) {
+      const int ks = j % C::KST;
+      if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
+      const KeySeg& sg = p.seg[find_seg(p, j)];
+      const int off = (j - sg.tile0) * C::BN;
+      if (off + r < sg.nrows) {
+        const int lr = off + r;
+        const int f = lr / p.T;
+        const int s = lr - f * p.T;
+        const int t = sg.t0 + f;
+        const int y = s / p.grid_w;
+        const int x = s - y * p.grid_w;
+        rope_row<D, false>(sK + ks * C::TILE, r, tab_t + t * C::PT, tab_h + y * C::PH, tab_w + x * C::PW, 1.0f);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&k_ready[ks]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, kStatusTimeout);
+}
+
+template <int D>
+size_t smem_for(const AttnParams& p) {
+  using C = AttnCfg<D>;
+  const size_t ntab = static_cast<size_t>(p.tab_t_rows) * C::PT + static_cast<size_t>(p.tab_h_rows) * C::PH +
+                      static_cast<size_t>(p.tab_w_rows) * C::PW;
+  const size_t need = C::FIXED + ntab * sizeof(float2);
+  // at least half the SM's shared memory: one CTA per SM, so the 512-column
+  // TMEM allocation never has to wait for a co-resident CTA
+  return need > 120 * 1024 ? need : 120 * 1024;
+}
+
+template <int D>
+int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v, int S,
+             cudaStream_t s) {
+  const size_t smem = smem_for<D>(p);
+  auto kern = attn_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  dim3 grid((p.Nq + 255) / 256, p.H, S);
+  kern<<<grid, AttnCfg<D>::THREADS, smem, s>>>(q, k[0], v[0], k[1], v[1], k[2], v[2], p);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+size_t attend_smem_bytes(int D, const AttnParams& p) { return D == 128 ? smem_for<128>(p) : smem_for<64>(p); }
+
+int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v,
+                  int S, cudaStream_t s) {
+  if (D == 128) return launch_t<128>(p, q, k, v, S, s);
+  if (D == 64) return launch_t<64>(p, q, k, v, S, s);
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+}  // namespace ckv

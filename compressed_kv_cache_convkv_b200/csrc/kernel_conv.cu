@@ -1,0 +1,192 @@
+// Conv compression of evicted frames on the 5th-generation tensor cores.
+//
+// SoulX-LiveAct blog walk-through, section "ConvKV Memory": old KV is
+// compressed by a lightweight 1D convolution into a fixed-length memory; the
+// aiboss88.com summary (ConvKV Memory bullet) gives the 5:1 ratio.  Per head h,
+// for one group of 5 evicted frames x_0..x_4 (oldest first):
+//     out[s, o] = sum_{j<5} sum_{i<D} W[h, o, i, j] * x_j[s, i]
+// i.e. one GEMM per (group, K|V, head): [T x 5D] . [5D x D], accumulated in
+// fp32 in tensor memory and rounded to bf16 into the memory slot.
+//
+// One CTA computes a 128-token x D tile: five k-blocks (one per evicted frame),
+// each a TMA box of the frame's rows for this head (ring slots may wrap; each
+// k-block is its own load, so wrap costs nothing) and the matching D x D
+// weight block.  Warp 0 issues TMA, warp 1 issues tcgen05.mma (M=128, N=D,
+// K=16 steps) and owns the TMEM accumulator, warps 2-5 drain it.
+#include "convkv_internal.h"
+#include "sm100.cuh"
+
+namespace ckv {
+namespace {
+
+using namespace dev;
+
+template <int D>
+struct ConvCfg {
+  static constexpr int BM = 128;
+  static constexpr int STAGES = 3;
+  static constexpr int NBOX = D / 64;                // 64-channel (128-byte) boxes per row
+  static constexpr int A_BYTES = BM * D * 2;         // token rows x input channels
+  static constexpr int B_BYTES = D * D * 2;          // output channels x input channels
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = D < 32 ? 32 : D;
+  static constexpr int THREADS = 192;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
+    conv_bf16_kernel(const __grid_constant__ CUtensorMap tmRingK, const __grid_constant__ CUtensorMap tmRingV,
+                     const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
+  using C = ConvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = base;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES]
+  uint64_t* empty = bars + C::STAGES;    // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x, head = blockIdx.y;
+  const int kv = blockIdx.z & 1;
+  const int sg = blockIdx.z >> 1;
+  const int state = sg % p.S;
+  const int g = sg / p.S;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const CUtensorMap* ring = kv ? &tmRingV : &tmRingK;
+      tma_prefetch_desc(ring);
+      tma_prefetch_desc(&tmW);
+      int issued[C::STAGES] = {};
+      for (int j = 0; j < kEvict; ++j) {
+        const int st = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(&empty[st], ((j / C::STAGES) - 1) & 1, abort_flag)) break;
+        uint8_t* a = stages + st * C::STAGE_BYTES;
+        uint8_t* b = a + C::A_BYTES;
+        mbar_expect_tx(&full[st], C::STAGE_BYTES);
+        const int row = p.grp[g].ring_slot[j] * p.T + mt * C::BM;
+        const int wrow = ((kv * p.H + head) * kEvict + j) * D;
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_4d(a + bx * (C::BM * 128), ring, &full[st], bx * 64, head, row, state);
+          tma_load_3d(b + bx * (D * 128), &tmW, &full[st], bx * 64, wrow, state);
+        }
+        ++issued[st];
+      }
+      // drain: every load issued must have landed before the CTA may exit
+      for (int st = 0; st < C::STAGES; ++st) {
+        if (issued[st] > 0) {
+          volatile int no_abort = 0;
+          mbar_wait(&full[st], (issued[st] - 1) & 1, &no_abort);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, D, false, false);
+      bool any = false;
+      for (int j = 0; j < kEvict; ++j) {
+        const int st = j % C::STAGES;
+        if (!mbar_wait(&full[st], (j / C::STAGES) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(stages + st * C::STAGE_BYTES);
+        const uint32_t b = a + C::A_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks & 3) * 32;
+          const uint64_t ad = sdesc_sw128(a + (ks >> 2) * (C::BM * 128) + koff, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b + (ks >> 2) * (D * 128) + koff, 16, 1024);
+          mma_ss(tmem, ad, bd, idesc, (j | ks) != 0);
+        }
+        any = true;
+        tc_commit(&empty[st]);
+      }
+      tc_commit(acc_full);
+      if (any) {
+        volatile int no_abort = 0;
+        tc_commit(drain);
+        mbar_wait(drain, 0, &no_abort);
+      }
+    }
+  } else {
+    // epilogue: warps 2..5 -> TMEM lanes 32*(warp%4) .. +31
+    const int lane_base = (warp & 3) * 32;
+    const int r = lane_base + lane;
+    const int token = mt * C::BM + r;
+    if (mbar_wait_warp(acc_full, 0, abort_flag)) {
+      tc_fence_after();
+      __nv_bfloat16* dst_base = static_cast<__nv_bfloat16*>(kv ? p.memV : p.memK);
+      const int64_t row = (static_cast<int64_t>(state) * p.C + p.grp[g].mem_pos) * p.T + token;
+      uint4* dst = reinterpret_cast<uint4*>(dst_base + (row * p.H + head) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        if (token < p.T) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[c * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, kStatusTimeout);
+}
+
+}  // namespace
+
+size_t conv_smem_bytes(int D) { return D == 128 ? ConvCfg<128>::SMEM : ConvCfg<64>::SMEM; }
+
+int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const CUtensorMap& ringV,
+                     const CUtensorMap& wmap, cudaStream_t s) {
+  if (p.ngroups <= 0) return 0;
+  dim3 grid((p.T + 127) / 128, p.H, p.ngroups * p.S * 2);
+  if (D == 128) {
+    auto k = conv_bf16_kernel<128>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<128>::SMEM);
+    k<<<grid, ConvCfg<128>::THREADS, ConvCfg<128>::SMEM, s>>>(ringK, ringV, wmap, p);
+  } else if (D == 64) {
+    auto k = conv_bf16_kernel<64>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<64>::SMEM);
+    k<<<grid, ConvCfg<64>::THREADS, ConvCfg<64>::SMEM, s>>>(ringK, ringV, wmap, p);
+  } else {
+    return static_cast<int>(cudaErrorInvalidValue);
+  }
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace ckv

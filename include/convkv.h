@@ -1,0 +1,164 @@
+/*
+ * convkv.h -- C ABI of the ConvKV Memory attention step for NVIDIA B200 (sm_100a).
+ *
+ * The method (SoulX-LiveAct):
+ *   - blog walk-through (gongshangzheng.github.io/paper-liveact.html), section
+ *     "ConvKV Memory": recent KV is kept exact, older KV is compressed by a
+ *     lightweight 1D convolution into a fixed-length long-term memory; the
+ *     context is [long-term memory | short-term window | current block]; cached
+ *     KV is append-only and compression starts with the third block;
+ *   - same page, section "Streaming Pipeline": the conv runs once between
+ *     blocks, and the KV footprint is the same for any stream length;
+ *   - same page, section "Neighbor Forcing": block-wise causal mask (the current
+ *     block sees all history and all of itself);
+ *   - digi.china.com press article: RoPE Reset re-aligns position encoding;
+ *     aiboss88.com summary, ConvKV Memory bullet: 1D conv at a 5:1 ratio, RoPE
+ *     position encoding reset;
+ *   - model card (hf.xjtesla.cn/Soul-AILab/LiveAct), Command Line Arguments
+ *     table, --fp8_kv_cache: KV stored in FP8, dequantised to BF16 on use.
+ *
+ * One handle holds the KV cache of `num_states` independent layer/denoising-
+ * step states that advance in lock step (same block sizes).  Per block the
+ * caller makes one convkv_append_block() and then one convkv_attend().
+ *
+ * Tensor layout of every q, k, v, out buffer (bf16, row-major, contiguous):
+ *     [num_states][frames * T][heads][head_dim]
+ * where T = grid_h * grid_w tokens per latent frame and token s of a frame sits
+ * at spatial position (row, col) = (s / grid_w, s % grid_w).
+ *
+ * Errors: every call returns 0 (CONVKV_OK) or a negative CONVKV_ERR_* code.
+ * A call that fails validation leaves the state unchanged.  Nothing is thrown
+ * across the ABI.  A handle is not thread-safe; all its device work is ordered
+ * on the stream given at create.
+ */
+#ifndef CONVKV_H
+#define CONVKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CONVKV_OK 0
+#define CONVKV_ERR_INVALID_ARG (-1)    /* null pointer, size out of range, bad config */
+#define CONVKV_ERR_UNSUPPORTED (-2)    /* valid but not implemented (e.g. evict_frames != 5) */
+#define CONVKV_ERR_BAD_ORDER (-3)      /* attend before any append; handle in dry-run mode */
+#define CONVKV_ERR_OOM (-4)            /* device allocation failed at create */
+#define CONVKV_ERR_CUDA (-5)           /* a CUDA runtime/driver call failed; see convkv_last_cuda_error */
+#define CONVKV_ERR_DEVICE_TIMEOUT (-6) /* a kernel gave up waiting on a barrier and returned early */
+
+#define CONVKV_KV_BF16 0               /* cache stored in bf16 */
+#define CONVKV_KV_FP8_E4M3 1           /* window + memory stored e4m3 with per-(head, frame) fp32 scale */
+
+#define CONVKV_COMPRESS_CONV 0         /* 1D conv, kernel 5, stride 5 (the method) */
+#define CONVKV_COMPRESS_MEAN 1         /* mean of the 5 evicted frames (--mean_memory option) */
+
+#define CONVKV_FLAG_DRY_RUN 1          /* bookkeeping only: no device memory, no kernel launches */
+#define CONVKV_FLAG_HOST_IO 2          /* also allocate device staging for the *_host entry points */
+
+/* Configuration.  All sizes are positive unless stated. */
+typedef struct convkv_cfg {
+  int heads;               /* H */
+  int head_dim;            /* D: 64 or 128 */
+  int grid_h, grid_w;      /* tokens per latent frame T = grid_h * grid_w (each <= 255) */
+  int first_block_frames;  /* b1: frames of the first block */
+  int block_frames;        /* b : frames of later blocks; any append may carry 1..max(b1, b) frames */
+  int window_frames;       /* W >= 4: past-block frames kept exact */
+  int evict_frames;        /* must be 5 (conv kernel = stride = eviction group) */
+  int mem_slots;           /* C >= 1: FIFO capacity of compressed slots */
+  int rope_t, rope_h, rope_w; /* RoPE channels per axis (even, sum = D); all 0 -> D-4*floor(D/6), 2*floor(D/6), 2*floor(D/6) */
+  double rope_theta;       /* RoPE base, e.g. 1e4 */
+  int kv_format;           /* CONVKV_KV_BF16 or CONVKV_KV_FP8_E4M3 */
+  int compress_mode;       /* CONVKV_COMPRESS_CONV or CONVKV_COMPRESS_MEAN */
+  int num_states;          /* independent states advanced together (>= 1) */
+  int flags;               /* CONVKV_FLAG_* */
+  int t_offset;            /* added to every RoPE time index (outputs must not depend on it); normally 0 */
+  const void* conv_weight; /* device bf16 [num_states][2 (K,V)][H][D_out][D_in][5]; read once at create,
+                              not retained; may be NULL for CONVKV_COMPRESS_MEAN or dry-run */
+  void* stream;            /* cudaStream_t for all device work of this handle (NULL = legacy default) */
+} convkv_cfg;
+
+typedef struct convkv convkv_t;
+
+/* Validate cfg, allocate the whole device state in one arena (zero-filled),
+ * build the RoPE tables, and permute the conv weights into the kernel layout.
+ * No device memory is allocated after this call.  *out receives the handle.
+ * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
+int convkv_create(const convkv_cfg* cfg, convkv_t** out);
+
+/* Append one block (SoulX-LiveAct blog, "ConvKV Memory" / "Streaming Pipeline"):
+ *   1. the previous current block joins the window;
+ *   2. while the window holds more than W frames, its oldest 5 frames are
+ *      compressed into one memory slot (FIFO of C slots, oldest dropped);
+ *   3. k, v become the current block (copied into the ring; e4m3 + scale in the
+ *      fp8 format, with a bf16 copy kept for this block's attend).
+ * k, v: DEVICE pointers, [num_states][frames*T][H][D] bf16; the copy is
+ * asynchronous on the handle's stream, so keep them unchanged until it passes.
+ * frames: 1 .. max(b1, b).  Errors: INVALID_ARG, BAD_ORDER (dry-run with
+ * non-null pointers is fine), CUDA. */
+int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames);
+
+/* Attention of the current block's queries over [memory | window | current]
+ * with RoPE time indices reset to start at 0 (memory slot i -> i, window frame
+ * j -> m + j, current frame f -> m + w + f), spatial indices unchanged,
+ * softmax scale 1/sqrt(D), no mask inside the attended set.
+ * q, out: DEVICE pointers, [num_states][frames*T][H][D] bf16 with `frames` of
+ * the last append.  Does not change the state (may be repeated).
+ * Errors: INVALID_ARG, BAD_ORDER, CUDA. */
+int convkv_attend(convkv_t* h, const void* q, void* out);
+
+/* Same as append_block / attend but with HOST buffers (pinned or pageable):
+ * the inputs are copied into handle-owned device staging, the output is copied
+ * back, and the call returns after the copy back completed.  Needs
+ * CONVKV_FLAG_HOST_IO at create.  Errors: as above, plus BAD_ORDER without the flag. */
+int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames);
+int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host);
+
+/* Device bytes owned by the handle; constant from create to destroy. */
+size_t convkv_state_bytes(const convkv_t* h);
+
+/* Release everything the handle owns (waits for its stream).  NULL is a no-op. */
+void convkv_destroy(convkv_t* h);
+
+/* Key-frame layout of the next attend, in attended order, 4 int32 per frame:
+ * {partition (0 memory, 1 window, 2 current), source index (slot index for
+ * memory -- slot k covers stream frames [5k, 5k+5) -- else stream frame index),
+ * physical slot (memory position, ring slot, or staging slot for the fp8
+ * current block), RoPE time index}.  Returns the number of key frames, or a
+ * negative error; writes at most `cap` records. */
+int convkv_layout(const convkv_t* h, int32_t* rec, int cap);
+
+/* Counters {P promoted frames, E evicted frames, S slots produced, m stored
+ * slots, w window frames, b current frames, blocks appended, groups compressed
+ * by the last append}.  Returns 0 or INVALID_ARG. */
+int convkv_counters(const convkv_t* h, int64_t out[8]);
+
+/* Copy one stored memory slot (memory position `pos` in [0, C)) of one state
+ * and one of K (kv = 0) or V (kv = 1) to host memory: [T][H][D] bf16, or e4m3
+ * bytes in the fp8 format with scales[H] fp32 written to host_scales (may be
+ * NULL for bf16).  Synchronises the stream.  Errors: INVALID_ARG, BAD_ORDER, CUDA. */
+int convkv_read_slot(const convkv_t* h, int state, int kv, int pos, void* host_dst, float* host_scales);
+
+/* Copy one ring frame slot (`slot` in [0, W + max(b1, b))) the same way. */
+int convkv_read_ring(const convkv_t* h, int state, int kv, int slot, void* host_dst, float* host_scales);
+
+/* Synchronise the stream, return CONVKV_OK or the first error recorded by a
+ * kernel (DEVICE_TIMEOUT), and clear the device status word. */
+int convkv_status(convkv_t* h);
+
+/* Number of kernels this handle has launched so far. */
+int64_t convkv_launch_count(const convkv_t* h);
+
+/* cudaError_t of the last failing CUDA call made through this handle (0 if none). */
+int convkv_last_cuda_error(const convkv_t* h);
+
+/* Static description of an error code. */
+const char* convkv_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVKV_H */

@@ -130,29 +130,44 @@ def rope_split(D: int) -> Tuple[int, int, int]:
     return D - 2 * dh, dh, dh
 
 
+def rope_angles(t: np.ndarray, y: np.ndarray, xc: np.ndarray, split: Tuple[int, int, int],
+                theta: float) -> np.ndarray:
+    """Rotation angle of every channel pair at positions (t, y, xc): [..., D/2].
+
+    Pairs [0, d_t/2) follow the time index, the next d_h/2 the row index, the
+    rest the column index; pair i of an axis segment of width d turns by
+    pos * theta^(-2i/d).
+    """
+    parts = []
+    for width, pos in zip(split, (t, y, xc)):
+        i = np.arange(width // 2, dtype=np.float64)
+        freq = theta ** (-2.0 * i / width)
+        parts.append(np.asarray(pos, dtype=np.float64)[..., None] * freq)
+    shape = np.broadcast_shapes(*[p.shape[:-1] for p in parts])
+    return np.concatenate([np.broadcast_to(p, shape + p.shape[-1:]) for p in parts], axis=-1)
+
+
+def rope_apply(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Turn each adjacent channel pair (2i, 2i+1) of x[..., D] by the angle whose
+    cosine and sine are cos[..., i], sin[..., i]: (a, b) -> (a cos - b sin, a sin + b cos)."""
+    x = np.asarray(x, dtype=np.float64)
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, cos.shape[:-1] + (x.shape[-1],)))
+    out[..., 0::2] = a * cos - b * sin
+    out[..., 1::2] = a * sin + b * cos
+    return out
+
+
 def rope_rotate(x: np.ndarray, t: np.ndarray, y: np.ndarray, xc: np.ndarray,
                 split: Tuple[int, int, int], theta: float) -> np.ndarray:
     """Rotate x[..., D] by 3D RoPE at positions (t, y, xc) (broadcast over x[..., 0]).
 
     Channels [0, d_t) use the time index, [d_t, d_t+d_h) the row index and the
     rest the column index.  Inside an axis segment of width d, pair i (channels
-    2i, 2i+1 of the segment) turns by angle pos * theta^(-2i/d):
-    (a, b) -> (a cos - b sin, a sin + b cos).
+    2i, 2i+1 of the segment) turns by angle pos * theta^(-2i/d).
     """
-    x = np.asarray(x, dtype=np.float64)
-    out = np.empty_like(x)
-    start = 0
-    for width, pos in zip(split, (t, y, xc)):
-        i = np.arange(width // 2, dtype=np.float64)
-        freq = theta ** (-2.0 * i / width)
-        ang = np.asarray(pos, dtype=np.float64)[..., None] * freq
-        c, s = np.cos(ang), np.sin(ang)
-        a = x[..., start:start + width:2]
-        b = x[..., start + 1:start + width:2]
-        out[..., start:start + width:2] = a * c - b * s
-        out[..., start + 1:start + width:2] = a * s + b * c
-        start += width
-    return out
+    ang = rope_angles(t, y, xc, split, theta)
+    return rope_apply(x, np.cos(ang), np.sin(ang))
 
 
 # --------------------------------------------------------------------------
@@ -164,12 +179,19 @@ def conv_compress(group: np.ndarray, w: np.ndarray) -> np.ndarray:
 
     out[s, h, o] = sum_j sum_i w[h, o, i, j] * group[j, s, h, i]
     (per-head channel mixing, kernel 5 = stride 5 over time, no padding,
-    no bias, tap j = j-th oldest frame).
+    no bias, tap j = j-th oldest frame).  Per head this is one matrix product
+    over the combined (j, i) index: [T x 5D] . [5D x D].
     """
     g = np.asarray(group, dtype=np.float64)
     wf = np.asarray(w, dtype=np.float64)
     assert g.shape[0] == EVICT and wf.shape[-1] == EVICT
-    return np.einsum("hoij,jshi->sho", wf, g, optimize=True)
+    n, T, H, D = g.shape
+    out = np.empty((T, H, wf.shape[1]))
+    for h in range(H):
+        x = g[:, :, h, :].transpose(1, 0, 2).reshape(T, EVICT * D)      # [s, (j, i)]
+        wt = wf[h].transpose(2, 1, 0).reshape(EVICT * D, wf.shape[1])   # [(j, i), o]
+        out[:, h, :] = x @ wt
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -354,12 +376,14 @@ class OracleStream:
         split = cfg.rope()
         o = np.zeros((len(rows), len(heads), D))
         psum = np.zeros((len(rows), len(heads)))
+        k_ang = rope_angles(k_t, k_y, k_x, split, cfg.theta)             # [Nk, D/2], shared by all heads
+        q_ang = rope_angles(q_t, q_y, q_x, split, cfg.theta)             # [n, D/2]
+        kc, ks, qc, qs_ = np.cos(k_ang), np.sin(k_ang), np.cos(q_ang), np.sin(q_ang)
         for hi, h in enumerate(heads):
             kh = np.concatenate([f.k[:, h, :] for _, f, _ in kf])
             vh = np.concatenate([f.v[:, h, :] for _, f, _ in kf])
-            k_rot = rope_rotate(kh, k_t, k_y, k_x, split, cfg.theta)
-            q_rows = np.asarray(q[qf, qs, h, :], dtype=np.float64)
-            q_rot = rope_rotate(q_rows, q_t, q_y, q_x, split, cfg.theta)
+            k_rot = rope_apply(kh, kc, ks)
+            q_rot = rope_apply(np.asarray(q[qf, qs, h, :], dtype=np.float64), qc, qs_)
             o[:, hi, :], psum[:, hi] = attend_rows(q_rot, k_rot, vh)
         return o, psum
 

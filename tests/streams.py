@@ -1,0 +1,113 @@
+"""Drive one workload through the CUDA path and the oracle on the same seeded inputs.
+
+Inputs for block n are frames [F_n, F_n + b_n) of the seeded Q, K, V tensors
+(SoulX-style streams: stream frame index = latent frame index), generated on
+the device for the CUDA path and on the host for the oracle, bit-identical.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterator, Optional, Sequence
+
+import numpy as np
+
+import seeded_inputs as si
+from oracle import convkv_oracle as O
+
+# tolerances (spec bounds; relative form for compressed K/V of magnitude > 1,
+# plus a relative-L2 gate on attention outputs whose magnitude is ~1e-2)
+ATT_MAX, ATT_MEAN, ATT_REL_L2 = 1e-2, 1e-3, 1e-2
+SLOT_MAX_REL, SLOT_MEAN = 1e-2, 1e-3
+FP8_MAX = 5e-2
+
+
+def oracle_for(w, state: int = 0, conv_w: Optional[np.ndarray] = None, mean: bool = False) -> O.OracleStream:
+    cfg = O.OracleConfig(H=w.heads, D=w.head_dim, grid_h=w.grid_h, grid_w=w.grid_w, window=w.window_frames,
+                         mem_slots=w.mem_slots, fp8=w.fp8)
+    if mean:
+        wts = np.zeros((2, w.heads, w.head_dim, w.head_dim, 5))
+        for o in range(w.head_dim):
+            wts[:, :, o, o, :] = 0.2
+    else:
+        wts = si.bf16_bits_to_f64(conv_w if conv_w is not None else si.conv_weights(w.seed, state, w.heads, w.head_dim))
+    return O.OracleStream(cfg, wts)
+
+
+def host_frames(w, tensor: int, state: int, frame0: int, nframes: int) -> np.ndarray:
+    bits = si.frames(w.seed, tensor, state, frame0, nframes, w.T * w.heads * w.head_dim)
+    return bits.reshape(nframes, w.T, w.heads, w.head_dim)
+
+
+def device_frames(w, tensor: int, frame0: int, nframes: int, torch_mod, out=None):
+    """[S, nframes*T, H, D] bf16 CUDA tensor of the seeded values (all states)."""
+    torch = torch_mod
+    S = w.num_states
+    fe = w.T * w.heads * w.head_dim
+    if out is None:
+        out = torch.empty((S, nframes * w.T, w.heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for s in range(S):
+        si.frames_device(out[s].data_ptr(), w.seed, tensor, s, frame0, nframes, fe, 1.0, stream)
+    return out
+
+
+def device_weights(w, torch_mod, states: Optional[Sequence[int]] = None):
+    torch = torch_mod
+    S = w.num_states
+    n = w.heads * w.head_dim * w.head_dim * 5
+    out = torch.empty((S, 2, w.heads, w.head_dim, w.head_dim, 5), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for s in range(S):
+        for kv, tid in ((0, si.WK), (1, si.WV)):
+            si.frames_device(out[s, kv].data_ptr(), w.seed, tid, s, 0, 1, n, si.weight_scale(w.head_dim), stream)
+    return out
+
+
+def bf16_tensor_to_f64(t) -> np.ndarray:
+    import torch
+    return si.bf16_bits_to_f64(t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def sample_rows(w, b: int, n: int, rng: np.random.Generator) -> np.ndarray:
+    """Query rows to check: first/last rows, the ragged tail of the last 128-row tile, random rest."""
+    Nq = b * w.T
+    if n >= Nq:
+        return np.arange(Nq)
+    fixed = {0, 1, Nq - 1, Nq - 2, w.T - 1, w.T}
+    tail0 = (Nq // 128) * 128
+    fixed |= set(range(tail0, min(Nq, tail0 + 4)))
+    fixed |= {r for r in range(127, Nq, 128)}
+    fixed = sorted(x for x in fixed if 0 <= x < Nq)[: n // 2]
+    rest = rng.choice(Nq, size=n - len(fixed), replace=False)
+    return np.unique(np.concatenate([np.array(fixed, dtype=np.int64), rest]))
+
+
+def attention_errors(gpu: np.ndarray, ref: np.ndarray) -> dict:
+    d = np.abs(gpu - ref)
+    return {"max": float(d.max()), "mean": float(d.mean()),
+            "rel_l2": float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-300))}
+
+
+# Sharp-softmax variant (queries x8, outputs of order 1): the bf16 rounding of the
+# rotated operands (relative 2^-9 each) moves a logit of size ~8 by ~0.03, i.e. a few
+# percent on the weights of competing keys, so the absolute bound scales with it.
+SHARP_MAX, SHARP_MEAN = 6e-2, 5e-3
+
+
+def check_attention(gpu: np.ndarray, ref: np.ndarray, fp8: bool = False, what: str = "", sharp: bool = False) -> dict:
+    e = attention_errors(gpu, ref)
+    if sharp:
+        assert e["max"] <= SHARP_MAX and e["mean"] <= SHARP_MEAN and e["rel_l2"] <= ATT_REL_L2, (what, e)
+    elif fp8:
+        assert e["max"] <= FP8_MAX and e["rel_l2"] <= 5 * ATT_REL_L2, (what, e)
+    else:
+        assert e["max"] <= ATT_MAX and e["mean"] <= ATT_MEAN and e["rel_l2"] <= ATT_REL_L2, (what, e)
+    return e
+
+
+def check_slot(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
+    d = np.abs(gpu - ref)
+    rel = d / np.maximum(1.0, np.abs(ref))
+    e = {"max_rel": float(rel.max()), "mean": float(d.mean())}
+    assert e["max_rel"] <= SLOT_MAX_REL and e["mean"] <= SLOT_MEAN, (what, e)
+    return e

@@ -1,0 +1,137 @@
+"""C-ABI library on the host (no GPU): exports, argument checks, bookkeeping.
+
+The library's integer bookkeeping (dry-run handles allocate no device memory
+and launch nothing) must agree bit for bit with the oracle's stream state and
+with the closed form of the eviction rule, for every block of every workload.
+"""
+import ctypes
+import math
+import re
+
+import numpy as np
+import pytest
+
+import compressed_kv_cache_convkv_b200 as ckv
+from compressed_kv_cache_convkv_b200.configs import PRESETS
+from oracle import convkv_oracle as O
+
+
+def _header_functions():
+    import os
+    text = open(os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "convkv.h")).read()
+    return sorted(set(re.findall(r"^[\w\s\*]*?\b(convkv_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ckv.library()
+    names = _header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(ckv._SIGNATURES), "binding is missing a declared function"
+
+
+def test_strerror():
+    lib = ckv.library()
+    assert lib.convkv_strerror(0) == b"ok"
+    assert lib.convkv_strerror(ckv.ERR_DEVICE_TIMEOUT) == b"device wait timed out"
+
+
+def _dry(w, **kw):
+    return ckv.ConvKV(w.config(dry_run=True, **kw))
+
+
+def test_invalid_configs_rejected():
+    base = PRESETS["tiny"].config(dry_run=True)
+    bad = [
+        (base.with_(window_frames=3), ckv.ERR_INVALID_ARG),
+        (base.with_(mem_slots=0), ckv.ERR_INVALID_ARG),
+        (base.with_(evict_frames=4), ckv.ERR_UNSUPPORTED),
+        (base.with_(head_dim=96), ckv.ERR_UNSUPPORTED),
+        (base.with_(rope=(20, 22, 22)), ckv.ERR_UNSUPPORTED),
+        (base.with_(num_states=0), ckv.ERR_INVALID_ARG),
+        (base.with_(rope_theta=0.0), ckv.ERR_INVALID_ARG),
+        (base.with_(grid_h=4096, grid_w=4096), ckv.ERR_UNSUPPORTED),
+    ]
+    for cfg, code in bad:
+        with pytest.raises(ckv.ConvKVError) as e:
+            ckv.ConvKV(cfg)
+        assert e.value.code == code, cfg
+    # a real (non dry-run) conv handle needs weights; rejected before any CUDA call
+    lib = ckv.library()
+    assert lib.convkv_create(None, None) == ckv.ERR_INVALID_ARG
+    c = PRESETS["tiny"].config()._c(0, 0)
+    out = ctypes.c_void_p()
+    assert lib.convkv_create(ctypes.byref(c), ctypes.byref(out)) == ckv.ERR_INVALID_ARG and not out
+
+
+def test_call_order_and_argument_checks():
+    h = _dry(PRESETS["tiny"])
+    lib = ckv.library()
+    assert lib.convkv_attend(h._h, None, None) == ckv.ERR_BAD_ORDER
+    assert lib.convkv_append_block(h._h, None, None, 0) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_append_block(h._h, None, None, 3) == ckv.ERR_INVALID_ARG  # > max block
+    c0 = h.counters()
+    assert lib.convkv_append_block(h._h, None, None, 3) == ckv.ERR_INVALID_ARG
+    assert h.counters() == c0, "a rejected call must leave the state unchanged"
+    h.dry_append(2)
+    assert lib.convkv_attend(h._h, None, None) == ckv.OK
+    assert lib.convkv_read_slot(h._h, 0, 0, 0, None, None) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_append_block_host(h._h, None, None, 2) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_state_bytes(h._h) == 0 and h.launch_count() == 0
+    lib.convkv_destroy(None)
+
+
+def _oracle_layout(st):
+    return [(int(p), int(s), int(t)) for p, s, t in st.layout()]
+
+
+@pytest.mark.parametrize("name", ["tiny", "512x512", "720x416", "fp8_480x832"])
+def test_bookkeeping_matches_oracle_every_block(name):
+    w = PRESETS[name]
+    h = _dry(w)
+    cfg = O.OracleConfig(H=1, D=6, grid_h=1, grid_w=1, window=w.window_frames, mem_slots=w.mem_slots)
+    st = O.OracleStream(cfg, np.zeros((2, 1, 6, 6, 5)))
+    R = w.window_frames + max(w.first_block_frames, w.block_frames)
+    for n, b in enumerate(w.block_sizes()):
+        h.dry_append(b)
+        ev = st.append(np.zeros((b, 1, 1, 6)), np.zeros((b, 1, 1, 6)))
+        c = h.counters()
+        assert (c["P"], c["E"], c["S"], c["m"], c["w"], c["b"], c["blocks"], c["groups"]) == \
+            (st.P, st.E, st.S, st.m, st.w_frames, b, n + 1, len(ev))
+        lay = h.layout()
+        assert [tuple(r) for r in lay[:, [0, 1, 3]]] == _oracle_layout(st)
+        # physical slots: memory position = slot mod C, ring slot = frame mod R
+        for part, src, phys, _ in lay:
+            assert phys == (src % w.mem_slots if part == 0 else src % R)
+
+
+def test_soak_bookkeeping_closed_form_and_constant_footprint():
+    w = PRESETS["soak"]
+    h = _dry(w)
+    W, C = w.window_frames, w.mem_slots
+    total = 0
+    sizes = w.block_sizes()
+    assert len(sizes) == 2251 and sum(sizes) == 18000
+    max_keys = 0
+    for b in sizes:
+        h.dry_append(b)
+        c = h.counters()
+        E = 5 * math.ceil(max(0, total - W) / 5)
+        S = E // 5
+        assert (c["P"], c["E"], c["S"], c["m"], c["w"]) == (total, E, S, min(S, C), total - E)
+        lay = h.layout()
+        assert list(lay[:, 3]) == list(range(len(lay)))          # reset time indices 0..n-1
+        assert list(lay[lay[:, 0] == 0, 1]) == list(range(S - min(S, C), S))
+        total += b
+        max_keys = max(max_keys, len(lay))
+    assert max_keys <= C + W + max(w.first_block_frames, w.block_frames)
+
+
+def test_first_conv_at_block_3_for_512():
+    h = _dry(PRESETS["512x512"])
+    groups = []
+    for b in PRESETS["512x512"].block_sizes()[:4]:
+        h.dry_append(b)
+        groups.append(h.counters()["groups"])
+    assert groups[:3] == [0, 0, 1]

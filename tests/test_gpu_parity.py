@@ -1,0 +1,160 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every check compares the library's result with the oracle on the same seeded
+inputs.  Indices (layout, slot positions) must be bit-exact, appended ring
+frames must be bit-exact copies, attention outputs and compressed slots must
+hold the stated tolerances.
+"""
+import numpy as np
+import pytest
+
+import seeded_inputs as si
+from compressed_kv_cache_convkv_b200.configs import PRESETS, Workload
+from streams import (attention_errors, bf16_tensor_to_f64, check_attention, check_slot, device_frames,
+                     device_weights, host_frames, oracle_for, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as t
+    assert t.cuda.is_available(), "GPU tests need a CUDA device"
+    from compressed_kv_cache_convkv_b200 import build
+    build.build()
+    si.build(device=True)
+    return t
+
+
+def _ckv():
+    import compressed_kv_cache_convkv_b200 as ckv
+    return ckv
+
+
+def test_device_generator_matches_host(torch):
+    w = PRESETS["720x416"]
+    d = device_frames(w, si.K, 7, 2, torch)[0]
+    h = host_frames(w, si.K, 0, 7, 2).reshape(-1, w.heads, w.head_dim)
+    assert np.array_equal(d.view(torch.int16).cpu().numpy().view(np.uint16), h)
+
+
+def _run(torch, w: Workload, attend_blocks=None, rows=None, compress=0, t_offset=0, override=None,
+         check_slots=True, ring_frames=None, max_blocks=None, collect=None, sharp=False):
+    """Stream w through both sides; returns per-block error records."""
+    ckv = _ckv()
+    weights = device_weights(w, torch)
+    cfg = w.config(compress_mode=compress, t_offset=t_offset)
+    h = ckv.ConvKV(cfg, None if compress == ckv.COMPRESS_MEAN else weights)
+    st = oracle_for(w, mean=(compress == ckv.COMPRESS_MEAN))
+    rng = np.random.default_rng(w.seed)
+    R = cfg.ring_frames
+    F = 0
+    recs = []
+    sizes = w.block_sizes()[: max_blocks or None]
+    for n, b in enumerate(sizes, start=1):
+        kd, vd, qd = (device_frames(w, t, F, b, torch) for t in (si.K, si.V, si.Q))
+        kh, vh, qh = (host_frames(w, t, 0, F, b) for t in (si.K, si.V, si.Q))
+        if override is not None:
+            kd, vd, qd, kh, vh, qh = override(torch, kd, vd, qd, kh, vh, qh)
+        h.append(kd, vd)
+        out = h.attend(qd)
+        ev = st.append(si.bf16_bits_to_f64(kh), si.bf16_bits_to_f64(vh))
+        # indices: bit-exact layout
+        lay = h.layout()
+        assert [tuple(r) for r in lay[:, [0, 1, 3]]] == [tuple(r) for r in st.layout()], f"block {n}"
+        c = h.counters()
+        assert (c["P"], c["E"], c["S"], c["groups"]) == (st.P, st.E, st.S, len(ev))
+        # append: ring frames are bit-exact copies of the inputs
+        frames = range(b) if ring_frames is None else [x for x in ring_frames if x < b]
+        for f in frames:
+            kb, _ = h.read_ring(0, 0, (F + f) % R)
+            vb, _ = h.read_ring(0, 1, (F + f) % R)
+            assert np.array_equal(kb, kh[f]) and np.array_equal(vb, vh[f]), f"ring frame {F + f}"
+        # compression: new memory slots
+        if check_slots:
+            for e in ev[-cfg.mem_slots:]:
+                pos = e.slot % cfg.mem_slots
+                age = st.m - (st.S - e.slot)
+                ref_k, ref_v = st.memory_slot(age)
+                gk, _ = h.read_slot(0, 0, pos)
+                gv, _ = h.read_slot(0, 1, pos)
+                ek = check_slot(si.bf16_bits_to_f64(gk), ref_k, f"K slot {e.slot}")
+                ev_ = check_slot(si.bf16_bits_to_f64(gv), ref_v, f"V slot {e.slot}")
+                recs.append(("slot", n, e.slot, ek, ev_))
+        # attention
+        if attend_blocks is None or n in attend_blocks:
+            r = sample_rows(w, b, rows or b * w.T, rng)
+            ref, psum = st.attend(si.bf16_bits_to_f64(qh), rows=r)
+            assert np.abs(psum - 1).max() < 1e-12
+            gpu = bf16_tensor_to_f64(out[0][torch.as_tensor(r, device="cuda")])
+            e = check_attention(gpu, ref, what=f"{w.name} block {n}", sharp=sharp)
+            recs.append(("attend", n, len(r), e))
+            if collect is not None:
+                collect.append((n, r, gpu, ref))
+        F += b
+    assert h.status() == 0
+    h.close()
+    return recs
+
+
+def test_tiny_stream_full_parity(torch):
+    recs = _run(torch, PRESETS["tiny"])
+    assert sum(1 for r in recs if r[0] == "slot") == 5        # conv events at blocks 4, 6, 9, 11, 14
+    assert sum(1 for r in recs if r[0] == "attend") == 15
+
+
+def test_tiny_mean_memory(torch):
+    ckv = _ckv()
+    _run(torch, PRESETS["tiny"], compress=ckv.COMPRESS_MEAN)
+
+
+def test_tiny_time_shift_invariance(torch):
+    """Adding 1000 to every RoPE time index changes nothing (RoPE is relative)."""
+    a, b = [], []
+    _run(torch, PRESETS["tiny"], t_offset=0, collect=a)
+    _run(torch, PRESETS["tiny"], t_offset=1000, collect=b)
+    for (n, r, g0, ref), (_, _, g1, _) in zip(a, b):
+        e = attention_errors(g1, g0)
+        assert e["max"] <= 1e-2 and e["rel_l2"] <= 1e-2, (n, e)
+
+
+def test_tiny_v_ones_gives_ones(torch):
+    """V = 1 everywhere and mean compression: every output is exactly 1 (rows sum to 1)."""
+    ckv = _ckv()
+
+    def ones_v(t, kd, vd, qd, kh, vh, qh):
+        vd = t.ones_like(vd)
+        vh = np.full_like(vh, 0x3F80)
+        return kd, vd, qd, kh, vh, qh
+
+    col = []
+    _run(torch, PRESETS["tiny"], compress=ckv.COMPRESS_MEAN, override=ones_v, collect=col)
+    for n, r, gpu, ref in col:
+        assert np.all(gpu == 1.0), n
+
+
+def test_tiny_k_zero_gives_mean_of_valid_v(torch):
+    """K = 0: uniform weights, so a padded key leaking into a ragged tile would show."""
+    def zero_k(t, kd, vd, qd, kh, vh, qh):
+        return t.zeros_like(kd), vd, qd, np.zeros_like(kh), vh, qh
+
+    _run(torch, PRESETS["tiny"], override=zero_k)
+
+
+def test_tiny_sharp_softmax(torch):
+    """Queries scaled by 8: peaky softmax exercises the running-max rescale."""
+    def sharp(t, kd, vd, qd, kh, vh, qh):
+        qd = (qd.float() * 8).to(t.bfloat16)
+        qh8 = si.bf16_bits_to_f64(qh) * 8
+        qh = (qh8.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        return kd, vd, qd, kh, vh, qh
+
+    _run(torch, PRESETS["tiny"], override=sharp, sharp=True)
+
+
+def test_512_stream(torch):
+    _run(torch, PRESETS["512x512"], attend_blocks={1, 3, 4, 7, 9, 13, 20, 26}, rows=64, ring_frames=[0, 5])
+
+
+def test_720_stream_ragged(torch):
+    _run(torch, PRESETS["720x416"], attend_blocks={1, 3, 12, 13, 27, 38}, rows=64, ring_frames=[0, 5])
