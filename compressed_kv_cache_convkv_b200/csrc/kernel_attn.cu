@@ -12,16 +12,16 @@
 //
 // CTA = one (state, head, 256 query rows) work unit, 16 warps:
 //   warp 0      TMA producer: Q (2 tiles of 128 rows), then K/V tiles of 128
-//               keys through a 2-stage ring, per key segment
+//               keys through 3 (K) and 2 (V) stage rings, per key segment
 //   warp 1      tcgen05.mma issuer and TMEM owner: S_i = Q_i K^T (SS form),
 //               O_i += P_i V (P read from TMEM, TS form); tiles i = 0, 1 are
 //               interleaved so one tile's softmax overlaps the other's MMAs
 //   warps 4-7   softmax of query tile 0; warps 8-11 softmax of tile 1: one
 //               thread per query row; online softmax in fp32 registers with a
 //               lazily rescaled running max (the O rescale is only done when
-//               the max grows by more than 2^8); P written back over S as bf16,
-//               and the row sum taken over the same bf16 values the MMA uses
+//               the max grows by more than 2^8); P written back over S as bf16
 //   warps 12-15 RoPE of each landed K tile, in place in shared memory
+//               (cos/sin tables read through the read-only data cache)
 // TMEM: S_0 | S_1 | O_0 | O_1 = 128 | 128 | D | D columns of 512.
 // Every barrier wait is bounded; on expiry the CTA raises an abort flag, skips
 // the remaining work, drains its outstanding copies and MMAs, frees TMEM and
@@ -36,7 +36,7 @@ using namespace dev;
 
 template <int D>
 struct AttnCfg {
-  static constexpr int BM = 128, BN = 128, QT = 2, KST = 2, VST = 2;
+  static constexpr int BM = 128, BN = 128, QT = 2, KST = 3, VST = 2;
   static constexpr int NBOX = D / 64;
   static constexpr int TILE = 128 * D * 2;     // bytes of one 128-row bf16 tile
   static constexpr int BOX = 128 * 128;        // bytes of one 128-row x 64-channel box
@@ -46,17 +46,26 @@ struct AttnCfg {
   static constexpr int O_COL = 256;
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 512;
-  static constexpr int NBARS = 20;
-  static constexpr size_t FIXED = 1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16;
+  // registers per thread after re-balancing: the block launches with 128 x 512;
+  // producer/MMA warpgroup + RoPE warpgroup + two softmax warpgroups must sum to it
+  static constexpr int REG_LAUNCH = 128, REG_CTRL = 96, REG_ROPE = 80, REG_SOFTMAX = 168;
+  static_assert(128 * REG_CTRL + 128 * REG_ROPE + 256 * REG_SOFTMAX == THREADS * REG_LAUNCH,
+                "register split must add up to the launch allocation");
+  static constexpr int NBARS = 1 + 1 + 3 * KST + 2 * VST + 3 * 2 + 1;
+  static constexpr size_t FIXED =
+      1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16 + kMaxSegs * sizeof(KeySeg);
 };
 
-__device__ __forceinline__ int find_seg(const AttnParams& p, int j) {
-  int s = 0;
-#pragma unroll
-  for (int i = 1; i < kMaxSegs; ++i)
-    if (i < p.nseg && j >= p.seg[i].tile0) s = i;
-  return s;
-}
+// Walks the attend's key tiles segment by segment (no division, no search).
+struct TileCursor {
+  int s = 0, jt = 0;
+  __device__ __forceinline__ void next(const KeySeg* seg) {
+    if (++jt * 128 >= seg[s].nrows) {
+      ++s;
+      jt = 0;
+    }
+  }
+};
 
 // Rotate one 128-byte-swizzled row of a tile in place: adjacent channel pairs
 // (2i, 2i+1) of each axis segment [t | h | w] turn by the tabulated angle.
@@ -77,7 +86,8 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int row, const float2* c
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int pi = 4 * c + q;
-      const float2 cs = pi < C::PT ? cs_t[pi] : (pi < C::PT + C::PH ? cs_h[pi - C::PT] : cs_w[pi - C::PT - C::PH]);
+      const float2 cs = pi < C::PT ? __ldg(&cs_t[pi])
+                                   : (pi < C::PT + C::PH ? __ldg(&cs_h[pi - C::PT]) : __ldg(&cs_w[pi - C::PT - C::PH]));
       const float a = bf16lo_to_f32(w[q]), b = bf16hi_to_f32(w[q]);
       float ra = a * cs.x - b * cs.y;
       float rb = a * cs.y + b * cs.x;
@@ -104,21 +114,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint8_t* sK = sQ + C::QT * C::TILE;
   uint8_t* sV = sK + C::KST * C::TILE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::VST * C::TILE);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_ready = bars + 1;
-  uint64_t* k_full = bars + 2;    // [KST]
-  uint64_t* k_ready = bars + 4;   // [KST]
-  uint64_t* k_empty = bars + 6;   // [KST]
-  uint64_t* v_full = bars + 8;    // [VST]
-  uint64_t* v_empty = bars + 10;  // [VST]
-  uint64_t* s_full = bars + 12;   // [2]
-  uint64_t* p_full = bars + 14;   // [2]
-  uint64_t* o_full = bars + 16;   // [2]
-  uint64_t* drain = bars + 18;
+  uint64_t* q_full = bars;
+  uint64_t* q_ready = q_full + 1;
+  uint64_t* k_full = q_ready + 1;        // [KST]
+  uint64_t* k_ready = k_full + C::KST;   // [KST]
+  uint64_t* k_empty = k_ready + C::KST;  // [KST]
+  uint64_t* v_full = k_empty + C::KST;   // [VST]
+  uint64_t* v_empty = v_full + C::VST;   // [VST]
+  uint64_t* s_full = v_empty + C::VST;   // [2]
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* o_full = p_full + 2;         // [2]
+  uint64_t* drain = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float2* tab = reinterpret_cast<float2*>(tmem_slot + 4);
-  const float2* tab_t = tab;
+  KeySeg* seg = reinterpret_cast<KeySeg*>(tmem_slot + 4);
+  // cos/sin tables stay in global memory and are read through the read-only cache
+  const float2* tab_t = p.tables;
   const float2* tab_h = tab_t + p.tab_t_rows * C::PT;
   const float2* tab_w = tab_h + p.tab_h_rows * C::PH;
 
@@ -147,10 +158,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  {
-    const int ntab = p.tab_t_rows * C::PT + p.tab_h_rows * C::PH + p.tab_w_rows * C::PW;
-    for (int i = threadIdx.x; i < ntab; i += blockDim.x) tab[i] = p.tables[i];
-  }
+  if (threadIdx.x < kMaxSegs) seg[threadIdx.x] = p.seg[threadIdx.x];
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -160,11 +168,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < 4) {
+    regs_dec<C::REG_CTRL>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const CUtensorMap* kmap[3] = {&tmK0, &tmK1, &tmK2};
-      const CUtensorMap* vmap[3] = {&tmV0, &tmV1, &tmV2};
+      auto kmap = [&](int buf) { return buf == 0 ? &tmK0 : (buf == 1 ? &tmK1 : &tmK2); };
+      auto vmap = [&](int buf) { return buf == 0 ? &tmV0 : (buf == 1 ? &tmV1 : &tmV2); };
       tma_prefetch_desc(&tmQ);
       mbar_expect_tx(q_full, C::QT * C::TILE);
 #pragma unroll
@@ -173,22 +183,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(sQ + i * C::TILE + bx * C::BOX, &tmQ, q_full, bx * 64, head, q_row0 + i * C::BM, state);
       int kiss[C::KST] = {}, viss[C::VST] = {};
-      for (int j = 0; j < p.ntiles; ++j) {
-        const KeySeg& sg = p.seg[find_seg(p, j)];
-        const int row = sg.row0 + (j - sg.tile0) * C::BN;
+      TileCursor cur;
+      for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
+        const KeySeg& sg = seg[cur.s];
+        const int row = sg.row0 + cur.jt * C::BN;
         const int ks = j % C::KST;
         if (j >= C::KST && !mbar_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
         mbar_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap[sg.buf], &k_full[ks], bx * 64, head, row, state);
+          tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap(sg.buf), &k_full[ks], bx * 64, head, row, state);
         ++kiss[ks];
         const int vs = j % C::VST;
         if (j >= C::VST && !mbar_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, abort_flag)) break;
         mbar_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap[sg.buf], &v_full[vs], bx * 64, head, row, state);
+          tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap(sg.buf), &v_full[vs], bx * 64, head, row, state);
         ++viss[vs];
       }
       // drain: every issued copy must land before the CTA exits
@@ -204,23 +215,28 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, C::BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // descriptors of the tile bases; stepping along K or between tiles only adds
+      // (byte offset >> 4) to the 14-bit start-address field, which cannot overflow
+      // inside the CTA's shared memory
+      const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(sV), C::BOX, 1024);
       bool issued_any = false;
       auto issue_s = [&](int i, int ks) {
-        const uint32_t a = q_addr + i * C::TILE, b = k_addr + ks * C::TILE;
+        const uint64_t a = dq + static_cast<uint64_t>((i * C::TILE) >> 4);
+        const uint64_t b = dk + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          mma_ss(tmem + i * 128, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc_qk,
-                 kk > 0);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::BOX + (kk & 3) * 32) >> 4);
+          mma_ss(tmem + i * 128, a + off, b + off, idesc_qk, kk > 0);
         }
         issued_any = true;
       };
       auto issue_pv = [&](int i, int vs, bool acc) {
-        const uint32_t b = v_addr + vs * C::TILE;
+        const uint64_t b = dv + static_cast<uint64_t>((vs * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          mma_ts(tmem + C::O_COL + i * D, tmem + i * 128 + kk * 8, sdesc_sw128(b + kk * 16 * 128, C::BOX, 1024),
+          mma_ts(tmem + C::O_COL + i * D, tmem + i * 128 + kk * 8, b + static_cast<uint64_t>((kk * 16 * 128) >> 4),
                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
@@ -265,7 +281,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         mbar_wait(drain, 0, &no_abort);
       }
     }
-  } else if (warp >= 4 && warp < 12) {
+  }  // warps 2, 3: no role
+  } else if (warp < 12) {
+    regs_inc<C::REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int i = (warp - 4) >> 2;
     const int lane_base = (warp & 3) * 32;
@@ -286,28 +304,34 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const uint32_t tS = tmem + (static_cast<uint32_t>(lane_base) << 16) + i * 128;
     const uint32_t tO = tmem + (static_cast<uint32_t>(lane_base) << 16) + C::O_COL + i * D;
     float m_run = -INFINITY, l_run = 0.0f;
-    for (int j = 0; j < p.ntiles; ++j) {
+    TileCursor cur;
+    for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
       if (!mbar_wait_warp(&s_full[i], j & 1, abort_flag)) { alive = false; break; }
       tc_fence_after();
-      const KeySeg& sg = p.seg[find_seg(p, j)];
-      const int valid = min(C::BN, sg.nrows - (j - sg.tile0) * C::BN);
-      // pass 1: row max over the valid columns
-      float mx = -INFINITY;
+      const int valid = min(C::BN, seg[cur.s].nrows - cur.jt * C::BN);
+      // pass 1: row max over the valid columns (two chunks in flight, 4 chains of 3-input max)
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
+      for (int c = 0; c < C::BN / 32; c += 2) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(tS + c * 32, va);
+        tmem_ld32(tS + (c + 1) * 32, vb);
         tmem_ld_wait();
-        if (valid >= (c + 1) * 32) {
+        if (valid < (c + 2) * 32) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
-        } else {
+          for (int e = 0; e < 32; ++e) {
+            if (c * 32 + e >= valid) va[e] = __float_as_uint(-INFINITY);
+            if ((c + 1) * 32 + e >= valid) vb[e] = __float_as_uint(-INFINITY);
+          }
+        }
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e < valid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int e = 0; e < 32; e += 2) {
+          mx[(e >> 1) & 3] = max3f(mx[(e >> 1) & 3], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
+          mx[((e >> 1) + 2) & 3] = max3f(mx[((e >> 1) + 2) & 3], __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
         }
       }
-      const float m_new = fmaxf(m_run, mx);
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m_run, m_tile);
       if (j == 0) {
         m_run = m_new;
       } else {
@@ -330,31 +354,45 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
       }
-      // pass 2: P = exp2(S - m) as bf16, written over the first half of S's columns
+      // pass 2: P = exp2(S - m) as bf16, written over the first half of S's columns;
+      // the next 32-column chunk is loaded while this one is exponentiated.  Pairs of
+      // columns go through the packed fp32x2 add (S - m, and the running row sum).
+      const uint64_t neg_m = f2_make(-m_run, -m_run);
+      uint64_t lsum[4] = {0, 0, 0, 0};
+      uint32_t va[32];
+      tmem_ld32(tS, va);
+      tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_ld_wait();
+        uint32_t vb[32];
+        if (c + 1 < C::BN / 32) tmem_ld32(tS + (c + 1) * 32, vb);
+        if (valid < (c + 1) * 32) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e >= valid) va[e] = __float_as_uint(-INFINITY);
+        }
         uint32_t pk[16];
-        if (valid >= (c + 1) * 32) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(__uint_as_float(v[2 * e]) - m_run);
-            const float p1 = fast_exp2(__uint_as_float(v[2 * e + 1]) - m_run);
-            pk[e] = pack_bf16x2(p0, p1);
-            l_run += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = (c * 32 + 2 * e < valid) ? fast_exp2(__uint_as_float(v[2 * e]) - m_run) : 0.0f;
-            const float p1 = (c * 32 + 2 * e + 1 < valid) ? fast_exp2(__uint_as_float(v[2 * e + 1]) - m_run) : 0.0f;
-            pk[e] = pack_bf16x2(p0, p1);
-            l_run += bf16lo_to_f32(pk[e]) + bf16hi_to_f32(pk[e]);
-          }
+        for (int e = 0; e < 16; ++e) {
+          float d0, d1;
+          f2_split(f2_add(f2_make(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1])), neg_m), d0, d1);
+          const float p0 = fast_exp2(d0), p1 = fast_exp2(d1);
+          pk[e] = pack_bf16x2(p0, p1);
+          lsum[e & 3] = f2_add(lsum[e & 3], f2_make(p0, p1));
         }
         tmem_st16(tS + c * 16, pk);
+        if (c + 1 < C::BN / 32) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) va[e] = vb[e];
+        }
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_split(f2_add(f2_add(lsum[0], lsum[1]), f2_add(lsum[2], lsum[3])), a0, a1);
+        (void)b0;
+        (void)b1;
+        l_run += a0 + a1;
       }
       tmem_st_wait();
       tc_fence_before();
@@ -380,16 +418,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
       }
     }
-  } else if (warp >= 12) {
+  } else {
+    regs_dec<C::REG_ROPE>();
     // ------------------------------------------------------------ K RoPE
     const int r = threadIdx.x - 384;
-    for (int j = 0; j < p.ntiles; ++j) {
+    TileCursor cur;
+    for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
       const int ks = j % C::KST;
       if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
-      const KeySeg& sg = p.seg[find_seg(p, j)];
-      const int off = (j - sg.tile0) * C::BN;
-      if (off + r < sg.nrows) {
-        const int lr = off + r;
+      const KeySeg& sg = seg[cur.s];
+      const int lr = cur.jt * C::BN + r;
+      if (lr < sg.nrows) {
         const int f = lr / p.T;
         const int s = lr - f * p.T;
         const int t = sg.t0 + f;
@@ -412,14 +451,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 }
 
 template <int D>
-size_t smem_for(const AttnParams& p) {
+size_t smem_for(const AttnParams&) {
   using C = AttnCfg<D>;
-  const size_t ntab = static_cast<size_t>(p.tab_t_rows) * C::PT + static_cast<size_t>(p.tab_h_rows) * C::PH +
-                      static_cast<size_t>(p.tab_w_rows) * C::PW;
-  const size_t need = C::FIXED + ntab * sizeof(float2);
   // at least half the SM's shared memory: one CTA per SM, so the 512-column
   // TMEM allocation never has to wait for a co-resident CTA
-  return need > 120 * 1024 ? need : 120 * 1024;
+  return C::FIXED > 120 * 1024 ? C::FIXED : 120 * 1024;
 }
 
 template <int D>

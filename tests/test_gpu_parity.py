@@ -119,7 +119,9 @@ def test_tiny_time_shift_invariance(torch):
 
 
 def test_tiny_v_ones_gives_ones(torch):
-    """V = 1 everywhere and mean compression: every output is exactly 1 (rows sum to 1)."""
+    """V = 1 everywhere and mean compression: every output is 1 up to the bf16 rounding
+    of the attention weights (each weight is rounded to bf16 for the PV product, relative
+    error <= 2^-8, while the row sum uses the unrounded weights)."""
     ckv = _ckv()
 
     def ones_v(t, kd, vd, qd, kh, vh, qh):
@@ -130,7 +132,8 @@ def test_tiny_v_ones_gives_ones(torch):
     col = []
     _run(torch, PRESETS["tiny"], compress=ckv.COMPRESS_MEAN, override=ones_v, collect=col)
     for n, r, gpu, ref in col:
-        assert np.all(gpu == 1.0), n
+        assert np.abs(gpu - 1.0).max() <= 2.0 ** -8, n
+        assert np.mean(gpu == 1.0) > 0.9, n
 
 
 def test_tiny_k_zero_gives_mean_of_valid_v(torch):
