@@ -309,90 +309,72 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       if (!mbar_wait_warp(&s_full[i], j & 1, abort_flag)) { alive = false; break; }
       tc_fence_after();
       const int valid = min(C::BN, seg[cur.s].nrows - cur.jt * C::BN);
-      // pass 1: row max over the valid columns (two chunks in flight, 4 chains of 3-input max)
+      // the whole 128-column row of S in registers, one TMEM round trip
+      uint32_t sv[C::BN];
+      tmem_ld64(tS, sv);
+      tmem_ld64(tS + 64, sv + 64);
+      tmem_ld_wait();
+      if (valid < C::BN) {
+#pragma unroll
+        for (int e = 0; e < C::BN; ++e)
+          if (e >= valid) sv[e] = __float_as_uint(-INFINITY);
+      }
+      // row max: 4 independent chains of 3-input max
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; c += 2) {
-        uint32_t va[32], vb[32];
-        tmem_ld32(tS + c * 32, va);
-        tmem_ld32(tS + (c + 1) * 32, vb);
-        tmem_ld_wait();
-        if (valid < (c + 2) * 32) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (c * 32 + e >= valid) va[e] = __float_as_uint(-INFINITY);
-            if ((c + 1) * 32 + e >= valid) vb[e] = __float_as_uint(-INFINITY);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          mx[(e >> 1) & 3] = max3f(mx[(e >> 1) & 3], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
-          mx[((e >> 1) + 2) & 3] = max3f(mx[((e >> 1) + 2) & 3], __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
-        }
-      }
+      for (int e = 0; e < C::BN; e += 2)
+        mx[(e >> 1) & 3] = max3f(mx[(e >> 1) & 3], __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
       const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m_run, m_tile);
+      // lazy rescale: keep the running max unless it grows by more than 2^8
+      bool rescale = false;
+      float corr = 1.0f;
       if (j == 0) {
         m_run = m_new;
       } else {
         const bool need = m_new > m_run + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O has no MMA in flight here: PV_i(j-1) completed before S_i(j) was committed
-          const float corr = need ? fast_exp2(m_run - m_new) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + c * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-            tmem_st32(tO + c * 32, v);
-          }
-          if (need) {
-            l_run *= corr;
-            m_run = m_new;
-          }
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          corr = fast_exp2(m_run - m_new);
+          l_run *= corr;
+          m_run = m_new;
         }
       }
-      // pass 2: P = exp2(S - m) as bf16, written over the first half of S's columns;
-      // the next 32-column chunk is loaded while this one is exponentiated.  Pairs of
-      // columns go through the packed fp32x2 add (S - m, and the running row sum).
+      // P = exp2(S - m) as bf16 pairs, written over the first half of S's columns in two
+      // halves; pairs of columns go through the packed fp32x2 add (S - m and row sum)
       const uint64_t neg_m = f2_make(-m_run, -m_run);
       uint64_t lsum[4] = {0, 0, 0, 0};
-      uint32_t va[32];
-      tmem_ld32(tS, va);
-      tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t vb[32];
-        if (c + 1 < C::BN / 32) tmem_ld32(tS + (c + 1) * 32, vb);
-        if (valid < (c + 1) * 32) {
+      for (int h = 0; h < 2; ++h) {
+        // packed pair e of this half lands in sv[h*64 + e], a slot already consumed
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e >= valid) va[e] = __float_as_uint(-INFINITY);
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 32; ++e) {
+          const int col = h * 64 + 2 * e;
           float d0, d1;
-          f2_split(f2_add(f2_make(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1])), neg_m), d0, d1);
+          f2_split(f2_add(f2_make(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), neg_m), d0, d1);
           const float p0 = fast_exp2(d0), p1 = fast_exp2(d1);
-          pk[e] = pack_bf16x2(p0, p1);
+          sv[h * 64 + e] = pack_bf16x2(p0, p1);
           lsum[e & 3] = f2_add(lsum[e & 3], f2_make(p0, p1));
         }
-        tmem_st16(tS + c * 16, pk);
-        if (c + 1 < C::BN / 32) {
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) va[e] = vb[e];
-        }
+        tmem_st32p(tS + h * 32, sv + h * 64);
       }
       {
-        float a0, a1, b0, b1;
+        float a0, a1;
         f2_split(f2_add(f2_add(lsum[0], lsum[1]), f2_add(lsum[2], lsum[3])), a0, a1);
-        (void)b0;
-        (void)b1;
         l_run += a0 + a1;
+      }
+      if (rescale) {
+        // O has no MMA in flight here: PV_i(j-1) completed before S_i(j) was committed,
+        // and PV_i(j) is issued only after this thread arrives on p_full below
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
+          tmem_st32(tO + c * 32, v);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
