@@ -33,7 +33,10 @@ groups of 5 until the window holds at most W frames; the memory is a FIFO of
 C slots (oldest dropped); the conv is a per-head cross-correlation over the 5
 evicted frames (tap j = j-th oldest frame), no bias, applied to un-rotated K
 and V; compressed slots are stored in the cache's storage type (bf16 rounded
-to nearest even, or e4m3 with a per-(head, slot) fp32 scale); RoPE time
+to nearest even, or e4m3 with a per-(head, slot) fp32 scale); an e4m3 value is
+dequantised to BF16 on use as bf16(fp32(code * scale)), so every consumer (the
+conv of evicted window frames, the attention over window and memory) reads
+that bf16 value; RoPE time
 indices restart at 0 over [memory | window | current], one index per memory
 slot, spatial (row, column) indices are kept; RoPE rotates adjacent pairs of
 each axis segment [t | h | w] with frequency theta^(-2i/d_axis); softmax scale
@@ -100,12 +103,12 @@ def e4m3_rne_satfinite(x32: np.ndarray) -> np.ndarray:
     return np.where(a > 0, np.copysign(q, x), 0.0 * x)
 
 
-def fp8_quantize(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
-    """Per-head e4m3 quantisation of one frame or slot x[T, H, D].
+def fp8_encode(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-head e4m3 codes of one frame or slot x[T, H, D].
 
     scale = amax / 448 in fp32 (1 if amax == 0); code = e4m3(fp32(x) / scale)
-    with the fp32 divide rounded to nearest.  Returns (dequantised values
-    code * scale in float64, scales[H] as float32).
+    with the fp32 divide rounded to nearest.  Returns (code values as float64,
+    scales[H] as float32).
     """
     x = np.asarray(x, dtype=np.float64)
     x32 = x.astype(np.float32)
@@ -113,8 +116,20 @@ def fp8_quantize(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     scale = np.where(amax == 0, np.float32(1.0), (amax / np.float32(E4M3_MAX)).astype(np.float32))
     scale = scale.astype(np.float32)
     y = (x32 / scale[None, :, None]).astype(np.float32)      # IEEE fp32 divide
-    code = e4m3_rne_satfinite(y)
-    return code * scale.astype(np.float64)[None, :, None], scale
+    return e4m3_rne_satfinite(y), scale
+
+
+def fp8_dequantize(code: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Dequantise to BF16 on use: bf16(fp32(code * scale)), scale per head (axis 1)."""
+    prod = (np.asarray(code, dtype=np.float32) * np.asarray(scale, dtype=np.float32)[None, :, None]).astype(np.float32)
+    return round_to_bf16(prod.astype(np.float64))
+
+
+def fp8_quantize(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """e4m3 storage of x[T, H, D] followed by the bf16 dequantisation used by every
+    consumer (conv input, attention K/V).  Returns (dequantised values, scales[H])."""
+    code, scale = fp8_encode(x)
+    return fp8_dequantize(code, scale), scale
 
 
 # --------------------------------------------------------------------------
@@ -239,9 +254,10 @@ class OracleConfig:
 
 @dataclass
 class _Frame:
-    k: np.ndarray          # [T, H, D] float64 (stored values)
+    k: np.ndarray          # [T, H, D] float64 (stored values, as consumed)
     v: np.ndarray
     index: int             # stream frame index (window/current) or slot index (memory)
+    codes: Optional[tuple] = None   # fp8: (k codes, k scales, v codes, v scales)
 
 
 @dataclass
@@ -286,17 +302,20 @@ class OracleStream:
             group, self.window = self.window[:EVICT], self.window[EVICT:]
             kc = conv_compress(np.stack([f.k for f in group]), self.w[0])
             vc = conv_compress(np.stack([f.v for f in group]), self.w[1])
+            codes = None
             if cfg.fp8:
-                kc, sk = fp8_quantize(kc)
-                vc, sv = fp8_quantize(vc)
+                ck, sk = fp8_encode(kc)
+                cv, sv = fp8_encode(vc)
+                kc, vc = fp8_dequantize(ck, sk), fp8_dequantize(cv, sv)
                 scales = np.stack([sk, sv])
+                codes = (ck, sk, cv, sv)
             else:
                 kc, vc = round_to_bf16(kc), round_to_bf16(vc)
                 scales = None
             if len(self.memory) == cfg.mem_slots:
                 self.memory.pop(0)
                 self.mem_scales.pop(0)
-            self.memory.append(_Frame(kc, vc, self.S))
+            self.memory.append(_Frame(kc, vc, self.S, codes))
             self.mem_scales.append(scales)
             ev = ConvEvent(self.block, group[0].index, self.S)
             self.E += EVICT
@@ -311,9 +330,9 @@ class OracleStream:
             vf = np.asarray(v[f], dtype=np.float64)
             self.current.append(_Frame(kf, vf, idx))
             if cfg.fp8:
-                kq, sk = fp8_quantize(kf)
-                vq, sv = fp8_quantize(vf)
-                self.current_q8.append(_Frame(kq, vq, idx))
+                ck, sk = fp8_encode(kf)
+                cv, sv = fp8_encode(vf)
+                self.current_q8.append(_Frame(fp8_dequantize(ck, sk), fp8_dequantize(cv, sv), idx, (ck, sk, cv, sv)))
                 self.frame_scales[idx] = np.stack([sk, sv])
         return new_events
 

@@ -61,6 +61,17 @@ def test_e4m3_grid_round_trip():
     assert np.array_equal(O.e4m3_rne_satfinite(vals), vals.astype(np.float64))
 
 
+def test_fp8_dequantise_is_bf16_of_fp32_product():
+    # "dequantize to BF16 on use": the consumed value is bf16(fp32(code * scale)); checked
+    # against torch's own e4m3 decode, fp32 multiply and single-rounding fp32 -> bf16 cast
+    x = RNG.standard_normal((32, 2, 16)) * 3
+    code, scale = O.fp8_encode(x)
+    deq = O.fp8_dequantize(code, scale)
+    t = torch.from_numpy(code.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float32)
+    ref = (t * torch.from_numpy(scale)[None, :, None]).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(deq, ref)
+
+
 def test_fp8_quantize_scale_rule():
     x = RNG.standard_normal((16, 3, 8))
     x[:, 2, :] = 0.0
@@ -72,9 +83,9 @@ def test_fp8_quantize_scale_rule():
     for h in range(2):
         i = np.unravel_index(np.argmax(np.abs(x[:, h, :])), x[:, h, :].shape)
         assert abs(abs(deq[i[0], h, i[1]]) / scale[h] - 448) <= 32
-    # dequantised error is within half an e4m3 quantum (relative 2^-4) of the fp32 input
+    # dequantised error: half an e4m3 quantum (relative 2^-4) plus the bf16 rounding (2^-8)
     rel = np.abs(deq[:, :2] - x[:, :2].astype(np.float32)) / np.maximum(np.abs(x[:, :2]), 2 ** -6 * scale[:2][None, :, None])
-    assert rel.max() <= 2 ** -4 + 1e-6
+    assert rel.max() <= 2 ** -4 + 2 ** -8 + 1e-6
 
 
 # ---------------------------------------------------------------- RoPE
@@ -388,9 +399,12 @@ def test_stream_memory_slots_are_bf16_conv_of_group():
 def test_fp8_stream_window_is_quantised_current_is_exact():
     for st, (q, k, v), _ in _tiny_stream(W=4, C=3, blocks=5, fp8=True, seed=13):
         pass
-    # current block frames are the exact inputs; window frames are per-(head, frame) e4m3 * scale
+    # current block frames are the exact inputs; window frames are per-(head, frame) e4m3
+    # codes (fixed points of the quantiser) dequantised to bf16
     np.testing.assert_array_equal(st.current[0].k, k[0])
     for f in st.window:
-        sc = st.frame_scales[f.index]
-        codes = f.k / sc[0][None, :, None]
-        np.testing.assert_array_equal(O.e4m3_rne_satfinite(codes.astype(np.float32)), codes)
+        ck, sk, cv, sv = f.codes
+        np.testing.assert_array_equal(O.e4m3_rne_satfinite(ck.astype(np.float32)), ck)
+        np.testing.assert_array_equal(sk, st.frame_scales[f.index][0])
+        np.testing.assert_array_equal(f.k, O.fp8_dequantize(ck, sk))
+        np.testing.assert_array_equal(O.round_to_bf16(f.k), f.k)
