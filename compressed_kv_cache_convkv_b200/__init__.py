@@ -252,19 +252,23 @@ class ConvKV:
         return rec[:n]
 
     def read_slot(self, state: int, kv: int, pos: int):
-        """(bf16 bits [T, H, D] as uint16, scales[H] or None) of memory position `pos`."""
+        """(bf16 bits [T, H, D] as uint16 -- or e4m3 codes as uint8 in the fp8 format --,
+        scales[H] or None) of memory position `pos`."""
         import numpy as np
         cfg = self.cfg
-        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=np.uint16)
+        dt = np.uint8 if cfg.kv_format == KV_FP8_E4M3 else np.uint16
+        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=dt)
         sc = np.zeros(cfg.heads, dtype=np.float32)
         self._check(_lib().convkv_read_slot(self._h, state, kv, pos, dst.ctypes.data, sc.ctypes.data),
                     "convkv_read_slot")
         return dst, (sc if cfg.kv_format == KV_FP8_E4M3 else None)
 
     def read_ring(self, state: int, kv: int, slot: int):
+        """Same as read_slot for ring slot `slot`."""
         import numpy as np
         cfg = self.cfg
-        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=np.uint16)
+        dt = np.uint8 if cfg.kv_format == KV_FP8_E4M3 else np.uint16
+        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=dt)
         sc = np.zeros(cfg.heads, dtype=np.float32)
         self._check(_lib().convkv_read_ring(self._h, state, kv, slot, dst.ctypes.data, sc.ctypes.data),
                     "convkv_read_ring")

@@ -58,10 +58,14 @@ struct convkv {
   void* arena = nullptr;
   size_t arena_bytes = 0;
   void *ringK = nullptr, *ringV = nullptr, *memK = nullptr, *memV = nullptr, *weights = nullptr;
+  // fp8 format: ringK/ringV/memK/memV hold e4m3 codes; scales per (state, K|V, slot, head)
+  float *ring_scale = nullptr, *mem_scale = nullptr;
+  void *stageK = nullptr, *stageV = nullptr;  // bf16 copy of the current block
+  unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
   float2* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
-  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{};
+  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{};
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
   int last_cuda = 0;
@@ -132,7 +136,7 @@ int validate(const convkv_cfg* c) {
   const int64_t tabs = (int64_t(c->mem_slots) + c->window_frames + Bmax) * (D - 2 * dh) / 2 +
                        (int64_t(c->grid_h) + c->grid_w) * dh / 2;
   if (tabs * 8 > 32 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables must fit in shared memory
-  if (c->kv_format == CONVKV_KV_FP8_E4M3 && !(c->flags & CONVKV_FLAG_DRY_RUN)) return CONVKV_ERR_UNSUPPORTED;
+  if (c->kv_format == CONVKV_KV_FP8_E4M3 && c->compress_mode == CONVKV_COMPRESS_MEAN) return CONVKV_ERR_UNSUPPORTED;
   if (c->compress_mode == CONVKV_COMPRESS_CONV && !(c->flags & CONVKV_FLAG_DRY_RUN) && !c->conv_weight)
     return CONVKV_ERR_INVALID_ARG;
   return CONVKV_OK;
@@ -206,8 +210,14 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   }
 
   const size_t fe = static_cast<size_t>(h->frame_elems());
-  const size_t ring_b = static_cast<size_t>(h->S) * h->R * fe * 2;
-  const size_t mem_b = static_cast<size_t>(h->S) * h->C * fe * 2;
+  const size_t esz = h->fp8 ? 1 : 2;  // bytes per cached element
+  const size_t ring_b = static_cast<size_t>(h->S) * h->R * fe * esz;
+  const size_t mem_b = static_cast<size_t>(h->S) * h->C * fe * esz;
+  const size_t rsc_b = h->fp8 ? static_cast<size_t>(h->S) * 2 * h->R * h->H * sizeof(float) : 0;
+  const size_t msc_b = h->fp8 ? static_cast<size_t>(h->S) * 2 * h->C * h->H * sizeof(float) : 0;
+  const size_t stg_b = h->fp8 ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
+  const size_t amax_n = static_cast<size_t>(h->S) * 2 * h->H * (h->Bmax > kMaxGroups ? h->Bmax : kMaxGroups);
+  const size_t amax_b = h->fp8 ? amax_n * sizeof(unsigned int) : 0;
   const size_t w_b = h->mean ? 0 : static_cast<size_t>(h->S) * 2 * h->H * kEvict * h->D * h->D * 2;
   std::vector<float2> tab;
   build_tables(h, tab);
@@ -221,7 +231,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   };
   const size_t o_rk = take(ring_b), o_rv = take(ring_b), o_mk = take(mem_b), o_mv = take(mem_b), o_w = take(w_b),
                o_tab = take(tab_b), o_st = take(sizeof(int)), o_q = take(io_b), o_k = take(io_b),
-               o_v = take(io_b), o_o = take(io_b);
+               o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
+               o_sv = take(stg_b), o_am = take(amax_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -238,6 +249,13 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->weights = w_b ? a + o_w : nullptr;
   h->tables = reinterpret_cast<float2*>(a + o_tab);
   h->status = reinterpret_cast<int*>(a + o_st);
+  if (h->fp8) {
+    h->ring_scale = reinterpret_cast<float*>(a + o_rsc);
+    h->mem_scale = reinterpret_cast<float*>(a + o_msc);
+    h->stageK = a + o_sk;
+    h->stageV = a + o_sv;
+    h->amax = reinterpret_cast<unsigned int*>(a + o_am);
+  }
   if (h->host_io) {
     h->io_q = a + o_q;
     h->io_k = a + o_k;
@@ -255,10 +273,17 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->launches++;
   }
   if ((e = cudaStreamSynchronize(h->stream)) != cudaSuccess) goto fail_cuda;
-  rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
-  if (!rc) rc = encode_4d(&h->mapRingV, h->ringV, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
-  if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
-  if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+  if (h->fp8) {
+    // e4m3 ring and memory are read by the kernels' own dequantising loads; TMA only
+    // serves the bf16 staging of the current block
+    rc = encode_4d(&h->mapStageK, h->stageK, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapStageV, h->stageV, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
+  } else {
+    rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapRingV, h->ringV, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+  }
   if (!rc && w_b) rc = encode_weights(&h->mapW, h->weights, h->D, h->H, h->S);
   if (rc) {
     cudaFree(h->arena);
@@ -324,9 +349,20 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
     cp.memK = h->memK;
     cp.memV = h->memV;
     cp.status = h->status;
-    int e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
-                    : launch_conv_bf16(h->D, cp, h->mapRingK, h->mapRingV, h->mapW, h->stream);
-    h->launches++;
+    int e;
+    if (h->fp8) {
+      cp.ring8[0] = static_cast<const uint8_t*>(h->ringK);
+      cp.ring8[1] = static_cast<const uint8_t*>(h->ringV);
+      cp.ring_scale = h->ring_scale;
+      cp.amax = h->amax;
+      cp.mem_scale = h->mem_scale;
+      e = launch_conv_fp8(h->D, cp, h->mapW, h->stream);
+      h->launches += 2;
+    } else {
+      e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
+                  : launch_conv_bf16(h->D, cp, h->mapRingK, h->mapRingV, h->mapW, h->stream);
+      h->launches++;
+    }
     if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   }
   // 3. the new block becomes the current block: copy into ring slots (P + f) mod R
@@ -336,8 +372,23 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
   ap.R = h->R;
   ap.slot0 = static_cast<int>(h->P % h->R);
   ap.frame_elems = h->frame_elems();
-  int e = launch_append_bf16(ap, k, v, h->ringK, h->ringV, h->stream);
-  h->launches++;
+  int e;
+  if (h->fp8) {
+    ap.H = h->H;
+    ap.D = h->D;
+    ap.amax = h->amax;
+    ap.ring8[0] = static_cast<uint8_t*>(h->ringK);
+    ap.ring8[1] = static_cast<uint8_t*>(h->ringV);
+    ap.ring_scale = h->ring_scale;
+    ap.stage[0] = h->stageK;
+    ap.stage[1] = h->stageV;
+    ap.stage_frames = h->Bmax;
+    e = launch_append_fp8(ap, k, v, h->stream);
+    h->launches += 2;
+  } else {
+    e = launch_append_bf16(ap, k, v, h->ringK, h->ringV, h->stream);
+    h->launches++;
+  }
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   return CONVKV_OK;
 }
@@ -361,6 +412,8 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
     s.nrows = nframes * T;
     s.t0 = t0;
     s.tile0 = tiles;
+    s.fp8 = (h->fp8 && buf != 2) ? 1 : 0;
+    s.slot0 = frame0;
     tiles += (s.nrows + 127) / 128;
   };
   if (m > 0) {
@@ -370,11 +423,14 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
     if (m > n1) add(1, 0, m - n1, n1);
   }
   {
-    const int n = w + b;
+    // bf16: window and current block are consecutive ring frames; fp8: the window
+    // is e4m3 in the ring and the current block bf16 in staging
+    const int n = h->fp8 ? w : w + b;
     const int start = static_cast<int>(h->E % h->R);
     const int n1 = n < h->R - start ? n : h->R - start;
-    add(0, start, n1, m);
+    if (n1 > 0) add(0, start, n1, m);
     if (n > n1) add(0, 0, n - n1, m + n1);
+    if (h->fp8) add(2, 0, b, m + w);
   }
   ap.ntiles = tiles;
   ap.tab_t_rows = h->tab_t_rows;
@@ -389,9 +445,21 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
   CUtensorMap mq;
   int rc = encode_4d(&mq, const_cast<void*>(q), h->D, h->H, ap.Nq, h->S);
   if (rc) return rc;
-  CUtensorMap km[3] = {h->mapRingK, h->mapMemK, h->mapRingK};
-  CUtensorMap vm[3] = {h->mapRingV, h->mapMemV, h->mapRingV};
-  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->stream);
+  CUtensorMap km[3], vm[3];
+  if (h->fp8) {
+    ap.ring_scale = h->ring_scale;
+    ap.mem_scale = h->mem_scale;
+    ap.ring8[0] = static_cast<const uint8_t*>(h->ringK);
+    ap.ring8[1] = static_cast<const uint8_t*>(h->ringV);
+    ap.mem8[0] = static_cast<const uint8_t*>(h->memK);
+    ap.mem8[1] = static_cast<const uint8_t*>(h->memV);
+    km[0] = km[1] = km[2] = h->mapStageK;  // only the staging map is used by TMA
+    vm[0] = vm[1] = vm[2] = h->mapStageV;
+  } else {
+    km[0] = h->mapRingK; km[1] = h->mapMemK; km[2] = h->mapRingK;
+    vm[0] = h->mapRingV; vm[1] = h->mapMemV; vm[2] = h->mapRingV;
+  }
+  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp8, h->stream);
   h->launches++;
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   return CONVKV_OK;
@@ -439,7 +507,7 @@ int convkv_layout(const convkv_t* h, int32_t* rec, int cap) {
     put(0, k, k % h->C, i);
   }
   for (int i = 0; i < w; ++i) put(1, h->E + i, (h->E + i) % h->R, m + i);
-  for (int f = 0; f < b; ++f) put(2, h->P + f, (h->P + f) % h->R, m + w + f);
+  for (int f = 0; f < b; ++f) put(2, h->P + f, h->fp8 ? f : (h->P + f) % h->R, m + w + f);
   return n;
 }
 
@@ -456,30 +524,32 @@ int convkv_counters(const convkv_t* h, int64_t out[8]) {
   return CONVKV_OK;
 }
 
-static int read_frame(const convkv_t* hc, const void* dev_base, int nslots, int state, int slot, void* host_dst) {
+static int read_frame(const convkv_t* hc, const void* dev_base, int nslots, int state, int slot, void* host_dst,
+                      const float* scales, int kv, float* host_scales) {
   convkv_t* h = const_cast<convkv_t*>(hc);
-  const size_t fb = static_cast<size_t>(h->frame_elems()) * 2;
+  const size_t fb = static_cast<size_t>(h->frame_elems()) * (h->fp8 ? 1 : 2);
   const char* src = static_cast<const char*>(dev_base) + (static_cast<size_t>(state) * nslots + slot) * fb;
   cudaError_t e = cudaStreamSynchronize(h->stream);
   if (e == cudaSuccess) e = cudaMemcpy(host_dst, src, fb, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && h->fp8 && host_scales)
+    e = cudaMemcpy(host_scales, scales + ((static_cast<size_t>(state) * 2 + kv) * nslots + slot) * h->H,
+                   sizeof(float) * h->H, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return h->cuda_fail(e);
   return CONVKV_OK;
 }
 
 int convkv_read_slot(const convkv_t* h, int state, int kv, int pos, void* host_dst, float* host_scales) {
-  (void)host_scales;
   if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || pos < 0 || pos >= h->C)
     return CONVKV_ERR_INVALID_ARG;
   if (h->dry) return CONVKV_ERR_BAD_ORDER;
-  return read_frame(h, kv ? h->memV : h->memK, h->C, state, pos, host_dst);
+  return read_frame(h, kv ? h->memV : h->memK, h->C, state, pos, host_dst, h->mem_scale, kv, host_scales);
 }
 
 int convkv_read_ring(const convkv_t* h, int state, int kv, int slot, void* host_dst, float* host_scales) {
-  (void)host_scales;
   if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || slot < 0 || slot >= h->R)
     return CONVKV_ERR_INVALID_ARG;
   if (h->dry) return CONVKV_ERR_BAD_ORDER;
-  return read_frame(h, kv ? h->ringV : h->ringK, h->R, state, slot, host_dst);
+  return read_frame(h, kv ? h->ringV : h->ringK, h->R, state, slot, host_dst, h->ring_scale, kv, host_scales);
 }
 
 int convkv_status(convkv_t* h) {

@@ -18,14 +18,14 @@ constexpr int kStatusTimeout = 1;
 
 // One contiguous run of key rows in one buffer.
 struct KeySeg {
-  int buf;     // which K/V tensor maps: 0 ring, 1 memory, 2 fp8 current-block staging
+  int buf;     // 0 ring, 1 memory, 2 current-block staging (fp8 format only)
   int row0;    // first row (token) in that buffer, a frame boundary
   int nrows;   // rows = frames * T
   int t0;      // RoPE time index of the segment's first frame
   int tile0;   // index of the segment's first 128-row key tile in the attend's tile list
-  int fp8;     // 1 if the rows are e4m3 with per-frame scales
-  int scale_slot0;  // fp8: slot index (ring slot or memory position) of the first frame
-  int scale_nslots; // fp8: slots in the scale array (R or C) for wrap-free indexing
+  int fp8;     // 1 if the rows are e4m3 with per-(frame, head) fp32 scales
+  int slot0;   // ring slot or memory position of the segment's first frame (row0 / T)
+  int pad;
 };
 
 struct AttnParams {
@@ -39,6 +39,8 @@ struct AttnParams {
   float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
   const float* ring_scale;  // fp8: [S][2][R][H]
   const float* mem_scale;   // fp8: [S][2][C][H]
+  const uint8_t* ring8[2];  // fp8: e4m3 K, V rings [S][R*T][H][D]
+  const uint8_t* mem8[2];   // fp8: e4m3 K, V memory [S][C*T][H][D]
   int R, C;
   int* status;
 };
@@ -51,14 +53,27 @@ struct ConvGroup {
 struct ConvParams {
   int H, T, S, C, R, ngroups;
   ConvGroup grp[kMaxGroups];
-  void* memK;             // bf16 [S][C*T][H][D], or fp32 scratch in the fp8 format
+  void* memK;             // bf16 [S][C*T][H][D], or e4m3 in the fp8 format
   void* memV;
   int* status;
+  // fp8 format: e4m3 ring input with per-(frame, head) scales, two passes
+  int pass;                   // 1: amax of the conv output only, 2: quantise with that amax
+  const uint8_t* ring8[2];    // e4m3 K, V rings [S][R*T][H][D]
+  const float* ring_scale;    // [S][2][R][H]
+  unsigned int* amax;         // [S][2][ngroups][H] fp32 bit patterns (scratch, zeroed before pass 1)
+  float* mem_scale;           // [S][2][C][H]
 };
 
 struct AppendParams {
   int S, b, R, slot0;         // states, frames, ring frames, ring slot of frame 0
   int64_t frame_elems;        // T * H * D
+  // fp8 format
+  int H, D;
+  unsigned int* amax;         // [S][2][b][H] fp32 bit patterns (scratch, zeroed before the amax pass)
+  uint8_t* ring8[2];          // e4m3 K, V rings
+  float* ring_scale;          // [S][2][R][H]
+  void* stage[2];             // bf16 K, V current-block staging [S][stage_frames*T][H][D]
+  int stage_frames;           // frames per state in the staging buffers (max block)
 };
 
 // Kernel launchers (return cudaError_t of the launch).
@@ -68,8 +83,10 @@ int launch_permute_weights(const void* src, void* dst, int S, int H, int D, cuda
 int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const CUtensorMap& ringV,
                      const CUtensorMap& wmap, cudaStream_t s);
 int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s);
+int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
+int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s);
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k,
-                  const CUtensorMap* v, int S, cudaStream_t s);
+                  const CUtensorMap* v, int S, bool fp8, cudaStream_t s);
 size_t attend_smem_bytes(int D, const AttnParams& p);
 size_t conv_smem_bytes(int D);
 

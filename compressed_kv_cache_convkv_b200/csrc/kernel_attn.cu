@@ -51,7 +51,7 @@ struct AttnCfg {
   static constexpr int REG_LAUNCH = 128, REG_CTRL = 96, REG_ROPE = 80, REG_SOFTMAX = 168;
   static_assert(128 * REG_CTRL + 128 * REG_ROPE + 256 * REG_SOFTMAX == THREADS * REG_LAUNCH,
                 "register split must add up to the launch allocation");
-  static constexpr int NBARS = 1 + 1 + 3 * KST + 2 * VST + 3 * 2 + 1;
+  static constexpr int NBARS = 1 + 1 + 3 * KST + 3 * VST + 3 * 2 + 1;
   static constexpr size_t FIXED =
       1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16 + kMaxSegs * sizeof(KeySeg);
 };
@@ -101,7 +101,58 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int row, const float2* c
   }
 }
 
-template <int D>
+// Two e4m3 codes (low byte first) -> two fp32 values (exact).
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// Dequantise one e4m3 row (D codes at src, scale s) to bf16 value x*s, rotate it
+// (ROTATE) and store it as row `row` of a 128-byte-swizzled bf16 tile.  Rows
+// past the segment store zeros (valid == false) so masked columns stay finite.
+template <int D, bool ROTATE>
+__device__ __forceinline__ void dequant_row(uint8_t* tile, int row, const uint8_t* src, float sc, bool valid,
+                                            const float2* cs_t, const float2* cs_h, const float2* cs_w) {
+  using C = AttnCfg<D>;
+  uint8_t* rowp = tile + row * 128;
+  const int sw = row & 7;
+  uint4 raw[D / 16];
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) raw[k] = valid ? __ldg(reinterpret_cast<const uint4*>(src) + k) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {  // two bf16 chunks of 8 channels
+      const int c = 2 * k + u;
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t word = w[2 * u + (q >> 1)];
+        float a, b;
+        e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
+        a *= sc;
+        b *= sc;
+        if (ROTATE) {
+          const int pi = 4 * c + q;
+          const float2 cs = pi < C::PT ? __ldg(&cs_t[pi])
+                                       : (pi < C::PT + C::PH ? __ldg(&cs_h[pi - C::PT]) : __ldg(&cs_w[pi - C::PT - C::PH]));
+          const float ra = a * cs.x - b * cs.y;
+          const float rb = a * cs.y + b * cs.x;
+          a = ra;
+          b = rb;
+        }
+        o[q] = pack_bf16x2(a, b);
+      }
+      const int bx = c >> 3, cc = c & 7;
+      *reinterpret_cast<uint4*>(rowp + bx * C::BOX + ((cc ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+template <int D, bool FP8>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                 const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
@@ -124,7 +175,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint64_t* s_full = v_empty + C::VST;   // [2]
   uint64_t* p_full = s_full + 2;         // [2]
   uint64_t* o_full = p_full + 2;         // [2]
-  uint64_t* drain = o_full + 2;
+  uint64_t* v_ready = o_full + 2;        // [VST] fp8: V tile dequantised by warps 2-3
+  uint64_t* drain = v_ready + C::VST;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   KeySeg* seg = reinterpret_cast<KeySeg*>(tmem_slot + 4);
@@ -148,6 +200,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     for (int i = 0; i < C::VST; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+      mbar_init(&v_ready[i], 64);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -189,17 +242,25 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int row = sg.row0 + cur.jt * C::BN;
         const int ks = j % C::KST;
         if (j >= C::KST && !mbar_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(&k_full[ks], C::TILE);
+        if (FP8 && sg.fp8) {
+          mbar_arrive(&k_full[ks]);  // stage free: the RoPE warpgroup loads and dequantises it
+        } else {
+          mbar_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap(sg.buf), &k_full[ks], bx * 64, head, row, state);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap(sg.buf), &k_full[ks], bx * 64, head, row, state);
+        }
         ++kiss[ks];
         const int vs = j % C::VST;
         if (j >= C::VST && !mbar_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(&v_full[vs], C::TILE);
+        if (FP8 && sg.fp8) {
+          mbar_arrive(&v_full[vs]);  // stage free: warps 2-3 load and dequantise it
+        } else {
+          mbar_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap(sg.buf), &v_full[vs], bx * 64, head, row, state);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap(sg.buf), &v_full[vs], bx * 64, head, row, state);
+        }
         ++viss[vs];
       }
       // drain: every issued copy must land before the CTA exits
@@ -252,7 +313,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         bool ok = true;
         for (int j = 0; j < p.ntiles && ok; ++j) {
           const int vs = j % C::VST;
-          if (!mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(FP8 ? &v_ready[vs] : &v_full[vs], (j / C::VST) & 1, abort_flag)) { ok = false; break; }
           const bool has_next = j + 1 < p.ntiles;
           const int ksn = (j + 1) % C::KST;
           for (int i = 0; i < 2; ++i) {
@@ -281,7 +342,39 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         mbar_wait(drain, 0, &no_abort);
       }
     }
-  }  // warps 2, 3: no role
+  } else if (FP8 && (warp == 2 || warp == 3)) {
+      // ---------------------------------------------------------- V dequantisation
+      const int r0 = (warp - 2) * 32 + lane;  // rows r0 and r0 + 64 of each V tile
+      TileCursor cur;
+      for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
+        const int vs = j % C::VST;
+        if (!mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag)) break;
+        const KeySeg& sg = seg[cur.s];
+        if (sg.fp8) {
+          const uint8_t* base = p.ring8[1];
+          const float* scl = p.ring_scale;
+          int nsl = p.R;
+          if (sg.buf == 1) {
+            base = p.mem8[1];
+            scl = p.mem_scale;
+            nsl = p.C;
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r = r0 + 64 * u;
+            const int lr = cur.jt * C::BN + r;
+            const bool valid = lr < sg.nrows;
+            const int f = valid ? lr / p.T : 0;
+            const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
+            const float sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
+            dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, nullptr, nullptr,
+                                  nullptr);
+          }
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(&v_ready[vs]);
+      }
+  }
   } else if (warp < 12) {
     regs_inc<C::REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
@@ -410,12 +503,26 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
       const KeySeg& sg = seg[cur.s];
       const int lr = cur.jt * C::BN + r;
-      if (lr < sg.nrows) {
-        const int f = lr / p.T;
-        const int s = lr - f * p.T;
-        const int t = sg.t0 + f;
-        const int y = s / p.grid_w;
-        const int x = s - y * p.grid_w;
+      const bool valid = lr < sg.nrows;
+      const int f = valid ? lr / p.T : 0;
+      const int s = valid ? lr - f * p.T : 0;
+      const int t = sg.t0 + f;
+      const int y = s / p.grid_w;
+      const int x = s - y * p.grid_w;
+      if (FP8 && sg.fp8) {
+        const uint8_t* base = p.ring8[0];
+        const float* scl = p.ring_scale;
+        int nsl = p.R;
+        if (sg.buf == 1) {
+          base = p.mem8[0];
+          scl = p.mem_scale;
+          nsl = p.C;
+        }
+        const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
+        const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
+        dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, tab_t + t * C::PT,
+                             tab_h + y * C::PH, tab_w + x * C::PW);
+      } else if (valid) {
         rope_row<D, false>(sK + ks * C::TILE, r, tab_t + t * C::PT, tab_h + y * C::PH, tab_w + x * C::PW, 1.0f);
       }
       fence_proxy_async_smem();
@@ -440,11 +547,11 @@ size_t smem_for(const AttnParams&) {
   return C::FIXED > 120 * 1024 ? C::FIXED : 120 * 1024;
 }
 
-template <int D>
+template <int D, bool FP8>
 int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v, int S,
              cudaStream_t s) {
   const size_t smem = smem_for<D>(p);
-  auto kern = attn_kernel<D>;
+  auto kern = attn_kernel<D, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid((p.Nq + 255) / 256, p.H, S);
@@ -457,9 +564,9 @@ int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, co
 size_t attend_smem_bytes(int D, const AttnParams& p) { return D == 128 ? smem_for<128>(p) : smem_for<64>(p); }
 
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v,
-                  int S, cudaStream_t s) {
-  if (D == 128) return launch_t<128>(p, q, k, v, S, s);
-  if (D == 64) return launch_t<64>(p, q, k, v, S, s);
+                  int S, bool fp8, cudaStream_t s) {
+  if (D == 128) return fp8 ? launch_t<128, true>(p, q, k, v, S, s) : launch_t<128, false>(p, q, k, v, S, s);
+  if (D == 64) return fp8 ? launch_t<64, true>(p, q, k, v, S, s) : launch_t<64, false>(p, q, k, v, S, s);
   return static_cast<int>(cudaErrorInvalidValue);
 }
 

@@ -95,6 +95,88 @@ __global__ void mean_bf16_kernel(const uint4* __restrict__ ringK, const uint4* _
   }
 }
 
+// ---------------------------------------------------------------------------
+// Append in the fp8 format (model card, --fp8_kv_cache: the cache is stored in
+// FP8 and dequantised to BF16 on use).  Per (state, K|V, frame, head):
+//   scale = amax / 448 over the frame's [T, D] values (1 if amax == 0),
+//   code  = e4m3(x / scale), IEEE fp32 divide, round-to-nearest-even, saturating.
+// The block's bf16 values are also copied to staging: the current block is
+// attended in bf16 and joins the window, e4m3, at the next append.
+
+// pass 1: amax.  grid = (row splits, frames, states * 2), one block reduces a
+// slice of rows per head in shared memory, then one atomicMax per head.
+__global__ void append_amax_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p,
+                                   int rows_per_block) {
+  extern __shared__ unsigned int sh_amax[];
+  const int f = blockIdx.y;
+  const int kv = blockIdx.z & 1, s = blockIdx.z >> 1;
+  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
+  for (int h = threadIdx.x; h < p.H; h += blockDim.x) sh_amax[h] = 0;
+  __syncthreads();
+  const int vec_per_row = p.H * p.D / 8;
+  const int r0 = blockIdx.x * rows_per_block;
+  const int r1 = min(T, r0 + rows_per_block);
+  const uint4* src = (kv ? v : k) + (static_cast<int64_t>(s) * p.b + f) * (p.frame_elems / 8);
+  for (int64_t i = static_cast<int64_t>(r0) * vec_per_row + threadIdx.x; i < static_cast<int64_t>(r1) * vec_per_row;
+       i += blockDim.x) {
+    const uint4 x = __ldg(src + i);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
+      m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
+    }
+    const int h = static_cast<int>((i % vec_per_row) * 8 / p.D);
+    atomicMax(&sh_amax[h], m);
+  }
+  __syncthreads();
+  for (int h = threadIdx.x; h < p.H; h += blockDim.x)
+    if (sh_amax[h]) atomicMax(&p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h], sh_amax[h]);
+}
+
+// pass 2: quantise into the ring, copy to staging, record the scales.
+__global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
+  const int64_t fv = p.frame_elems / 8;
+  const int64_t per_kv = static_cast<int64_t>(p.S) * p.b * fv;
+  const int64_t total = 2 * per_kv;
+  const int vec_per_row = p.H * p.D / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int kv = static_cast<int>(i / per_kv);
+    const int64_t iv = i - kv * per_kv;       // vector index within [S][b*T][H][D]
+    const int64_t sf = iv / fv;               // s * b + f
+    const int64_t e = iv - sf * fv;
+    const int s = static_cast<int>(sf / p.b);
+    const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
+    const int h = static_cast<int>((e % vec_per_row) * 8 / p.D);
+    const uint4 x = __ldg((kv ? v : k) + iv);
+    reinterpret_cast<uint4*>(p.stage[kv])[(static_cast<int64_t>(s) * p.stage_frames + f) * fv + e] = x;
+    const float amax = __uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]);
+    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint16_t lo, hi;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+          : "=h"(lo)
+          : "f"(__fdiv_rn(__uint_as_float(w[2 * q] & 0xFFFF0000u), scale)),
+            "f"(__fdiv_rn(__uint_as_float(w[2 * q] << 16), scale)));
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+          : "=h"(hi)
+          : "f"(__fdiv_rn(__uint_as_float(w[2 * q + 1] & 0xFFFF0000u), scale)),
+            "f"(__fdiv_rn(__uint_as_float(w[2 * q + 1] << 16), scale)));
+      o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    int slot = p.slot0 + f;
+    if (slot >= p.R) slot -= p.R;
+    reinterpret_cast<uint2*>(p.ring8[kv])[(static_cast<int64_t>(s) * p.R + slot) * fv + e] = make_uint2(o[0], o[1]);
+    if (e < vec_per_row && (e * 8) % p.D == 0)  // first vector of head h in token 0 of the frame
+      p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
+  }
+}
+
 }  // namespace
 
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
@@ -118,6 +200,21 @@ int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* 
   mean_bf16_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(ringK),
                                                         static_cast<const uint4*>(ringV), static_cast<uint4*>(p.memK),
                                                         static_cast<uint4*>(p.memV), p, frame_vecs);
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(unsigned int) * p.S * 2 * p.b * p.H, s);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
+  const int rows_per_block = 64;
+  dim3 g1((T + rows_per_block - 1) / rows_per_block, p.b, p.S * 2);
+  append_amax_kernel<<<g1, 256, p.H * sizeof(unsigned int), s>>>(static_cast<const uint4*>(k),
+                                                                 static_cast<const uint4*>(v), p, rows_per_block);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  const int64_t total = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
+  append_quant_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }
 

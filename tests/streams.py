@@ -111,3 +111,40 @@ def check_slot(gpu: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
     e = {"max_rel": float(rel.max()), "mean": float(d.mean())}
     assert e["max_rel"] <= SLOT_MAX_REL and e["mean"] <= SLOT_MEAN, (what, e)
     return e
+
+
+def e4m3_bytes_to_f64(b: np.ndarray) -> np.ndarray:
+    """Values of e4m3 codes (uint8 bit patterns)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+E4M3_CODE_MISMATCH = 1e-3   # fraction of conv-output codes allowed to sit one step apart
+
+
+def check_codes(gpu_bytes: np.ndarray, gpu_scales: np.ndarray, ref_codes: np.ndarray, ref_scales: np.ndarray,
+                exact: bool, what: str = "") -> dict:
+    """e4m3 codes and per-head scales against the oracle's.
+
+    exact: bit-exact (quantised from identical bf16 inputs with the same fp32
+    arithmetic).  Otherwise (quantised conv outputs, fp32 accumulation on the GPU
+    against fp64 in the oracle): scales within 1e-5 relative, codes equal except
+    for a small fraction one quantisation step apart (values next to a rounding
+    boundary)."""
+    g = e4m3_bytes_to_f64(gpu_bytes)
+    if exact:
+        assert np.array_equal(gpu_scales, ref_scales.astype(np.float32)), (what, "scales")
+        assert np.array_equal(g, ref_codes), (what, "codes", int(np.sum(g != ref_codes)))
+        return {"mismatch": 0.0}
+    rs = np.abs(gpu_scales.astype(np.float64) / ref_scales.astype(np.float64) - 1).max()
+    assert rs <= 1e-5, (what, "scale", rs)
+    diff = g != ref_codes
+    frac = float(diff.mean())
+    assert frac <= E4M3_CODE_MISMATCH, (what, "code mismatch fraction", frac)
+    if diff.any():
+        a = np.abs(ref_codes[diff])
+        _, ex = np.frexp(np.where(a > 0, a, 1.0))
+        step = np.exp2(np.maximum(ex - 1.0, -6.0) - 3.0)      # e4m3 quantum at the reference value
+        assert np.all(np.abs(g[diff] - ref_codes[diff]) <= step * 2 + 1e-30), (what, "code step")
+    return {"mismatch": frac}

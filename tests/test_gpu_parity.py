@@ -10,7 +10,9 @@ import pytest
 
 import seeded_inputs as si
 from compressed_kv_cache_convkv_b200.configs import PRESETS, Workload
-from streams import (attention_errors, bf16_tensor_to_f64, check_attention, check_slot, device_frames,
+from dataclasses import replace
+
+from streams import (attention_errors, bf16_tensor_to_f64, check_attention, check_codes, check_slot, device_frames,
                      device_weights, host_frames, oracle_for, sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -161,3 +163,58 @@ def test_512_stream(torch):
 
 def test_720_stream_ragged(torch):
     _run(torch, PRESETS["720x416"], attend_blocks={1, 3, 12, 13, 27, 38}, rows=64, ring_frames=[0, 5])
+
+
+def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, ring_frames=None):
+    """fp8 format: window codes bit-exact, memory codes within one step, attention <= 5e-2."""
+    ckv = _ckv()
+    weights = device_weights(w, torch)
+    cfg = w.config()
+    h = ckv.ConvKV(cfg, weights)
+    oracles = {s: oracle_for(w, state=s) for s in states}
+    rng = np.random.default_rng(w.seed)
+    R = cfg.ring_frames
+    F = 0
+    for n, b in enumerate(w.block_sizes(), start=1):
+        kd, vd, qd = (device_frames(w, t, F, b, torch) for t in (si.K, si.V, si.Q))
+        h.append(kd, vd)
+        out = h.attend(qd)
+        for s, st in oracles.items():
+            kh, vh, qh = (host_frames(w, t, s, F, b) for t in (si.K, si.V, si.Q))
+            ev = st.append(si.bf16_bits_to_f64(kh), si.bf16_bits_to_f64(vh))
+            if s == states[0]:
+                lay = h.layout()
+                assert [tuple(r) for r in lay[:, [0, 1, 3]]] == [tuple(r) for r in st.layout()], f"block {n}"
+                assert [int(x) for x in lay[lay[:, 0] == 2, 2]] == list(range(b))  # staging slots
+            # the new block's e4m3 ring codes and scales: bit-exact
+            frames = range(b) if ring_frames is None else [x for x in ring_frames if x < b]
+            for f in frames:
+                ck, sk, cv, sv = st.current_q8[f].codes
+                for kv, (rc, rsc) in enumerate(((ck, sk), (cv, sv))):
+                    gb, gs = h.read_ring(s, kv, (F + f) % R)
+                    check_codes(gb, gs, rc, rsc, exact=True, what=f"state {s} frame {F + f} kv {kv}")
+            # new memory slots: codes within one step of the oracle's
+            for e in ev[-cfg.mem_slots:]:
+                age = st.m - (st.S - e.slot)
+                ck, sk, cv, sv = st.memory[age].codes
+                for kv, (rc, rsc) in enumerate(((ck, sk), (cv, sv))):
+                    gb, gs = h.read_slot(s, kv, e.slot % cfg.mem_slots)
+                    check_codes(gb, gs, rc, rsc, exact=False, what=f"state {s} slot {e.slot} kv {kv}")
+            if attend_blocks is None or n in attend_blocks:
+                r = sample_rows(w, b, rows or b * w.T, rng)
+                ref, _ = st.attend(si.bf16_bits_to_f64(qh), rows=r)
+                gpu = bf16_tensor_to_f64(out[s][torch.as_tensor(r, device="cuda")])
+                check_attention(gpu, ref, fp8=True, what=f"{w.name} state {s} block {n}")
+        F += b
+    assert h.status() == 0
+    h.close()
+
+
+def test_tiny_fp8_two_states(torch):
+    w = replace(PRESETS["tiny"], fp8=True, num_states=2, name="tiny_fp8")
+    _run_fp8(torch, w, states=(0, 1))
+
+
+def test_fp8_480x832_40_states(torch):
+    _run_fp8(torch, PRESETS["fp8_480x832"], states=(0, 39), attend_blocks={1, 2, 5, 9, 17, 25}, rows=32,
+             ring_frames=[0, 7])
