@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_HERE, "lib", "libconvkv.so")
 
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_BAD_ORDER, ERR_OOM, ERR_CUDA, ERR_DEVICE_TIMEOUT = -1, -2, -3, -4, -5, -6
+ERR_SCRATCH_LIMIT = -7
+NOALLOC_MAX_FRAME_HEADS = 4096
 KV_BF16, KV_FP8_E4M3 = 0, 1
 COMPRESS_CONV, COMPRESS_MEAN = 0, 1
 FLAG_DRY_RUN, FLAG_HOST_IO = 1, 2
@@ -43,6 +45,8 @@ _SIGNATURES = {
     "convkv_launch_count": (ctypes.c_int64, [_P]),
     "convkv_last_cuda_error": (ctypes.c_int, [_P]),
     "convkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "convkv_quantize_e4m3_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int, _P]),
 }
 
 
@@ -87,6 +91,23 @@ def _lib():
 def library():
     """The loaded ctypes library (raises if it is not built)."""
     return _lib()
+
+
+def quantize_e4m3_noalloc(x, codes, scales, stream=None) -> None:
+    """e4m3 codes and per-(frame, head) scales of bf16 frames x[frames, tokens, heads, head_dim],
+    written into the caller's `codes` (uint8, same shape) and `scales` (float32 [frames, heads]),
+    without any device allocation (for callers that cannot allocate while they run).  Calls that
+    overlap on the GPU share one fixed scratch array and race."""
+    import torch
+    f, t, h, d = x.shape
+    if x.dtype != torch.bfloat16 or codes.dtype != torch.uint8 or scales.dtype != torch.float32 or \
+            tuple(codes.shape) != (f, t, h, d) or tuple(scales.shape) != (f, h) or \
+            not (x.is_contiguous() and codes.is_contiguous() and scales.is_contiguous()):
+        raise ValueError("x bf16 [F,T,H,D], codes uint8 [F,T,H,D], scales float32 [F,H], all contiguous")
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    rc = _lib().convkv_quantize_e4m3_noalloc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), f, t, h, d, s)
+    if rc != OK:
+        raise ConvKVError(rc, "convkv_quantize_e4m3_noalloc")
 
 
 @dataclass

@@ -170,6 +170,7 @@ const char* convkv_strerror(int code) {
     case CONVKV_ERR_OOM: return "device allocation failed";
     case CONVKV_ERR_CUDA: return "CUDA error";
     case CONVKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case CONVKV_ERR_SCRATCH_LIMIT: return "request exceeds the fixed scratch area";
     default: return "unknown error";
   }
 }

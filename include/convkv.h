@@ -48,6 +48,7 @@ extern "C" {
 #define CONVKV_ERR_OOM (-4)            /* device allocation failed at create */
 #define CONVKV_ERR_CUDA (-5)           /* a CUDA runtime/driver call failed; see convkv_last_cuda_error */
 #define CONVKV_ERR_DEVICE_TIMEOUT (-6) /* a kernel gave up waiting on a barrier and returned early */
+#define CONVKV_ERR_SCRATCH_LIMIT (-7)  /* request larger than a fixed scratch area (no-allocation entry point) */
 
 #define CONVKV_KV_BF16 0               /* cache stored in bf16 */
 #define CONVKV_KV_FP8_E4M3 1           /* window + memory stored e4m3 with per-(head, frame) fp32 scale */
@@ -156,6 +157,36 @@ int convkv_last_cuda_error(const convkv_t* h);
 
 /* Static description of an error code. */
 const char* convkv_strerror(int code);
+
+/* ------------------------------------------------------------------------
+ * Allocation-free quantiser.  The paper has no counterpart of this call; it
+ * exists for callers that cannot allocate device memory while they run -- a
+ * serving engine that hands out every device byte from its own fixed pool, or
+ * a thread on a latency-critical path where cudaMalloc would synchronise the
+ * device and stall its other streams.
+ *
+ * Quantises `frames` bf16 frames x [frames][tokens][heads][head_dim] (DEVICE)
+ * to e4m3 exactly as the fp8 append does (per frame and head: scale =
+ * amax / 448, 1 if amax is 0; code = e4m3(x / scale), IEEE fp32 divide,
+ * round-to-nearest-even, saturating to +-448) and writes the codes to `codes`
+ * (DEVICE, same layout, 1 byte each) and the scales to `scales` (DEVICE fp32
+ * [frames][heads]), asynchronously on `stream` (cudaStream_t, NULL = legacy
+ * default).  The caller owns all three buffers.
+ *
+ * No device memory is allocated: the only scratch, one amax per (frame, head),
+ * is a fixed array of CONVKV_NOALLOC_MAX_FRAME_HEADS entries (16 KiB) inside
+ * the library, kept on every GPU that loads the library until the process
+ * exits.  frames * heads above that limit returns CONVKV_ERR_SCRATCH_LIMIT.
+ * The first call on a device resolves the array's address there (with that
+ * device current); make that first call before any stream capture.  Every call
+ * shares the array and it keeps the last call's contents (each call clears the
+ * part it uses), so calls whose work overlaps on the GPU -- on different
+ * streams, or from several host threads at once -- race and give wrong results.
+ * head_dim must be a multiple of 8.  Errors: INVALID_ARG, SCRATCH_LIMIT,
+ * UNSUPPORTED (device ordinal >= 128), CUDA. */
+#define CONVKV_NOALLOC_MAX_FRAME_HEADS 4096
+int convkv_quantize_e4m3_noalloc(const void* x, void* codes, float* scales, int frames, int tokens, int heads,
+                                 int head_dim, void* stream);
 
 #ifdef __cplusplus
 }
