@@ -39,6 +39,33 @@ def attention_flops(Nq, Nk, D, H, S=1):
     return 4.0 * Nq * Nk * D * H * S
 
 
+def attention_bytes(Nq, Nk, D, H, S=1, kv_bytes=2):
+    """Algorithmic HBM bytes of one attend: Q and O (bf16) plus every key's K and V."""
+    return (2.0 * Nq * H * D * 2 + 2.0 * Nk * H * D * kv_bytes) * S
+
+
+def measured_traffic(algorithmic_bytes):
+    """DRAM bytes per attention launch from the committed ncu capture, scaled to this
+    launch's algorithmic bytes; None when the kernel sources changed since the capture."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "attn_kernel_512x512.md")
+    src = os.path.join(ROOT, "compressed_kv_cache_convkv_b200", "csrc")
+    if not os.path.exists(prof):
+        return None
+    fields = {}
+    for line in open(prof):
+        if ":" in line and line.split(":")[0] in ("source_sha256", "dram_bytes_per_launch",
+                                                  "algorithmic_bytes_per_launch"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    h = hashlib.sha256()
+    for f in ("kernel_attn.cu", "sm100.cuh", "convkv_internal.h"):
+        h.update(open(os.path.join(src, f), "rb").read())
+    if fields.get("source_sha256") != h.hexdigest():
+        return None
+    return float(fields["dram_bytes_per_launch"]) / float(fields["algorithmic_bytes_per_launch"]) * algorithmic_bytes
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 def oracle_sample(w, rows: int, seed_offset: int = 0):
@@ -305,6 +332,8 @@ def run_ours(args, w):
     att_avg_ms = statistics.mean(att_ms)
     att_achieved = statistics.mean(flops) / (att_avg_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
+    att_bytes = attention_bytes(b * T, statistics.mean(nk_list), D, H, S)
+    traffic = measured_traffic(att_bytes)
     frames_per_s = K * b * S * world / (total_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -321,8 +350,11 @@ def run_ours(args, w):
         "kernels_ms": {"attend_avg": att_avg_ms, "append_compress_avg": (total_ms - sum(att_ms)) / K,
                        "conv_groups_per_step": groups / K},
         "roofline": {"bound": "tensor", "achieved": att_achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": att_achieved / peak, "traffic": None,
-                     "kernel": "attn_kernel<128>", "peak_source": f"{kind} bf16 burst (MEASURED_PEAKS.json)"},
+                     "frac": att_achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes": att_bytes, "kernel": "attn_kernel<128>",
+                     "peak_source": f"{kind} bf16 burst (MEASURED_PEAKS.json)",
+                     "traffic_source": "ncu dram__bytes_read+write of one launch (profiles/attn_kernel_512x512.md), "
+                                       "scaled by algorithmic bytes; null if the kernel changed since"},
         "e2e": {"value": e2e_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 3 * S * b * fe * 2, "d2h_bytes_per_step": S * b * fe * 2},
         "gpu_launches": launches,
