@@ -207,6 +207,7 @@ def run_ours(args, w):
     import seeded_inputs as si
     import compressed_kv_cache_convkv_b200 as ckv
     from compressed_kv_cache_convkv_b200 import build
+    from compressed_kv_cache_convkv_b200.sharding import max_over_ranks
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -291,10 +292,7 @@ def run_ours(args, w):
     launches = h.launch_count() - launches0
     total_ms = start.elapsed_time(end)
     att_ms = [a.elapsed_time(bb) for a, bb in ev]
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     clocks = clk.summary()
 
     # end to end through the host-buffer entry points: pinned host q/k/v in, host out back, every step
@@ -320,10 +318,7 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
     assert h.status() == 0, "device status reported an error"
 
     pk, kind = peaks()

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "convkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "convkv_quantize_e4m3_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_int, _P]),
+    "convkv_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
 }
 
 

@@ -48,13 +48,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // CTA-wide abort flag) when the budget runs out or another thread already
 // aborted; callers then skip the rest of their work but still reach the
 // kernel's final barrier, so the CTA always ends.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long budget_clocks = kWaitBudgetClocks) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (*abort_flag) return false;
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitBudgetClocks) {
+    if (clock64() - t0 > budget_clocks) {
       *abort_flag = 1;
       return false;
     }

@@ -152,6 +152,15 @@ int convkv_status(convkv_t* h);
 /* Number of kernels this handle has launched so far. */
 int64_t convkv_launch_count(const convkv_t* h);
 
+/* Self-test of the bounded device waits (failure detection): launches one CTA
+ * that waits on a barrier nothing arrives on, with a budget of budget_clocks SM
+ * clocks (1000 .. 2e9).  The wait gives up, the kernel writes the timeout code
+ * to *dev_status (DEVICE int, caller-owned, zero on entry) and returns; the
+ * call synchronises `stream` and returns CONVKV_ERR_DEVICE_TIMEOUT -- the
+ * expected result -- or CONVKV_OK if the wait somehow completed.  The context
+ * stays usable.  Errors: INVALID_ARG, CUDA. */
+int convkv_selftest_wait_timeout(int* dev_status, long long budget_clocks, void* stream);
+
 /* cudaError_t of the last failing CUDA call made through this handle (0 if none). */
 int convkv_last_cuda_error(const convkv_t* h);
 

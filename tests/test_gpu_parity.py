@@ -40,6 +40,23 @@ def test_device_generator_matches_host(torch):
     assert np.array_equal(d.view(torch.int16).cpu().numpy().view(np.uint16), h)
 
 
+def test_bounded_wait_reports_timeout_and_context_survives(torch):
+    """A kernel whose barrier never completes gives up after its budget (~10 ms here),
+    reports CONVKV_ERR_DEVICE_TIMEOUT through the status word, and the context keeps
+    working (the tiny stream still matches the oracle afterwards)."""
+    import time
+    ckv = _ckv()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    rc = ckv.library().convkv_selftest_wait_timeout(status.data_ptr(), 20_000_000,
+                                                    torch.cuda.current_stream().cuda_stream)
+    assert rc == ckv.ERR_DEVICE_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert int(status.item()) != 0
+    assert ckv.library().convkv_selftest_wait_timeout(status.data_ptr(), 10, 0) == ckv.ERR_INVALID_ARG
+    _run(torch, PRESETS["tiny"], max_blocks=5)
+
+
 def _run(torch, w: Workload, attend_blocks=None, rows=None, compress=0, t_offset=0, override=None,
          check_slots=True, ring_frames=None, max_blocks=None, collect=None, sharp=False):
     """Stream w through both sides; returns per-block error records."""
