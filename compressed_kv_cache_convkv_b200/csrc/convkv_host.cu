@@ -62,7 +62,7 @@ struct convkv {
   float *ring_scale = nullptr, *mem_scale = nullptr;
   void *stageK = nullptr, *stageV = nullptr;  // bf16 copy of the current block
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
-  float2* tables = nullptr;
+  float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
   CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{};
@@ -133,28 +133,40 @@ int validate(const convkv_cfg* c) {
   // TMA coordinates and row counts are 32-bit
   if (T * (R > c->mem_slots ? R : c->mem_slots) > (int64_t(1) << 30) || T * Bmax > (int64_t(1) << 30))
     return CONVKV_ERR_UNSUPPORTED;
-  const int64_t tabs = (int64_t(c->mem_slots) + c->window_frames + Bmax) * (D - 2 * dh) / 2 +
-                       (int64_t(c->grid_h) + c->grid_w) * dh / 2;
-  if (tabs * 8 > 32 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables must fit in shared memory
+  const int pt = rope_pairs_t(D), ph = rope_pairs_h(D);
+  const int64_t tab_units = (int64_t(c->mem_slots) + c->window_frames + Bmax) * rope_units(0, pt) +
+                            int64_t(c->grid_h) * rope_units(pt, ph) + int64_t(c->grid_w) * rope_units(pt + ph, ph);
+  if (tab_units * 16 > 256 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables stay cache-resident
   if (c->kv_format == CONVKV_KV_FP8_E4M3 && c->compress_mode == CONVKV_COMPRESS_MEAN) return CONVKV_ERR_UNSUPPORTED;
   if (c->compress_mode == CONVKV_COMPRESS_CONV && !(c->flags & CONVKV_FLAG_DRY_RUN) && !c->conv_weight)
     return CONVKV_ERR_INVALID_ARG;
   return CONVKV_OK;
 }
 
-void build_tables(const convkv* h, std::vector<float2>& out) {
-  // rows of (cos, sin) for pair i of an axis with 2*npairs channels: angle = pos * theta^(-2i/(2*npairs))
-  auto axis = [&](int rows, int npairs, int offset) {
+void build_tables(const convkv* h, std::vector<float4>& out) {
+  // axis with global pairs [g, g + n), positions 0..rows-1 (+offset): for pair i of the
+  // axis the angle is pos * theta^(-2i/(2n)); units pack the pairs 2k, 2k+1 as
+  // (cos, cos, sin, sin), zero for a pair outside the axis
+  auto axis = [&](int rows, int g, int n, int offset) {
+    const int units = rope_units(g, n);
     for (int r = 0; r < rows; ++r)
-      for (int i = 0; i < npairs; ++i) {
-        const double freq = std::pow(h->cfg.rope_theta, -2.0 * i / (2.0 * npairs));
-        const double ang = static_cast<double>(r + offset) * freq;
-        out.push_back(make_float2(static_cast<float>(std::cos(ang)), static_cast<float>(std::sin(ang))));
+      for (int u = 0; u < units; ++u) {
+        float c[2] = {0.f, 0.f}, sn[2] = {0.f, 0.f};
+        for (int q = 0; q < 2; ++q) {
+          const int gp = 2 * (g / 2 + u) + q;  // global pair
+          if (gp < g || gp >= g + n) continue;
+          const int i = gp - g;
+          const double freq = std::pow(h->cfg.rope_theta, -2.0 * i / (2.0 * n));
+          const double ang = static_cast<double>(r + offset) * freq;
+          c[q] = static_cast<float>(std::cos(ang));
+          sn[q] = static_cast<float>(std::sin(ang));
+        }
+        out.push_back(make_float4(c[0], c[1], sn[0], sn[1]));
       }
   };
-  axis(h->tab_t_rows, h->PT, h->cfg.t_offset);
-  axis(h->gh, h->PH, 0);
-  axis(h->gw, h->PW, 0);
+  axis(h->tab_t_rows, 0, h->PT, h->cfg.t_offset);
+  axis(h->gh, h->PT, h->PH, 0);
+  axis(h->gw, h->PT + h->PH, h->PW, 0);
 }
 
 }  // namespace
@@ -220,9 +232,9 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t amax_n = static_cast<size_t>(h->S) * 2 * h->H * (h->Bmax > kMaxGroups ? h->Bmax : kMaxGroups);
   const size_t amax_b = h->fp8 ? amax_n * sizeof(unsigned int) : 0;
   const size_t w_b = h->mean ? 0 : static_cast<size_t>(h->S) * 2 * h->H * kEvict * h->D * h->D * 2;
-  std::vector<float2> tab;
+  std::vector<float4> tab;
   build_tables(h, tab);
-  const size_t tab_b = tab.size() * sizeof(float2);
+  const size_t tab_b = tab.size() * sizeof(float4);
   const size_t io_b = h->host_io ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -248,7 +260,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->memK = a + o_mk;
   h->memV = a + o_mv;
   h->weights = w_b ? a + o_w : nullptr;
-  h->tables = reinterpret_cast<float2*>(a + o_tab);
+  h->tables = reinterpret_cast<float4*>(a + o_tab);
   h->status = reinterpret_cast<int*>(a + o_st);
   if (h->fp8) {
     h->ring_scale = reinterpret_cast<float*>(a + o_rsc);

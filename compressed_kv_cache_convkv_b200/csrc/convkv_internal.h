@@ -12,6 +12,12 @@ constexpr int kEvict = 5;       // eviction group = conv kernel = conv stride (5
 constexpr int kMaxSegs = 6;     // key segments of one attend (memory 2 + ring 2 + staging 1)
 constexpr int kMaxGroups = 16;  // eviction groups one append may compress
 
+// RoPE channel pairs per axis for head_dim D: row and column floor(D/6), time the rest
+__host__ __device__ constexpr int rope_pairs_h(int D) { return D / 6; }
+__host__ __device__ constexpr int rope_pairs_t(int D) { return (D - 4 * (D / 6)) / 2; }
+// 16-byte table units of an axis whose pairs are global pairs [g, g + n)
+__host__ __device__ constexpr int rope_units(int g, int n) { return (g + n + 1) / 2 - g / 2; }
+
 // Device status word values (written by kernels, read by convkv_status()).
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
@@ -33,8 +39,12 @@ struct AttnParams {
   int tq0;                // RoPE time index of the current block's first frame (m + w)
   int nseg, ntiles;
   KeySeg seg[kMaxSegs];
-  int tab_t_rows, tab_h_rows, tab_w_rows;  // rows of the cos/sin tables
-  const float2* tables;   // [t rows][PT] ++ [grid_h][PH] ++ [grid_w][PW] (cos, sin)
+  int tab_t_rows, tab_h_rows, tab_w_rows;  // rows (positions) of the three RoPE tables
+  // RoPE tables, one per axis, rows of 16-byte units: unit u of a row holds
+  // (cos, cos, sin, sin) of the two channel pairs 2k, 2k+1 (k = floor(g/2) + u, g =
+  // the axis' first global pair) that belong to the axis, zeros for a pair that
+  // does not; [t rows][units_t] ++ [grid_h][units_h] ++ [grid_w][units_w]
+  const float4* tables;
   __nv_bfloat16* out;     // [S][Nq][H][D]
   float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
   const float* ring_scale;  // fp8: [S][2][R][H]

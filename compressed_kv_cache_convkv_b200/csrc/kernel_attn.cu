@@ -40,9 +40,15 @@ struct AttnCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int TILE = 128 * D * 2;     // bytes of one 128-row bf16 tile
   static constexpr int BOX = 128 * 128;        // bytes of one 128-row x 64-channel box
-  static constexpr int PT = (D - 4 * (D / 6)) / 2;  // rotation pairs on the time axis
-  static constexpr int PH = D / 6;                  // ... on the row axis
-  static constexpr int PW = D / 6;                  // ... on the column axis
+  static constexpr int PT = rope_pairs_t(D);  // rotation pairs on the time axis
+  static constexpr int PH = rope_pairs_h(D);  // ... on the row axis
+  static constexpr int PW = rope_pairs_h(D);  // ... on the column axis
+  // 16-byte table units per position of each axis
+  static constexpr int UT = rope_units(0, PT), UH = rope_units(PT, PH), UW = rope_units(PT + PH, PW);
+  // axis (0 t, 1 h, 2 w) of global pair p, and the unit that holds it
+  static constexpr int axis_of(int p) { return p < PT ? 0 : (p < PT + PH ? 1 : 2); }
+  static constexpr int axis_start(int a) { return a == 0 ? 0 : (a == 1 ? PT : PT + PH); }
+  static constexpr int unit_of(int p) { return p / 2 - axis_start(axis_of(p)) / 2; }
   static constexpr int O_COL = 256;
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 512;
@@ -67,36 +73,76 @@ struct TileCursor {
   }
 };
 
+// Row pointers into the three RoPE tables for one token position (t, y, x).
+struct RopeRow {
+  const float4* t;
+  const float4* h;
+  const float4* w;
+  __device__ __forceinline__ float4 unit(int axis, int u) const {
+    return __ldg((axis == 0 ? t : (axis == 1 ? h : w)) + u);
+  }
+};
+
+__device__ __forceinline__ uint32_t rot_pair(uint32_t word, float c, float s, float scale, bool do_scale) {
+  const float a = bf16lo_to_f32(word), b = bf16hi_to_f32(word);
+  float ra = a * c - b * s, rb = a * s + b * c;
+  if (do_scale) {
+    ra *= scale;
+    rb *= scale;
+  }
+  return pack_bf16x2(ra, rb);
+}
+
+// Rotate the 8 channels (4 adjacent pairs) of chunk c, held as bf16x2 words, in
+// place.  Two pairs of the same axis go through packed fp32x2 arithmetic with one
+// 16-byte table load; a pair-pair split by an axis boundary is rotated pair by pair.
+template <int D, bool SCALE>
+__device__ __forceinline__ void rope_chunk(uint32_t (&w)[4], int c, const RopeRow& rr, float scale) {
+  using C = AttnCfg<D>;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int p0 = 4 * c + 2 * hh, p1 = p0 + 1;  // p0 is even: slot 0 of its unit
+    if (C::axis_of(p0) == C::axis_of(p1)) {
+      const float4 U = rr.unit(C::axis_of(p0), C::unit_of(p0));
+      const uint64_t cc = f2_make(U.x, U.y), ss = f2_make(U.z, U.w);
+      const uint64_t a = f2_make(bf16lo_to_f32(w[2 * hh]), bf16lo_to_f32(w[2 * hh + 1]));
+      const uint64_t b = f2_make(bf16hi_to_f32(w[2 * hh]), bf16hi_to_f32(w[2 * hh + 1]));
+      uint64_t ra = f2_sub(f2_mul(a, cc), f2_mul(b, ss));
+      uint64_t rb = f2_fma(a, ss, f2_mul(b, cc));
+      if (SCALE) {
+        const uint64_t sc = f2_make(scale, scale);
+        ra = f2_mul(ra, sc);
+        rb = f2_mul(rb, sc);
+      }
+      float ra0, ra1, rb0, rb1;
+      f2_split(ra, ra0, ra1);
+      f2_split(rb, rb0, rb1);
+      w[2 * hh] = pack_bf16x2(ra0, rb0);
+      w[2 * hh + 1] = pack_bf16x2(ra1, rb1);
+    } else {
+      const float4 U0 = rr.unit(C::axis_of(p0), C::unit_of(p0));
+      const float4 U1 = rr.unit(C::axis_of(p1), C::unit_of(p1));
+      w[2 * hh] = rot_pair(w[2 * hh], U0.x, U0.z, scale, SCALE);
+      w[2 * hh + 1] = rot_pair(w[2 * hh + 1], U1.y, U1.w, scale, SCALE);
+    }
+  }
+}
+
 // Rotate one 128-byte-swizzled row of a tile in place: adjacent channel pairs
 // (2i, 2i+1) of each axis segment [t | h | w] turn by the tabulated angle.
 // The swizzle permutes 16-byte chunks only, and a pair never straddles a
 // chunk, so the rotation is independent of it.
 template <int D, bool SCALE>
-__device__ __forceinline__ void rope_row(uint8_t* tile, int row, const float2* cs_t, const float2* cs_h,
-                                         const float2* cs_w, float scale) {
+__device__ __forceinline__ void rope_row(uint8_t* tile, int row, const RopeRow& rr, float scale) {
   using C = AttnCfg<D>;
   uint8_t* rowp = tile + row * 128;
   const int sw = row & 7;
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) {
-    const int bx = c >> 3, cc = c & 7;
-    uint4* ptr = reinterpret_cast<uint4*>(rowp + bx * C::BOX + ((cc ^ sw) << 4));
+    uint4* ptr = reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4));
     const uint4 v = *ptr;
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int pi = 4 * c + q;
-      const float2 cs = pi < C::PT ? __ldg(&cs_t[pi])
-                                   : (pi < C::PT + C::PH ? __ldg(&cs_h[pi - C::PT]) : __ldg(&cs_w[pi - C::PT - C::PH]));
-      const float a = bf16lo_to_f32(w[q]), b = bf16hi_to_f32(w[q]);
-      float ra = a * cs.x - b * cs.y;
-      float rb = a * cs.y + b * cs.x;
-      if (SCALE) {
-        ra *= scale;
-        rb *= scale;
-      }
-      w[q] = pack_bf16x2(ra, rb);
-    }
+    rope_chunk<D, SCALE>(w, c, rr, scale);
     *ptr = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
@@ -114,7 +160,7 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi
 // past the segment store zeros (valid == false) so masked columns stay finite.
 template <int D, bool ROTATE>
 __device__ __forceinline__ void dequant_row(uint8_t* tile, int row, const uint8_t* src, float sc, bool valid,
-                                            const float2* cs_t, const float2* cs_h, const float2* cs_w) {
+                                            const RopeRow& rr) {
   using C = AttnCfg<D>;
   uint8_t* rowp = tile + row * 128;
   const int sw = row & 7;
@@ -133,21 +179,10 @@ __device__ __forceinline__ void dequant_row(uint8_t* tile, int row, const uint8_
         const uint32_t word = w[2 * u + (q >> 1)];
         float a, b;
         e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
-        a *= sc;
-        b *= sc;
-        if (ROTATE) {
-          const int pi = 4 * c + q;
-          const float2 cs = pi < C::PT ? __ldg(&cs_t[pi])
-                                       : (pi < C::PT + C::PH ? __ldg(&cs_h[pi - C::PT]) : __ldg(&cs_w[pi - C::PT - C::PH]));
-          const float ra = a * cs.x - b * cs.y;
-          const float rb = a * cs.y + b * cs.x;
-          a = ra;
-          b = rb;
-        }
-        o[q] = pack_bf16x2(a, b);
+        o[q] = pack_bf16x2(a * sc, b * sc);  // dequantised to bf16 on use
       }
-      const int bx = c >> 3, cc = c & 7;
-      *reinterpret_cast<uint4*>(rowp + bx * C::BOX + ((cc ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
+      *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
@@ -181,9 +216,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   KeySeg* seg = reinterpret_cast<KeySeg*>(tmem_slot + 4);
   // cos/sin tables stay in global memory and are read through the read-only cache
-  const float2* tab_t = p.tables;
-  const float2* tab_h = tab_t + p.tab_t_rows * C::PT;
-  const float2* tab_w = tab_h + p.tab_h_rows * C::PH;
+  const float4* tab_t = p.tables;
+  const float4* tab_h = tab_t + p.tab_t_rows * C::UT;
+  const float4* tab_w = tab_h + p.tab_h_rows * C::UH;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.y, state = blockIdx.z;
@@ -367,8 +402,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             const int f = valid ? lr / p.T : 0;
             const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
             const float sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-            dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, nullptr, nullptr,
-                                  nullptr);
+            dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid,
+                                  RopeRow{nullptr, nullptr, nullptr});
           }
           fence_proxy_async_smem();
         }
@@ -389,7 +424,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int t = p.tq0 + f;
       const int y = s / p.grid_w;
       const int x = s - y * p.grid_w;
-      rope_row<D, true>(sQ + i * C::TILE, r, tab_t + t * C::PT, tab_h + y * C::PH, tab_w + x * C::PW, p.q_scale);
+      const RopeRow rr{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW};
+      rope_row<D, true>(sQ + i * C::TILE, r, rr, p.q_scale);
     }
     fence_proxy_async_smem();
     mbar_arrive(q_ready);
@@ -509,6 +545,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int t = sg.t0 + f;
       const int y = s / p.grid_w;
       const int x = s - y * p.grid_w;
+      const RopeRow rr{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW};
       if (FP8 && sg.fp8) {
         const uint8_t* base = p.ring8[0];
         const float* scl = p.ring_scale;
@@ -520,10 +557,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
         const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
         const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-        dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, tab_t + t * C::PT,
-                             tab_h + y * C::PH, tab_w + x * C::PW);
+        dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, rr);
       } else if (valid) {
-        rope_row<D, false>(sK + ks * C::TILE, r, tab_t + t * C::PT, tab_h + y * C::PH, tab_w + x * C::PW, 1.0f);
+        rope_row<D, false>(sK + ks * C::TILE, r, rr, 1.0f);
       }
       fence_proxy_async_smem();
       mbar_arrive(&k_ready[ks]);

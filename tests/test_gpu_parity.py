@@ -197,8 +197,9 @@ def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, rin
         h.append(kd, vd)
         out = h.attend(qd)
         for s, st in oracles.items():
-            kh, vh, qh = (host_frames(w, t, s, F, b) for t in (si.K, si.V, si.Q))
+            kh, vh = (host_frames(w, t, s, F, b) for t in (si.K, si.V))
             ev = st.append(si.bf16_bits_to_f64(kh), si.bf16_bits_to_f64(vh))
+            del kh, vh
             if s == states[0]:
                 lay = h.layout()
                 assert [tuple(r) for r in lay[:, [0, 1, 3]]] == [tuple(r) for r in st.layout()], f"block {n}"
@@ -218,6 +219,7 @@ def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, rin
                     gb, gs = h.read_slot(s, kv, e.slot % cfg.mem_slots)
                     check_codes(gb, gs, rc, rsc, exact=False, what=f"state {s} slot {e.slot} kv {kv}")
             if attend_blocks is None or n in attend_blocks:
+                qh = host_frames(w, si.Q, s, F, b)
                 r = sample_rows(w, b, rows or b * w.T, rng)
                 ref, _ = st.attend(si.bf16_bits_to_f64(qh), rows=r)
                 gpu = bf16_tensor_to_f64(out[s][torch.as_tensor(r, device="cuda")])
