@@ -55,7 +55,7 @@ from typing import List, Optional, Sequence, Tuple
 import numpy as np
 
 # Partition codes of a key frame in the attended sequence.
-PART_MEMORY, PART_WINDOW, PART_CURRENT = 0, 1, 2
+PART_MEMORY, PART_WINDOW, PART_CURRENT, PART_SINK = 0, 1, 2, 3
 EVICT = 5          # frames per eviction group = conv kernel = conv stride (5:1)
 E4M3_MAX = 448.0   # largest finite e4m3 value
 
@@ -285,6 +285,15 @@ class OracleStream:
         self.events: List[ConvEvent] = []
         self.mem_scales: List[np.ndarray] = []  # fp8: per-slot [2, H] scales
         self.frame_scales = {}                  # fp8: stream frame -> [2, H] scales
+        self.sink: List[_Frame] = []            # reference-image frames, never evicted
+
+    # -- reference-image partition -------------------------------------------
+    def set_sink(self, k: np.ndarray, v: np.ndarray) -> None:
+        """Reference-image state (SoulX-LiveAct blog, "ConvKV Memory": the context is
+        reference-image state + long-term memory + short-term memory + current block).
+        k, v[n, T, H, D]: kept exact, never evicted or compressed, attended first."""
+        self.sink = [_Frame(np.asarray(k[i], dtype=np.float64), np.asarray(v[i], dtype=np.float64), i)
+                     for i in range(k.shape[0])]
 
     # -- append ------------------------------------------------------------
     def append(self, k: np.ndarray, v: np.ndarray) -> List[ConvEvent]:
@@ -338,9 +347,12 @@ class OracleStream:
 
     # -- layout ------------------------------------------------------------
     def key_frames(self) -> List[Tuple[int, _Frame, int]]:
-        """(partition, frame, RoPE time index) in attended order."""
+        """(partition, frame, RoPE time index) in attended order:
+        [reference image | memory | window | current], time indices from 0."""
         out = []
         t = 0
+        for f in self.sink:
+            out.append((PART_SINK, f, t)); t += 1
         for f in self.memory:
             out.append((PART_MEMORY, f, t)); t += 1
         for f in self.window:
@@ -390,7 +402,7 @@ class OracleStream:
         k_y = np.tile(ky, len(kf))
         k_x = np.tile(kx, len(kf))
         qf, qs = rows // T, rows % T
-        q_t = (self.m + self.w_frames + qf) + t_offset
+        q_t = (len(self.sink) + self.m + self.w_frames + qf) + t_offset
         q_y, q_x = qs // cfg.grid_w, qs % cfg.grid_w
         split = cfg.rope()
         o = np.zeros((len(rows), len(heads), D))

@@ -408,3 +408,39 @@ def test_fp8_stream_window_is_quantised_current_is_exact():
         np.testing.assert_array_equal(sk, st.frame_scales[f.index][0])
         np.testing.assert_array_equal(f.k, O.fp8_dequantize(ck, sk))
         np.testing.assert_array_equal(O.round_to_bf16(f.k), f.k)
+
+
+def test_sink_partition_equals_full_attention_over_concatenated_keys():
+    """With a reference-image partition, the output is the attention over
+    [sink | memory | window | current] with positions 0.. in that order: the same
+    as a stream without sink whose keys are prefixed by the sink frames and whose
+    time indices (queries included) are shifted by the sink length."""
+    H, D, gh, gw = 2, 64, 4, 4
+    T = gh * gw
+    rng = np.random.default_rng(21)
+    cfg = O.OracleConfig(H=H, D=D, grid_h=gh, grid_w=gw, window=4, mem_slots=3)
+    w = rng.standard_normal((2, H, D, D, 5)) / 16
+    st = O.OracleStream(cfg, w)
+    sk, sv = rng.standard_normal((2, T, H, D)), rng.standard_normal((2, T, H, D))
+    st.set_sink(sk, sv)
+    for n in range(7):
+        k, v, q = (rng.standard_normal((2, T, H, D)) for _ in range(3))
+        st.append(k, v)
+    o, ps = st.attend(q)
+    np.testing.assert_allclose(ps, 1.0, atol=1e-12)
+    lay = st.layout()
+    assert list(lay[:2, 0]) == [O.PART_SINK] * 2 and list(lay[:, 2]) == list(range(len(lay)))
+    # independent restatement: rotate with the complex form, SDPA over all key frames
+    kf = st.key_frames()
+    tok = np.arange(T)
+    for h in range(H):
+        kall = np.concatenate([f.k[:, h, :] for _, f, _ in kf])
+        vall = np.concatenate([f.v[:, h, :] for _, f, _ in kf])
+        kt = np.concatenate([np.full(T, t) for _, _, t in kf])
+        kr = _rope_complex(kall, kt, np.tile(tok // gw, len(kf)), np.tile(tok % gw, len(kf)), (24, 20, 20), 1e4)
+        qq = q[:, :, h, :].reshape(-1, D)
+        qt = len(kf) - 2 + np.arange(2 * T) // T
+        qr = _rope_complex(qq, qt, np.tile(tok // gw, 2), np.tile(tok % gw, 2), (24, 20, 20), 1e4)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qr)[None], torch.from_numpy(kr)[None], torch.from_numpy(vall)[None])[0].numpy()
+        np.testing.assert_allclose(o[:, h], ref, atol=1e-12)
