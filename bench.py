@@ -225,7 +225,8 @@ def run_ours(args, w):
         dist.barrier()
 
     S, H, D, T = w.num_states, w.heads, w.head_dim, w.T
-    cfg = w.config(host_io=True)
+    r = args.sink_frames
+    cfg = w.config(host_io=True, sink_frames=r)
     stream = torch.cuda.current_stream()
     fe = T * H * D
     # conv weights and inputs: seeded, generated on the device (each rank its own layer state)
@@ -235,6 +236,15 @@ def run_ours(args, w):
             si.frames_device(weights[s, kv].data_ptr(), w.seed + rank, tid, s, 0, 1, H * D * D * 5,
                              si.weight_scale(D), stream.cuda_stream)
     h = ckv.ConvKV(cfg, weights, stream=stream)
+    if r:
+        # reference-image frames, attended first by every block
+        ref = []
+        for tid in (si.RK, si.RV):
+            x = torch.empty((S, r * T, H, D), dtype=torch.bfloat16, device="cuda")
+            for s in range(S):
+                si.frames_device(x[s].data_ptr(), w.seed + rank, tid, s, 0, r, fe, 1.0, stream.cuda_stream)
+            ref.append(x)
+        h.set_sink(*ref)
     b = w.block_frames
     npool = 3
     pool = []
@@ -281,7 +291,7 @@ def run_ours(args, w):
             q = step(i)
             c = h.counters()
             groups += c["groups"]
-            nk = (c["m"] + c["w"] + c["b"]) * T
+            nk = (r + c["m"] + c["w"] + c["b"]) * T
             nk_list.append(nk)
             flops.append(attention_flops(b * T, nk, D, H, S))
             ev[i][0].record(stream)
@@ -313,7 +323,7 @@ def run_ours(args, w):
     for _ in range(Ke):
         h.append_host(kh, vh)
         c = h.counters()
-        e2e_flops += attention_flops(b * T, (c["m"] + c["w"] + c["b"]) * T, D, H, S)
+        e2e_flops += attention_flops(b * T, (r + c["m"] + c["w"] + c["b"]) * T, D, H, S)
         h.attend_host(qh, oh)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -334,9 +344,10 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
-        "config": {"workload": f"{w.name} steady state (memory full), one layer state per GPU",
+        "config": {"workload": f"{w.name} steady state (memory full), one layer state per GPU"
+                               + (f", {r} reference-image frame(s) attended first" if r else ""),
                    "heads": H, "head_dim": D, "tokens_per_frame": T, "block_frames": b,
-                   "window_frames": w.window_frames, "mem_slots": w.mem_slots, "states": S,
+                   "window_frames": w.window_frames, "mem_slots": w.mem_slots, "reference_frames": r, "states": S,
                    "keys_per_step_avg": statistics.mean(nk_list), "state_bytes": h.state_bytes(),
                    "l2": "inputs larger than L2 (q,k,v 252 MB/step + 671 MB K/V state vs 126 MB L2)",
                    "parallelism": f"replicas x{world} (independent layer states, no collective)"},
@@ -374,6 +385,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="512x512")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sink-frames", type=int, default=0,
+                    help="reference-image frames attended first by every block (default none)")
     args = ap.parse_args()
     from compressed_kv_cache_convkv_b200.configs import PRESETS
     w = PRESETS[args.workload]

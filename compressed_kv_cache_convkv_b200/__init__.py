@@ -33,6 +33,7 @@ _SIGNATURES = {
     "convkv_create": (ctypes.c_int, [_P, ctypes.POINTER(_P)]),
     "convkv_append_block": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     "convkv_attend": (ctypes.c_int, [_P, _P, _P]),
+    "convkv_set_sink": (ctypes.c_int, [_P, _P, _P]),
     "convkv_append_block_host": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     "convkv_attend_host": (ctypes.c_int, [_P, _P, _P]),
     "convkv_state_bytes": (ctypes.c_size_t, [_P]),
@@ -68,7 +69,7 @@ class _CCfg(ctypes.Structure):
         ("rope_h", ctypes.c_int), ("rope_w", ctypes.c_int), ("rope_theta", ctypes.c_double),
         ("kv_format", ctypes.c_int), ("compress_mode", ctypes.c_int), ("num_states", ctypes.c_int),
         ("flags", ctypes.c_int), ("t_offset", ctypes.c_int), ("conv_weight", ctypes.c_void_p),
-        ("stream", ctypes.c_void_p),
+        ("stream", ctypes.c_void_p), ("sink_frames", ctypes.c_int),
     ]
 
 
@@ -130,6 +131,7 @@ class Config:
     dry_run: bool = False
     host_io: bool = False
     t_offset: int = 0
+    sink_frames: int = 0
 
     @property
     def T(self) -> int:
@@ -150,7 +152,7 @@ class Config:
         c = _CCfg()
         for name in ("heads", "head_dim", "grid_h", "grid_w", "first_block_frames", "block_frames",
                      "window_frames", "evict_frames", "mem_slots", "rope_theta", "kv_format", "compress_mode",
-                     "num_states", "t_offset"):
+                     "num_states", "t_offset", "sink_frames"):
             setattr(c, name, getattr(self, name))
         c.rope_t, c.rope_h, c.rope_w = self.rope
         c.flags = (FLAG_DRY_RUN if self.dry_run else 0) | (FLAG_HOST_IO if self.host_io else 0)
@@ -237,6 +239,17 @@ class ConvKV:
             out = torch.empty_like(q)
         self._check(_lib().convkv_attend(self._h, q.data_ptr(), out.data_ptr()), "convkv_attend")
         return out
+
+    def set_sink(self, k, v) -> None:
+        """K/V of the ``sink_frames`` reference frames, attended first by every block and
+        never evicted; bf16 CUDA tensors [num_states, sink_frames*T, H, D]."""
+        if self.cfg.dry_run:
+            self._check(_lib().convkv_set_sink(self._h, None, None), "convkv_set_sink")
+            return
+        fk, fv = self._frames_of(k, "k"), self._frames_of(v, "v")
+        if fk != self.cfg.sink_frames or fv != fk or not (k.is_cuda and v.is_cuda):
+            raise ValueError(f"k, v must be CUDA tensors of {self.cfg.sink_frames} reference frames")
+        self._check(_lib().convkv_set_sink(self._h, k.data_ptr(), v.data_ptr()), "convkv_set_sink")
 
     def append_host(self, k, v) -> None:
         fk = self._frames_of(k, "k")

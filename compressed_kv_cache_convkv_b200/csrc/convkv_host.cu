@@ -8,8 +8,9 @@
 //   append(b): P += b_prev; while P - E > W: compress frames [E, E+5) into slot
 //              S (memory position S mod C), E += 5, S += 1; the new block goes to
 //              ring slots (P + f) mod R with R = W + max(b1, b).
-//   attend:    keys = stored slots S-m .. S-1 (m = min(S, C)) at time 0..m-1,
-//              then frames E .. P+b-1 at time m + (f - E).
+//   attend:    keys = the r reference frames at time 0..r-1 (r = sink_frames, given
+//              once, never evicted), stored slots S-m .. S-1 (m = min(S, C)) at
+//              time r..r+m-1, then frames E .. P+b-1 at time r + m + (f - E).
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -48,9 +49,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct convkv {
   convkv_cfg cfg{};
-  int H = 0, D = 0, T = 0, gh = 0, gw = 0, b1 = 0, bn = 0, Bmax = 0, W = 0, C = 0, R = 0, S = 0;
+  int H = 0, D = 0, T = 0, gh = 0, gw = 0, b1 = 0, bn = 0, Bmax = 0, W = 0, C = 0, R = 0, S = 0, Rs = 0;
   int PT = 0, PH = 0, PW = 0, tab_t_rows = 0;
-  bool dry = false, mean = false, fp8 = false, host_io = false;
+  bool dry = false, mean = false, fp8 = false, host_io = false, sink_set = false;
   // bookkeeping
   int64_t P = 0, E = 0, Sn = 0, blocks = 0;
   int bcur = 0, last_groups = 0;
@@ -61,11 +62,13 @@ struct convkv {
   // fp8 format: ringK/ringV/memK/memV hold e4m3 codes; scales per (state, K|V, slot, head)
   float *ring_scale = nullptr, *mem_scale = nullptr;
   void *stageK = nullptr, *stageV = nullptr;  // bf16 copy of the current block
+  void *sinkK = nullptr, *sinkV = nullptr;    // bf16 reference frames, both formats
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
-  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{};
+  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
+      mapSinkV{};
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
   int last_cuda = 0;
@@ -114,7 +117,7 @@ int validate(const convkv_cfg* c) {
   if (!c) return CONVKV_ERR_INVALID_ARG;
   if (c->heads < 1 || c->head_dim < 1 || c->grid_h < 1 || c->grid_w < 1 || c->first_block_frames < 1 ||
       c->block_frames < 1 || c->window_frames < 4 || c->mem_slots < 1 || c->num_states < 1 ||
-      !(c->rope_theta > 0.0) || c->t_offset < 0)
+      !(c->rope_theta > 0.0) || c->t_offset < 0 || c->sink_frames < 0)
     return CONVKV_ERR_INVALID_ARG;
   if (c->evict_frames != kEvict) return CONVKV_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return CONVKV_ERR_UNSUPPORTED;
@@ -131,10 +134,11 @@ int validate(const convkv_cfg* c) {
   const int64_t T = static_cast<int64_t>(c->grid_h) * c->grid_w;
   const int64_t R = c->window_frames + Bmax;
   // TMA coordinates and row counts are 32-bit
-  if (T * (R > c->mem_slots ? R : c->mem_slots) > (int64_t(1) << 30) || T * Bmax > (int64_t(1) << 30))
+  if (T * (R > c->mem_slots ? R : c->mem_slots) > (int64_t(1) << 30) || T * Bmax > (int64_t(1) << 30) ||
+      T * c->sink_frames > (int64_t(1) << 30))
     return CONVKV_ERR_UNSUPPORTED;
   const int pt = rope_pairs_t(D), ph = rope_pairs_h(D);
-  const int64_t tab_units = (int64_t(c->mem_slots) + c->window_frames + Bmax) * rope_units(0, pt) +
+  const int64_t tab_units = (int64_t(c->sink_frames) + c->mem_slots + c->window_frames + Bmax) * rope_units(0, pt) +
                             int64_t(c->grid_h) * rope_units(pt, ph) + int64_t(c->grid_w) * rope_units(pt + ph, ph);
   if (tab_units * 16 > 256 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables stay cache-resident
   if (c->kv_format == CONVKV_KV_FP8_E4M3 && c->compress_mode == CONVKV_COMPRESS_MEAN) return CONVKV_ERR_UNSUPPORTED;
@@ -210,7 +214,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->PH = cfg->head_dim / 6;
   h->PW = h->PH;
   h->PT = (cfg->head_dim - 4 * h->PH) / 2;
-  h->tab_t_rows = h->C + h->W + h->Bmax;
+  h->Rs = cfg->sink_frames;
+  h->tab_t_rows = h->Rs + h->C + h->W + h->Bmax;
   h->dry = (cfg->flags & CONVKV_FLAG_DRY_RUN) != 0;
   h->host_io = (cfg->flags & CONVKV_FLAG_HOST_IO) != 0;
   h->mean = cfg->compress_mode == CONVKV_COMPRESS_MEAN;
@@ -236,6 +241,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   build_tables(h, tab);
   const size_t tab_b = tab.size() * sizeof(float4);
   const size_t io_b = h->host_io ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
+  const size_t sink_b = static_cast<size_t>(h->S) * h->Rs * fe * 2;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -245,7 +251,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t o_rk = take(ring_b), o_rv = take(ring_b), o_mk = take(mem_b), o_mv = take(mem_b), o_w = take(w_b),
                o_tab = take(tab_b), o_st = take(sizeof(int)), o_q = take(io_b), o_k = take(io_b),
                o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
-               o_sv = take(stg_b), o_am = take(amax_b);
+               o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -268,6 +274,10 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->stageK = a + o_sk;
     h->stageV = a + o_sv;
     h->amax = reinterpret_cast<unsigned int*>(a + o_am);
+  }
+  if (h->Rs) {
+    h->sinkK = a + o_rfk;
+    h->sinkV = a + o_rfv;
   }
   if (h->host_io) {
     h->io_q = a + o_q;
@@ -297,6 +307,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
   }
+  if (!rc && h->Rs) rc = encode_4d(&h->mapSinkK, h->sinkK, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
+  if (!rc && h->Rs) rc = encode_4d(&h->mapSinkV, h->sinkV, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && w_b) rc = encode_weights(&h->mapW, h->weights, h->D, h->H, h->S);
   if (rc) {
     cudaFree(h->arena);
@@ -406,17 +418,30 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
   return CONVKV_OK;
 }
 
+int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
+  if (!h || (!h->dry && (!k || !v))) return CONVKV_ERR_INVALID_ARG;
+  if (h->Rs == 0) return CONVKV_ERR_BAD_ORDER;
+  if (!h->dry) {
+    const size_t bytes = static_cast<size_t>(h->S) * h->Rs * h->frame_elems() * 2;
+    cudaError_t e = cudaMemcpyAsync(h->sinkK, k, bytes, cudaMemcpyDeviceToDevice, h->stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(h->sinkV, v, bytes, cudaMemcpyDeviceToDevice, h->stream);
+    if (e != cudaSuccess) return h->cuda_fail(e);
+  }
+  h->sink_set = true;
+  return CONVKV_OK;
+}
+
 int convkv_attend(convkv_t* h, const void* q, void* out) {
   if (!h || (!h->dry && (!q || !out))) return CONVKV_ERR_INVALID_ARG;
-  if (h->blocks < 1) return CONVKV_ERR_BAD_ORDER;
+  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
   if (h->dry) return CONVKV_OK;
-  const int m = h->m(), w = h->w(), b = h->bcur, T = h->T;
+  const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur, T = h->T;
   AttnParams ap{};
   ap.H = h->H;
   ap.T = T;
   ap.grid_w = h->gw;
   ap.Nq = b * T;
-  ap.tq0 = m + w;
+  ap.tq0 = r + m + w;
   int tiles = 0;
   auto add = [&](int buf, int frame0, int nframes, int t0) {
     KeySeg& s = ap.seg[ap.nseg++];
@@ -425,15 +450,16 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
     s.nrows = nframes * T;
     s.t0 = t0;
     s.tile0 = tiles;
-    s.fp8 = (h->fp8 && buf != 2) ? 1 : 0;
+    s.fp8 = (h->fp8 && buf < 2) ? 1 : 0;
     s.slot0 = frame0;
     tiles += (s.nrows + 127) / 128;
   };
+  if (r > 0) add(3, 0, r, 0);
   if (m > 0) {
     const int pos0 = static_cast<int>((h->Sn - m) % h->C);
     const int n1 = m < h->C - pos0 ? m : h->C - pos0;
-    add(1, pos0, n1, 0);
-    if (m > n1) add(1, 0, m - n1, n1);
+    add(1, pos0, n1, r);
+    if (m > n1) add(1, 0, m - n1, r + n1);
   }
   {
     // bf16: window and current block are consecutive ring frames; fp8: the window
@@ -441,9 +467,9 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
     const int n = h->fp8 ? w : w + b;
     const int start = static_cast<int>(h->E % h->R);
     const int n1 = n < h->R - start ? n : h->R - start;
-    if (n1 > 0) add(0, start, n1, m);
-    if (n > n1) add(0, 0, n - n1, m + n1);
-    if (h->fp8) add(2, 0, b, m + w);
+    if (n1 > 0) add(0, start, n1, r + m);
+    if (n > n1) add(0, 0, n - n1, r + m + n1);
+    if (h->fp8) add(2, 0, b, r + m + w);
   }
   ap.ntiles = tiles;
   ap.tab_t_rows = h->tab_t_rows;
@@ -458,7 +484,7 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
   CUtensorMap mq;
   int rc = encode_4d(&mq, const_cast<void*>(q), h->D, h->H, ap.Nq, h->S);
   if (rc) return rc;
-  CUtensorMap km[3], vm[3];
+  CUtensorMap km[4], vm[4];
   if (h->fp8) {
     ap.ring_scale = h->ring_scale;
     ap.mem_scale = h->mem_scale;
@@ -466,12 +492,14 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
     ap.ring8[1] = static_cast<const uint8_t*>(h->ringV);
     ap.mem8[0] = static_cast<const uint8_t*>(h->memK);
     ap.mem8[1] = static_cast<const uint8_t*>(h->memV);
-    km[0] = km[1] = km[2] = h->mapStageK;  // only the staging map is used by TMA
+    km[0] = km[1] = km[2] = h->mapStageK;  // only staging and reference maps are used by TMA
     vm[0] = vm[1] = vm[2] = h->mapStageV;
   } else {
     km[0] = h->mapRingK; km[1] = h->mapMemK; km[2] = h->mapRingK;
     vm[0] = h->mapRingV; vm[1] = h->mapMemV; vm[2] = h->mapRingV;
   }
+  km[3] = r ? h->mapSinkK : km[2];
+  vm[3] = r ? h->mapSinkV : vm[2];
   int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp8, h->stream);
   h->launches++;
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
@@ -504,7 +532,7 @@ int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
 
 int convkv_layout(const convkv_t* h, int32_t* rec, int cap) {
   if (!h || (cap > 0 && !rec) || cap < 0) return CONVKV_ERR_INVALID_ARG;
-  const int m = h->m(), w = h->w(), b = h->bcur;
+  const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur;
   int n = 0;
   auto put = [&](int part, int64_t src, int64_t phys, int t) {
     if (n < cap) {
@@ -515,12 +543,13 @@ int convkv_layout(const convkv_t* h, int32_t* rec, int cap) {
     }
     ++n;
   };
+  for (int i = 0; i < r; ++i) put(3, i, i, i);
   for (int i = 0; i < m; ++i) {
     const int64_t k = h->Sn - m + i;
-    put(0, k, k % h->C, i);
+    put(0, k, k % h->C, r + i);
   }
-  for (int i = 0; i < w; ++i) put(1, h->E + i, (h->E + i) % h->R, m + i);
-  for (int f = 0; f < b; ++f) put(2, h->P + f, h->fp8 ? f : (h->P + f) % h->R, m + w + f);
+  for (int i = 0; i < w; ++i) put(1, h->E + i, (h->E + i) % h->R, r + m + i);
+  for (int f = 0; f < b; ++f) put(2, h->P + f, h->fp8 ? f : (h->P + f) % h->R, r + m + w + f);
   return n;
 }
 

@@ -9,7 +9,7 @@
 namespace ckv {
 
 constexpr int kEvict = 5;       // eviction group = conv kernel = conv stride (5:1)
-constexpr int kMaxSegs = 6;     // key segments of one attend (memory 2 + ring 2 + staging 1)
+constexpr int kMaxSegs = 6;     // key segments of one attend (reference 1 + memory 2 + ring 2 + staging 1)
 constexpr int kMaxGroups = 16;  // eviction groups one append may compress
 
 // RoPE channel pairs per axis for head_dim D: row and column floor(D/6), time the rest
@@ -24,7 +24,7 @@ constexpr int kStatusTimeout = 1;
 
 // One contiguous run of key rows in one buffer.
 struct KeySeg {
-  int buf;     // 0 ring, 1 memory, 2 current-block staging (fp8 format only)
+  int buf;     // 0 ring, 1 memory, 2 current-block staging (fp8 format only), 3 reference frames
   int row0;    // first row (token) in that buffer, a frame boundary
   int nrows;   // rows = frames * T
   int t0;      // RoPE time index of the segment's first frame
@@ -95,6 +95,7 @@ int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const
 int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s);
 int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s);
+// k, v: tensor maps of buffers 0..3 (ring, memory, staging, reference frames)
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k,
                   const CUtensorMap* v, int S, bool fp8, cudaStream_t s);
 size_t attend_smem_bytes(int D, const AttnParams& p);

@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                 const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
                 const __grid_constant__ CUtensorMap tmV1, const __grid_constant__ CUtensorMap tmK2,
-                const __grid_constant__ CUtensorMap tmV2, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV2, const __grid_constant__ CUtensorMap tmK3,
+                const __grid_constant__ CUtensorMap tmV3, const AttnParams p) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -261,8 +262,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      auto kmap = [&](int buf) { return buf == 0 ? &tmK0 : (buf == 1 ? &tmK1 : &tmK2); };
-      auto vmap = [&](int buf) { return buf == 0 ? &tmV0 : (buf == 1 ? &tmV1 : &tmV2); };
+      auto kmap = [&](int buf) { return buf == 0 ? &tmK0 : (buf == 1 ? &tmK1 : (buf == 2 ? &tmK2 : &tmK3)); };
+      auto vmap = [&](int buf) { return buf == 0 ? &tmV0 : (buf == 1 ? &tmV1 : (buf == 2 ? &tmV2 : &tmV3)); };
       tma_prefetch_desc(&tmQ);
       mbar_expect_tx(q_full, C::QT * C::TILE);
 #pragma unroll
@@ -591,7 +592,7 @@ int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, co
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid((p.Nq + 255) / 256, p.H, S);
-  kern<<<grid, AttnCfg<D>::THREADS, smem, s>>>(q, k[0], v[0], k[1], v[1], k[2], v[2], p);
+  kern<<<grid, AttnCfg<D>::THREADS, smem, s>>>(q, k[0], v[0], k[1], v[1], k[2], v[2], k[3], v[3], p);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -79,6 +79,8 @@ typedef struct convkv_cfg {
   const void* conv_weight; /* device bf16 [num_states][2 (K,V)][H][D_out][D_in][5]; read once at create,
                               not retained; may be NULL for CONVKV_COMPRESS_MEAN or dry-run */
   void* stream;            /* cudaStream_t for all device work of this handle (NULL = legacy default) */
+  int sink_frames;         /* reference-image frames attended first and never evicted (0 = none);
+                              their K/V are given once with convkv_set_sink */
 } convkv_cfg;
 
 typedef struct convkv convkv_t;
@@ -102,9 +104,11 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out);
 int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames);
 
 /* Attention of the current block's queries over [memory | window | current]
- * with RoPE time indices reset to start at 0 (memory slot i -> i, window frame
- * j -> m + j, current frame f -> m + w + f), spatial indices unchanged,
- * softmax scale 1/sqrt(D), no mask inside the attended set.
+ * (preceded by the reference frames when cfg.sink_frames > 0) with RoPE time
+ * indices reset to start at 0 (memory slot i -> r + i, window frame j -> r + m +
+ * j, current frame f -> r + m + w + f, r = sink_frames), spatial indices
+ * unchanged, softmax scale 1/sqrt(D), no mask inside the attended set.
+ * BAD_ORDER also when sink_frames > 0 and convkv_set_sink was not called.
  * q, out: DEVICE pointers, [num_states][frames*T][H][D] bf16 with `frames` of
  * the last append.  Does not change the state (may be repeated).
  * Errors: INVALID_ARG, BAD_ORDER, CUDA. */
@@ -123,12 +127,23 @@ size_t convkv_state_bytes(const convkv_t* h);
 /* Release everything the handle owns (waits for its stream).  NULL is a no-op. */
 void convkv_destroy(convkv_t* h);
 
+/* Reference-image partition (SoulX-LiveAct blog, "ConvKV Memory": the KV context
+ * is reference-image state + long-term memory + short-term memory + current
+ * block).  Stores the K/V of the cfg.sink_frames reference frames: DEVICE
+ * pointers, [num_states][sink_frames*T][H][D] bf16, copied asynchronously on
+ * the handle's stream (kept in bf16 in both formats).  They are never evicted
+ * or compressed and every attend takes them first, so the RoPE time indices run
+ * 0.. over [reference | memory | window | current].  May be called again to
+ * replace them.  Errors: INVALID_ARG, BAD_ORDER (sink_frames == 0), CUDA. */
+int convkv_set_sink(convkv_t* h, const void* k, const void* v);
+
 /* Key-frame layout of the next attend, in attended order, 4 int32 per frame:
- * {partition (0 memory, 1 window, 2 current), source index (slot index for
- * memory -- slot k covers stream frames [5k, 5k+5) -- else stream frame index),
- * physical slot (memory position, ring slot, or staging slot for the fp8
- * current block), RoPE time index}.  Returns the number of key frames, or a
- * negative error; writes at most `cap` records. */
+ * {partition (0 memory, 1 window, 2 current, 3 reference image), source index
+ * (slot index for memory -- slot k covers stream frames [5k, 5k+5) -- frame
+ * index within the reference for the reference image, else stream frame
+ * index), physical slot (memory position, ring slot, staging slot for the fp8
+ * current block, or reference frame), RoPE time index}.  Returns the number of
+ * key frames, or a negative error; writes at most `cap` records. */
 int convkv_layout(const convkv_t* h, int32_t* rec, int cap);
 
 /* Counters {P promoted frames, E evicted frames, S slots produced, m stored

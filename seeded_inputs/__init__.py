@@ -11,6 +11,7 @@ Tensor ids and element order:
              for token s of the frame, head h, channel d  ([T][H][D] per frame)
   WK, WV   : frame = 0, element = ((h*D + o)*D + i)*5 + j
              ([H][D_out][D_in][5] conv weights, scaled by 1/sqrt(5*D))
+  RK, RV   : frame = reference-image frame index, element as for K and V
 """
 from __future__ import annotations
 
@@ -21,7 +22,7 @@ import subprocess
 
 import numpy as np
 
-Q, K, V, WK, WV = 0, 1, 2, 3, 4
+Q, K, V, WK, WV, RK, RV = 0, 1, 2, 3, 4, 5, 6
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _HOST_SO = os.path.join(_HERE, "libseeded_inputs_host.so")

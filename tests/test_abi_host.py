@@ -52,6 +52,8 @@ def test_invalid_configs_rejected():
         (base.with_(num_states=0), ckv.ERR_INVALID_ARG),
         (base.with_(rope_theta=0.0), ckv.ERR_INVALID_ARG),
         (base.with_(grid_h=4096, grid_w=4096), ckv.ERR_UNSUPPORTED),
+        (base.with_(sink_frames=-1), ckv.ERR_INVALID_ARG),
+        (base.with_(sink_frames=100000), ckv.ERR_UNSUPPORTED),   # RoPE time table too large
     ]
     for cfg, code in bad:
         with pytest.raises(ckv.ConvKVError) as e:
@@ -107,6 +109,36 @@ def test_bookkeeping_matches_oracle_every_block(name):
                 assert phys == src - st.P
             else:
                 assert phys == (src % w.mem_slots if part == 0 else src % R)
+
+
+@pytest.mark.parametrize("name,sink", [("tiny", 2), ("512x512", 1), ("fp8_480x832", 1)])
+def test_reference_frames_lead_the_layout(name, sink):
+    """Reference-image frames come first at time 0..r-1, never move, and shift every other
+    time index by r; the rest of the layout is the sink-free one."""
+    w = PRESETS[name]
+    h = _dry(w, sink_frames=sink)
+    lib = ckv.library()
+    cfg = O.OracleConfig(H=1, D=6, grid_h=1, grid_w=1, window=w.window_frames, mem_slots=w.mem_slots)
+    st = O.OracleStream(cfg, np.zeros((2, 1, 6, 6, 5)))
+    st.set_sink(np.zeros((sink, 1, 1, 6)), np.zeros((sink, 1, 1, 6)))
+    h.dry_append(w.block_sizes()[0])
+    assert lib.convkv_attend(h._h, None, None) == ckv.ERR_BAD_ORDER      # reference not given yet
+    h.set_sink(None, None)
+    assert lib.convkv_attend(h._h, None, None) == ckv.OK
+    st.append(np.zeros((w.block_sizes()[0], 1, 1, 6)), np.zeros((w.block_sizes()[0], 1, 1, 6)))
+    for b in w.block_sizes()[1:]:
+        h.dry_append(b)
+        st.append(np.zeros((b, 1, 1, 6)), np.zeros((b, 1, 1, 6)))
+        lay = h.layout()
+        assert [tuple(r) for r in lay[:, [0, 1, 3]]] == _oracle_layout(st)
+        assert [tuple(r) for r in lay[:sink]] == [(3, i, i, i) for i in range(sink)]
+        assert list(lay[:, 3]) == list(range(len(lay)))
+
+
+def test_set_sink_needs_reference_frames():
+    h = _dry(PRESETS["tiny"])
+    assert ckv.library().convkv_set_sink(h._h, None, None) == ckv.ERR_BAD_ORDER
+    assert ckv.library().convkv_set_sink(None, None, None) == ckv.ERR_INVALID_ARG
 
 
 def test_soak_bookkeeping_closed_form_and_constant_footprint():

@@ -58,13 +58,16 @@ def test_bounded_wait_reports_timeout_and_context_survives(torch):
 
 
 def _run(torch, w: Workload, attend_blocks=None, rows=None, compress=0, t_offset=0, override=None,
-         check_slots=True, ring_frames=None, max_blocks=None, collect=None, sharp=False):
-    """Stream w through both sides; returns per-block error records."""
+         check_slots=True, ring_frames=None, max_blocks=None, collect=None, sharp=False, sink=0):
+    """Stream w through both sides; returns per-block error records.  sink > 0 gives both
+    sides that many reference-image frames (attended first, never evicted)."""
     ckv = _ckv()
     weights = device_weights(w, torch)
-    cfg = w.config(compress_mode=compress, t_offset=t_offset)
+    cfg = w.config(compress_mode=compress, t_offset=t_offset, sink_frames=sink)
     h = ckv.ConvKV(cfg, None if compress == ckv.COMPRESS_MEAN else weights)
     st = oracle_for(w, mean=(compress == ckv.COMPRESS_MEAN))
+    if sink:
+        _set_sink(torch, w, h, {0: st}, sink)
     rng = np.random.default_rng(w.seed)
     R = cfg.ring_frames
     F = 0
@@ -114,6 +117,13 @@ def _run(torch, w: Workload, attend_blocks=None, rows=None, compress=0, t_offset
     assert h.status() == 0
     h.close()
     return recs
+
+
+def _set_sink(torch, w, h, oracles, sink):
+    h.set_sink(device_frames(w, si.RK, 0, sink, torch), device_frames(w, si.RV, 0, sink, torch))
+    for s, st in oracles.items():
+        st.set_sink(si.bf16_bits_to_f64(host_frames(w, si.RK, s, 0, sink)),
+                    si.bf16_bits_to_f64(host_frames(w, si.RV, s, 0, sink)))
 
 
 def test_tiny_stream_full_parity(torch):
@@ -182,13 +192,15 @@ def test_720_stream_ragged(torch):
     _run(torch, PRESETS["720x416"], attend_blocks={1, 3, 12, 13, 27, 38}, rows=64, ring_frames=[0, 5])
 
 
-def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, ring_frames=None):
+def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, ring_frames=None, sink=0):
     """fp8 format: window codes bit-exact, memory codes within one step, attention <= 5e-2."""
     ckv = _ckv()
     weights = device_weights(w, torch)
-    cfg = w.config()
+    cfg = w.config(sink_frames=sink)
     h = ckv.ConvKV(cfg, weights)
     oracles = {s: oracle_for(w, state=s) for s in states}
+    if sink:
+        _set_sink(torch, w, h, oracles, sink)
     rng = np.random.default_rng(w.seed)
     R = cfg.ring_frames
     F = 0
@@ -237,3 +249,35 @@ def test_tiny_fp8_two_states(torch):
 def test_fp8_480x832_40_states(torch):
     _run_fp8(torch, PRESETS["fp8_480x832"], states=(0, 39), attend_blocks={1, 2, 5, 9, 17, 25}, rows=32,
              ring_frames=[0, 7])
+
+
+# -- reference-image partition (attended first, exact, never evicted) ------------------
+
+def test_tiny_reference_frames(torch):
+    """Two reference frames (32 keys: one ragged tile) ahead of memory|window|current."""
+    recs = _run(torch, PRESETS["tiny"], sink=2)
+    assert sum(1 for r in recs if r[0] == "attend") == 15
+
+
+def test_tiny_reference_frames_time_shift_invariance(torch):
+    a, b = [], []
+    _run(torch, PRESETS["tiny"], sink=2, t_offset=0, collect=a, max_blocks=8)
+    _run(torch, PRESETS["tiny"], sink=2, t_offset=1000, collect=b, max_blocks=8)
+    for (n, r, g0, ref), (_, _, g1, _) in zip(a, b):
+        e = attention_errors(g1, g0)
+        assert e["max"] <= 1e-2 and e["rel_l2"] <= 1e-2, (n, e)
+
+
+def test_512_reference_frame(torch):
+    _run(torch, PRESETS["512x512"], attend_blocks={1, 4, 13, 26}, rows=64, ring_frames=[0], sink=1)
+
+
+def test_720_reference_frame_ragged(torch):
+    """1170-token frames: the reference segment ends in a ragged tile, as do the others."""
+    _run(torch, PRESETS["720x416"], attend_blocks={1, 13, 38}, rows=64, ring_frames=[0], sink=1)
+
+
+def test_tiny_fp8_reference_frames_two_states(torch):
+    """fp8 window/memory with bf16 reference frames, one per state."""
+    w = replace(PRESETS["tiny"], fp8=True, num_states=2, name="tiny_fp8")
+    _run_fp8(torch, w, states=(0, 1), sink=1)
