@@ -226,7 +226,8 @@ def run_ours(args, w):
 
     S, H, D, T = w.num_states, w.heads, w.head_dim, w.T
     r = args.sink_frames
-    cfg = w.config(host_io=True, sink_frames=r)
+    mean = args.compress == "mean"
+    cfg = w.config(host_io=True, sink_frames=r, compress_mode=ckv.COMPRESS_MEAN if mean else ckv.COMPRESS_CONV)
     stream = torch.cuda.current_stream()
     fe = T * H * D
     # conv weights and inputs: seeded, generated on the device (each rank its own layer state)
@@ -235,7 +236,7 @@ def run_ours(args, w):
         for kv, tid in ((0, si.WK), (1, si.WV)):
             si.frames_device(weights[s, kv].data_ptr(), w.seed + rank, tid, s, 0, 1, H * D * D * 5,
                              si.weight_scale(D), stream.cuda_stream)
-    h = ckv.ConvKV(cfg, weights, stream=stream)
+    h = ckv.ConvKV(cfg, None if mean else weights, stream=stream)
     if r:
         # reference-image frames, attended first by every block
         ref = []
@@ -345,9 +346,10 @@ def run_ours(args, w):
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
         "config": {"workload": f"{w.name} steady state (memory full), one layer state per GPU"
-                               + (f", {r} reference-image frame(s) attended first" if r else ""),
+                               + (f", {r} reference-image frame(s) attended first" if r else "")
+                               + (", mean memory (5-frame mean instead of the conv)" if mean else ""),
                    "heads": H, "head_dim": D, "tokens_per_frame": T, "block_frames": b,
-                   "window_frames": w.window_frames, "mem_slots": w.mem_slots, "reference_frames": r, "states": S,
+                   "window_frames": w.window_frames, "mem_slots": w.mem_slots, "reference_frames": r, "compress": args.compress, "states": S,
                    "keys_per_step_avg": statistics.mean(nk_list), "state_bytes": h.state_bytes(),
                    "l2": "inputs larger than L2 (q,k,v 252 MB/step + 671 MB K/V state vs 126 MB L2)",
                    "parallelism": f"replicas x{world} (independent layer states, no collective)"},
@@ -385,6 +387,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="512x512")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--compress", choices=["conv", "mean"], default="conv",
+                    help="memory compression: the learned 1D conv (default) or the 5-frame mean")
     ap.add_argument("--sink-frames", type=int, default=0,
                     help="reference-image frames attended first by every block (default none)")
     args = ap.parse_args()
