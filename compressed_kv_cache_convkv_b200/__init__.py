@@ -34,6 +34,11 @@ _SIGNATURES = {
     "convkv_append_block": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     "convkv_attend": (ctypes.c_int, [_P, _P, _P]),
     "convkv_set_sink": (ctypes.c_int, [_P, _P, _P]),
+    "convkv_append_block_sp": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
+    "convkv_attend_sp": (ctypes.c_int, [_P, _P, _P]),
+    "convkv_ipc_export": (ctypes.c_int, [_P, _P, _P]),
+    "convkv_ipc_open": (ctypes.c_int, [_P, _P]),
+    "convkv_ipc_close": (ctypes.c_int, [_P]),
     "convkv_append_block_host": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     "convkv_attend_host": (ctypes.c_int, [_P, _P, _P]),
     "convkv_state_bytes": (ctypes.c_size_t, [_P]),
@@ -69,7 +74,8 @@ class _CCfg(ctypes.Structure):
         ("rope_h", ctypes.c_int), ("rope_w", ctypes.c_int), ("rope_theta", ctypes.c_double),
         ("kv_format", ctypes.c_int), ("compress_mode", ctypes.c_int), ("num_states", ctypes.c_int),
         ("flags", ctypes.c_int), ("t_offset", ctypes.c_int), ("conv_weight", ctypes.c_void_p),
-        ("stream", ctypes.c_void_p), ("sink_frames", ctypes.c_int),
+        ("stream", ctypes.c_void_p), ("sink_frames", ctypes.c_int), ("sp_ranks", ctypes.c_int),
+        ("sp_rank", ctypes.c_int),
     ]
 
 
@@ -132,6 +138,8 @@ class Config:
     host_io: bool = False
     t_offset: int = 0
     sink_frames: int = 0
+    sp_ranks: int = 1       # sequence-parallel group size; `heads` is then this rank's share
+    sp_rank: int = 0
 
     @property
     def T(self) -> int:
@@ -152,7 +160,7 @@ class Config:
         c = _CCfg()
         for name in ("heads", "head_dim", "grid_h", "grid_w", "first_block_frames", "block_frames",
                      "window_frames", "evict_frames", "mem_slots", "rope_theta", "kv_format", "compress_mode",
-                     "num_states", "t_offset", "sink_frames"):
+                     "num_states", "t_offset", "sink_frames", "sp_ranks", "sp_rank"):
             setattr(c, name, getattr(self, name))
         c.rope_t, c.rope_h, c.rope_w = self.rope
         c.flags = (FLAG_DRY_RUN if self.dry_run else 0) | (FLAG_HOST_IO if self.host_io else 0)
@@ -250,6 +258,23 @@ class ConvKV:
         if fk != self.cfg.sink_frames or fv != fk or not (k.is_cuda and v.is_cuda):
             raise ValueError(f"k, v must be CUDA tensors of {self.cfg.sink_frames} reference frames")
         self._check(_lib().convkv_set_sink(self._h, k.data_ptr(), v.data_ptr()), "convkv_set_sink")
+
+    # -- sequence-parallel forms: the all-to-all is fused into the kernels ----
+    def _ptrs(self, shards, name):
+        if len(shards) != self.cfg.sp_ranks:
+            raise ValueError(f"{name}: want {self.cfg.sp_ranks} shards, got {len(shards)}")
+        return (ctypes.c_void_p * len(shards))(*[t.data_ptr() for t in shards])
+
+    def append_sp(self, k_shards, v_shards, frames: int) -> None:
+        """k_shards[r], v_shards[r]: rank r's rows of the block (every head), bf16 CUDA
+        tensors [num_states, rows_r, sp_ranks*heads, D] with rows_r from shard_rows()."""
+        self._check(_lib().convkv_append_block_sp(self._h, self._ptrs(k_shards, "k"), self._ptrs(v_shards, "v"),
+                                                  frames), "convkv_append_block_sp")
+
+    def attend_sp(self, q_shards, out_shards) -> None:
+        """Queries from, and outputs into, the ranks' sequence shards (same layout as append_sp)."""
+        self._check(_lib().convkv_attend_sp(self._h, self._ptrs(q_shards, "q"), self._ptrs(out_shards, "out")),
+                    "convkv_attend_sp")
 
     def append_host(self, k, v) -> None:
         fk = self._frames_of(k, "k")

@@ -50,6 +50,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct convkv {
   convkv_cfg cfg{};
   int H = 0, D = 0, T = 0, gh = 0, gw = 0, b1 = 0, bn = 0, Bmax = 0, W = 0, C = 0, R = 0, S = 0, Rs = 0;
+  int G = 1, g = 0;  // sequence-parallel group size and this handle's rank
   int PT = 0, PH = 0, PW = 0, tab_t_rows = 0;
   bool dry = false, mean = false, fp8 = false, host_io = false, sink_set = false;
   // bookkeeping
@@ -117,7 +118,8 @@ int validate(const convkv_cfg* c) {
   if (!c) return CONVKV_ERR_INVALID_ARG;
   if (c->heads < 1 || c->head_dim < 1 || c->grid_h < 1 || c->grid_w < 1 || c->first_block_frames < 1 ||
       c->block_frames < 1 || c->window_frames < 4 || c->mem_slots < 1 || c->num_states < 1 ||
-      !(c->rope_theta > 0.0) || c->t_offset < 0 || c->sink_frames < 0)
+      !(c->rope_theta > 0.0) || c->t_offset < 0 || c->sink_frames < 0 || c->sp_ranks < 0 ||
+      c->sp_ranks > kMaxRanks || c->sp_rank < 0 || c->sp_rank >= (c->sp_ranks > 1 ? c->sp_ranks : 1))
     return CONVKV_ERR_INVALID_ARG;
   if (c->evict_frames != kEvict) return CONVKV_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return CONVKV_ERR_UNSUPPORTED;
@@ -145,6 +147,17 @@ int validate(const convkv_cfg* c) {
   if (c->compress_mode == CONVKV_COMPRESS_CONV && !(c->flags & CONVKV_FLAG_DRY_RUN) && !c->conv_weight)
     return CONVKV_ERR_INVALID_ARG;
   return CONVKV_OK;
+}
+
+// Sequence shards of a block of `frames` frames: rank r holds rows [r*N/G, (r+1)*N/G).
+ShardView make_view(const convkv* h, int frames) {
+  ShardView v{};
+  v.G = h->G;
+  v.Ht = h->G * h->H;
+  v.h0 = h->g * h->H;
+  const int64_t N = static_cast<int64_t>(frames) * h->T;
+  for (int r = 0; r <= h->G; ++r) v.off[r] = r * N / h->G;
+  return v;
 }
 
 void build_tables(const convkv* h, std::vector<float4>& out) {
@@ -215,6 +228,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->PW = h->PH;
   h->PT = (cfg->head_dim - 4 * h->PH) / 2;
   h->Rs = cfg->sink_frames;
+  h->G = cfg->sp_ranks > 1 ? cfg->sp_ranks : 1;
+  h->g = cfg->sp_rank;
   h->tab_t_rows = h->Rs + h->C + h->W + h->Bmax;
   h->dry = (cfg->flags & CONVKV_FLAG_DRY_RUN) != 0;
   h->host_io = (cfg->flags & CONVKV_FLAG_HOST_IO) != 0;
@@ -339,9 +354,8 @@ int64_t convkv_launch_count(const convkv_t* h) { return h ? h->launches : 0; }
 
 int convkv_last_cuda_error(const convkv_t* h) { return h ? h->last_cuda : 0; }
 
-int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
-  if (!h || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
-  if (!h->dry && (!k || !v)) return CONVKV_ERR_INVALID_ARG;
+static int append_impl(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
+                       const void* const* v_sh, int frames) {
   // 1. the previous current block joins the window
   h->P += h->bcur;
   // 2. evict groups of 5 while the window holds more than W frames
@@ -397,10 +411,17 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
   ap.R = h->R;
   ap.slot0 = static_cast<int>(h->P % h->R);
   ap.frame_elems = h->frame_elems();
+  ap.H = h->H;
+  ap.D = h->D;
+  if (k_sh) {
+    ap.sv = make_view(h, frames);
+    for (int r = 0; r < h->G; ++r) {
+      ap.k_sh[r] = k_sh[r];
+      ap.v_sh[r] = v_sh[r];
+    }
+  }
   int e;
   if (h->fp8) {
-    ap.H = h->H;
-    ap.D = h->D;
     ap.amax = h->amax;
     ap.ring8[0] = static_cast<uint8_t*>(h->ringK);
     ap.ring8[1] = static_cast<uint8_t*>(h->ringV);
@@ -418,6 +439,25 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
   return CONVKV_OK;
 }
 
+int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames) {
+  if (!h || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
+  if (!h->dry && (!k || !v)) return CONVKV_ERR_INVALID_ARG;
+  return append_impl(h, k, v, nullptr, nullptr, frames);
+}
+
+static bool shards_ok(const convkv_t* h, const void* const* a, const void* const* b) {
+  if (!a || !b) return false;
+  for (int r = 0; r < h->G; ++r)
+    if (!a[r] || !b[r]) return false;
+  return true;
+}
+
+int convkv_append_block_sp(convkv_t* h, const void* const* k_shards, const void* const* v_shards, int frames) {
+  if (!h || h->G < 2 || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
+  if (!h->dry && !shards_ok(h, k_shards, v_shards)) return CONVKV_ERR_INVALID_ARG;
+  return append_impl(h, nullptr, nullptr, h->dry ? nullptr : k_shards, h->dry ? nullptr : v_shards, frames);
+}
+
 int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
   if (!h || (!h->dry && (!k || !v))) return CONVKV_ERR_INVALID_ARG;
   if (h->Rs == 0) return CONVKV_ERR_BAD_ORDER;
@@ -431,10 +471,7 @@ int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
   return CONVKV_OK;
 }
 
-int convkv_attend(convkv_t* h, const void* q, void* out) {
-  if (!h || (!h->dry && (!q || !out))) return CONVKV_ERR_INVALID_ARG;
-  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
-  if (h->dry) return CONVKV_OK;
+static int attend_impl(convkv_t* h, const void* q, void* out, const void* const* q_sh, void* const* o_sh) {
   const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur, T = h->T;
   AttnParams ap{};
   ap.H = h->H;
@@ -481,9 +518,18 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
   ap.R = h->R;
   ap.C = h->C;
   ap.status = h->status;
-  CUtensorMap mq;
-  int rc = encode_4d(&mq, const_cast<void*>(q), h->D, h->H, ap.Nq, h->S);
-  if (rc) return rc;
+  CUtensorMap mq{};
+  if (q_sh) {
+    // queries are gathered from the sequence shards by the kernel: no TMA map for them
+    ap.sv = make_view(h, b);
+    for (int r = 0; r < h->G; ++r) {
+      ap.q_sh[r] = static_cast<const __nv_bfloat16*>(q_sh[r]);
+      ap.o_sh[r] = static_cast<__nv_bfloat16*>(o_sh[r]);
+    }
+  } else {
+    int rc = encode_4d(&mq, const_cast<void*>(q), h->D, h->H, ap.Nq, h->S);
+    if (rc) return rc;
+  }
   CUtensorMap km[4], vm[4];
   if (h->fp8) {
     ap.ring_scale = h->ring_scale;
@@ -504,6 +550,22 @@ int convkv_attend(convkv_t* h, const void* q, void* out) {
   h->launches++;
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   return CONVKV_OK;
+}
+
+int convkv_attend(convkv_t* h, const void* q, void* out) {
+  if (!h || (!h->dry && (!q || !out))) return CONVKV_ERR_INVALID_ARG;
+  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
+  if (h->dry) return CONVKV_OK;
+  return attend_impl(h, q, out, nullptr, nullptr);
+}
+
+int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_shards) {
+  if (!h || h->G < 2) return CONVKV_ERR_INVALID_ARG;
+  if (!h->dry && !shards_ok(h, q_shards, reinterpret_cast<const void* const*>(out_shards)))
+    return CONVKV_ERR_INVALID_ARG;
+  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
+  if (h->dry) return CONVKV_OK;
+  return attend_impl(h, nullptr, nullptr, q_shards, out_shards);
 }
 
 int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames) {

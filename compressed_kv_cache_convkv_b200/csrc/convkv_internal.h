@@ -34,6 +34,28 @@ struct KeySeg {
   int pad;
 };
 
+// A block's rows (frames * T tokens) split into G contiguous sequence shards, one
+// per rank, each holding every head of its rows: shard r is [S][off[r+1]-off[r]][Ht][D]
+// bf16 and this handle owns heads [h0, h0 + H) of Ht.  G == 0: not sharded, the
+// block is one [S][rows][H][D] tensor.
+constexpr int kMaxRanks = 8;
+struct ShardView {
+  int G, Ht, h0;
+  int64_t off[kMaxRanks + 1];
+};
+
+// Element offset (in bf16 units) of (state s, block row `row`, local head h, channel 0)
+// inside shard `r`, the shard that holds the row.
+__host__ __device__ __forceinline__ int64_t shard_elem(const ShardView& v, int s, int64_t row, int h, int D,
+                                                       int& r) {
+  r = 0;
+#pragma unroll
+  for (int q = 1; q < kMaxRanks; ++q)
+    if (q < v.G && row >= v.off[q]) r = q;
+  const int64_t n = v.off[r + 1] - v.off[r];
+  return ((static_cast<int64_t>(s) * n + (row - v.off[r])) * v.Ht + v.h0 + h) * D;
+}
+
 struct AttnParams {
   int H, T, grid_w, Nq;   // Nq = query rows per state (frames * T)
   int tq0;                // RoPE time index of the current block's first frame (m + w)
@@ -53,6 +75,11 @@ struct AttnParams {
   const uint8_t* mem8[2];   // fp8: e4m3 K, V memory [S][C*T][H][D]
   int R, C;
   int* status;
+  // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
+  // and written to the G ranks' shards (peer memory on a multi-GPU node)
+  ShardView sv;
+  const __nv_bfloat16* q_sh[kMaxRanks];
+  __nv_bfloat16* o_sh[kMaxRanks];
 };
 
 struct ConvGroup {
@@ -84,6 +111,11 @@ struct AppendParams {
   float* ring_scale;          // [S][2][R][H]
   void* stage[2];             // bf16 K, V current-block staging [S][stage_frames*T][H][D]
   int stage_frames;           // frames per state in the staging buffers (max block)
+  // sequence-sharded K, V (sv.G > 0): the block's rows are gathered from the G ranks'
+  // shards (peer memory on a multi-GPU node) instead of the k, v tensors
+  ShardView sv;
+  const void* k_sh[kMaxRanks];
+  const void* v_sh[kMaxRanks];
 };
 
 // Kernel launchers (return cudaError_t of the launch).

@@ -147,6 +147,20 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int row, const RopeRow& 
   }
 }
 
+// Copy one bf16 row of D channels from global (or peer) memory into row `row` of a
+// 128-byte-swizzled tile, zeros when src is null (rows past the block).
+template <int D>
+__device__ __forceinline__ void load_row(uint8_t* tile, int row, const __nv_bfloat16* src) {
+  using C = AttnCfg<D>;
+  uint8_t* rowp = tile + row * 128;
+  const int sw = row & 7;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 v = src ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = v;
+  }
+}
+
 // Two e4m3 codes (low byte first) -> two fp32 values (exact).
 __device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi) {
   uint32_t h2;
@@ -264,13 +278,16 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     if (lane == 0) {
       auto kmap = [&](int buf) { return buf == 0 ? &tmK0 : (buf == 1 ? &tmK1 : (buf == 2 ? &tmK2 : &tmK3)); };
       auto vmap = [&](int buf) { return buf == 0 ? &tmV0 : (buf == 1 ? &tmV1 : (buf == 2 ? &tmV2 : &tmV3)); };
-      tma_prefetch_desc(&tmQ);
-      mbar_expect_tx(q_full, C::QT * C::TILE);
+      if (p.sv.G == 0) {
+        // sequence-sharded queries are gathered row by row by the softmax warps instead
+        tma_prefetch_desc(&tmQ);
+        mbar_expect_tx(q_full, C::QT * C::TILE);
 #pragma unroll
-      for (int i = 0; i < C::QT; ++i)
+        for (int i = 0; i < C::QT; ++i)
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(sQ + i * C::TILE + bx * C::BOX, &tmQ, q_full, bx * 64, head, q_row0 + i * C::BM, state);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_4d(sQ + i * C::TILE + bx * C::BOX, &tmQ, q_full, bx * 64, head, q_row0 + i * C::BM, state);
+      }
       int kiss[C::KST] = {}, viss[C::VST] = {};
       TileCursor cur;
       for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
@@ -301,7 +318,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       }
       // drain: every issued copy must land before the CTA exits
       volatile int no_abort = 0;
-      mbar_wait(q_full, 0, &no_abort);
+      if (p.sv.G == 0) mbar_wait(q_full, 0, &no_abort);
       for (int i = 0; i < C::KST; ++i)
         if (kiss[i] > 0) mbar_wait(&k_full[i], (kiss[i] - 1) & 1, &no_abort);
       for (int i = 0; i < C::VST; ++i)
@@ -418,7 +435,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const int lane_base = (warp & 3) * 32;
     const int r = lane_base + lane;
     const int qr = q_row0 + i * C::BM + r;
-    bool alive = mbar_wait(q_full, 0, abort_flag);
+    bool alive = true;
+    if (p.sv.G == 0) {
+      alive = mbar_wait(q_full, 0, abort_flag);
+    } else {
+      // the row from the rank whose sequence shard holds it (the all-to-all of q)
+      int rk = 0;
+      const int64_t off = qr < p.Nq ? shard_elem(p.sv, state, qr, head, D, rk) : 0;
+      load_row<D>(sQ + i * C::TILE, r, qr < p.Nq ? p.q_sh[rk] + off : nullptr);
+    }
     if (alive && qr < p.Nq) {
       const int f = qr / p.T;
       const int s = qr - f * p.T;
@@ -514,7 +539,16 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     if (alive && mbar_wait_warp(&o_full[i], 0, abort_flag)) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + ((static_cast<int64_t>(state) * p.Nq + qr) * p.H + head) * D);
+      __nv_bfloat16* orow = nullptr;
+      if (p.sv.G == 0) {
+        orow = p.out + ((static_cast<int64_t>(state) * p.Nq + qr) * p.H + head) * D;
+      } else if (qr < p.Nq) {
+        // back to the rank whose sequence shard holds the row (the inverse all-to-all)
+        int rk = 0;
+        const int64_t off = shard_elem(p.sv, state, qr, head, D, rk);
+        orow = p.o_sh[rk] + off;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];

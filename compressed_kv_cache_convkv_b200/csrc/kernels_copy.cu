@@ -17,6 +17,23 @@ int grid_for(int64_t work_items, int threads) {
   return static_cast<int>(want < cap ? want : cap);
 }
 
+// 16-byte vector e of frame f of state s in the block's [T][H][D] layout: in the plain
+// tensor, or gathered from the sequence shard of the rank that holds the row (the
+// all-to-all of k/v fused into the append; the shard may live in a peer's memory).
+__device__ __forceinline__ const uint4* block_vec(const void* plain, const void* const* sh, const AppendParams& p,
+                                                  int s, int f, int64_t e) {
+  const int64_t fv = p.frame_elems / 8;
+  if (p.sv.G == 0) return static_cast<const uint4*>(plain) + (static_cast<int64_t>(s) * p.b + f) * fv + e;
+  const int vpr = p.H * p.D / 8;  // vectors per token
+  const int64_t T = p.frame_elems / (static_cast<int64_t>(p.H) * p.D);
+  const int64_t t = e / vpr;
+  const int rem = static_cast<int>(e - t * vpr);
+  const int h = rem / (p.D / 8);
+  int r = 0;
+  const int64_t off = shard_elem(p.sv, s, static_cast<int64_t>(f) * T + t, h, p.D, r);
+  return static_cast<const uint4*>(sh[r]) + off / 8 + (rem - h * (p.D / 8));
+}
+
 // Append (SoulX-LiveAct blog, "ConvKV Memory": append-only KV -- only the new
 // tokens' K/V are written, cached entries are never recomputed).
 // k, v: [S][b*T][H][D] bf16 -> ring slot (slot0 + f) % R of each state.
@@ -33,8 +50,8 @@ __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __r
     int slot = p.slot0 + f;
     if (slot >= p.R) slot -= p.R;
     const int64_t dst = (static_cast<int64_t>(s) * p.R + slot) * fv + e;
-    const uint4 kv = __ldcs(k + i);
-    const uint4 vv = __ldcs(v + i);
+    const uint4 kv = __ldcs(block_vec(k, p.k_sh, p, s, f, e));
+    const uint4 vv = __ldcs(block_vec(v, p.v_sh, p, s, f, e));
     ringK[dst] = kv;
     ringV[dst] = vv;
   }
@@ -116,10 +133,9 @@ __global__ void append_amax_kernel(const uint4* __restrict__ k, const uint4* __r
   const int vec_per_row = p.H * p.D / 8;
   const int r0 = blockIdx.x * rows_per_block;
   const int r1 = min(T, r0 + rows_per_block);
-  const uint4* src = (kv ? v : k) + (static_cast<int64_t>(s) * p.b + f) * (p.frame_elems / 8);
   for (int64_t i = static_cast<int64_t>(r0) * vec_per_row + threadIdx.x; i < static_cast<int64_t>(r1) * vec_per_row;
        i += blockDim.x) {
-    const uint4 x = __ldg(src + i);
+    const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, i));
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
     uint32_t m = 0;
 #pragma unroll
@@ -150,7 +166,7 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
     const int s = static_cast<int>(sf / p.b);
     const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
     const int h = static_cast<int>((e % vec_per_row) * 8 / p.D);
-    const uint4 x = __ldg((kv ? v : k) + iv);
+    const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
     reinterpret_cast<uint4*>(p.stage[kv])[(static_cast<int64_t>(s) * p.stage_frames + f) * fv + e] = x;
     const float amax = __uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]);
     const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;

@@ -81,6 +81,9 @@ typedef struct convkv_cfg {
   void* stream;            /* cudaStream_t for all device work of this handle (NULL = legacy default) */
   int sink_frames;         /* reference-image frames attended first and never evicted (0 = none);
                               their K/V are given once with convkv_set_sink */
+  int sp_ranks;            /* sequence-parallel group size G, 1..8 (0 or 1: no sharding); with G > 1
+                              `heads` is this rank's share of the G*heads heads */
+  int sp_rank;             /* this handle's rank g in [0, G): it owns heads [g*heads, (g+1)*heads) */
 } convkv_cfg;
 
 typedef struct convkv convkv_t;
@@ -136,6 +139,37 @@ void convkv_destroy(convkv_t* h);
  * 0.. over [reference | memory | window | current].  May be called again to
  * replace them.  Errors: INVALID_ARG, BAD_ORDER (sink_frames == 0), CUDA. */
 int convkv_set_sink(convkv_t* h, const void* k, const void* v);
+
+/* Sequence-parallel forms of append and attend (SoulX-LiveAct blog walk-through,
+ * system-level optimisation section, item (2): the sequence dimension is split over
+ * two GPUs that synchronise by communication; read here as the all-to-all between
+ * sequence shards and head shards, heads being independent in this step).  The caller's activations
+ * are split by sequence: rank r holds rows [off_r, off_{r+1}) of the block's
+ * frames*T rows, off_r = floor(r * frames*T / G), with ALL G*heads heads, as
+ * [num_states][off_{r+1}-off_r][G*heads][D] bf16.  The exchange is fused into the
+ * kernels: append gathers this rank's heads of every row from the G shards, attend
+ * reads its heads' query rows from the G q shards and writes each output row back
+ * into the shard of the rank that holds it.  shards[r] are DEVICE pointers valid in
+ * this process (a peer GPU's buffer mapped here, or a local buffer); the arrays
+ * themselves are host arrays of cfg.sp_ranks pointers, read during the call.  The
+ * caller orders the ranks around each call: every shard is written before any
+ * rank's kernels read it, and outputs are read after every rank's attend ends.
+ * Errors: as the plain forms; INVALID_ARG when the handle has sp_ranks < 2 or a
+ * shard pointer is null. */
+int convkv_append_block_sp(convkv_t* h, const void* const* k_shards, const void* const* v_shards, int frames);
+int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_shards);
+
+/* CUDA IPC helpers for sequence-parallel shards on a multi-GPU node (no counterpart
+ * on the pages; plumbing for the fused exchange above).  export: the 64-byte IPC
+ * handle of the cudaMalloc allocation that holds dev_ptr, and dev_ptr's byte
+ * offset in it (the allocation must come from cudaMalloc, not a virtual-memory
+ * pool).  open: maps a handle exported by another process on this node, with peer
+ * access enabled on first use; the shard is at *dev_ptr + offset.  close: unmaps
+ * a pointer returned by open.  Errors: INVALID_ARG (null argument, pointer not in
+ * a device allocation), CUDA. */
+int convkv_ipc_export(const void* dev_ptr, void* handle64, size_t* offset);
+int convkv_ipc_open(const void* handle64, void** dev_ptr);
+int convkv_ipc_close(void* dev_ptr);
 
 /* Key-frame layout of the next attend, in attended order, 4 int32 per frame:
  * {partition (0 memory, 1 window, 2 current, 3 reference image), source index
