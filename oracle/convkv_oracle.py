@@ -26,6 +26,10 @@ What it computes, and where that is stated:
 * Model card (hf.xjtesla.cn/Soul-AILab/LiveAct), "Command Line Arguments"
   table, ``--fp8_kv_cache``: the KV cache is stored in FP8 and dequantised to
   BF16 on use.
+* Same model card, open-source plan: FP4 for B-series GPUs (planned, format not
+  given).  Read as NVFP4, the Blackwell 4-bit format: e2m1 values with one e4m3
+  scale per 16 consecutive channels and one fp32 scale per (frame, head), stored
+  and dequantised to BF16 on use like the FP8 cache.
 
 Readings taken where the pages are silent (each listed in the design notes):
 W counts past-block frames only and eviction happens at append time in
@@ -58,6 +62,8 @@ import numpy as np
 PART_MEMORY, PART_WINDOW, PART_CURRENT, PART_SINK = 0, 1, 2, 3
 EVICT = 5          # frames per eviction group = conv kernel = conv stride (5:1)
 E4M3_MAX = 448.0   # largest finite e4m3 value
+E2M1_MAX = 6.0     # largest finite e2m1 value
+FP4_BLOCK = 16     # channels per NVFP4 block scale
 
 
 # --------------------------------------------------------------------------
@@ -130,6 +136,62 @@ def fp8_quantize(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     consumer (conv input, attention K/V).  Returns (dequantised values, scales[H])."""
     code, scale = fp8_encode(x)
     return fp8_dequantize(code, scale), scale
+
+
+def e2m1_rne_satfinite(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest e2m1 value (ties to even), saturating to +-6.
+
+    e2m1 (OCP FP4): 1 sign, 2 exponent bits (bias 1), 1 mantissa bit; the
+    magnitudes are 0, 0.5 (subnormal), 1, 1.5, 2, 3, 4, 6.  A value with exponent
+    e >= 0 (|x| in [2^e, 2^(e+1))) has quantum 2^(e-1); below 1 the quantum is
+    1/2.  Ties go to the even multiple of the quantum (mantissa bit 0).
+    """
+    x = np.asarray(x32, dtype=np.float32).astype(np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))   # a = m * 2^ex, 0.5 <= m < 1
+    e = np.maximum(ex.astype(np.float64) - 1.0, 0.0)
+    quantum = np.exp2(e - 1.0)
+    q = np.round(a / quantum) * quantum          # exact: a and quantum are dyadic
+    q = np.minimum(q, E2M1_MAX)
+    return np.where(a > 0, np.copysign(q, x), 0.0 * x)
+
+
+def fp4_encode(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """NVFP4 codes of one frame or slot x[T, H, D], in fp32 steps:
+
+      g   = amax / (448 * 6) per head over the frame's [T, D] (1 if amax == 0)
+      s_b = e4m3(a_b / (g * 6)) per block b of 16 channels of a token, a_b = max|x| in b
+      e_b = s_b * g
+      code = e2m1(x / e_b)   (0 where e_b == 0)
+
+    every product and quotient rounded to nearest in fp32, e4m3 and e2m1 rounding
+    to nearest even with saturation.  Returns (code values [T, H, D], block scale
+    values [T, H, D/16] (e4m3, as float64), tensor scales [H] (float32)).
+    """
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    T, H, D = x32.shape
+    amax = np.abs(x32).max(axis=(0, 2))
+    g = np.where(amax == 0, np.float32(1.0),
+                 (amax / np.float32(E4M3_MAX * E2M1_MAX)).astype(np.float32)).astype(np.float32)
+    xb = x32.reshape(T, H, D // FP4_BLOCK, FP4_BLOCK)
+    ab = np.abs(xb).max(axis=3)                                          # [T, H, nb], fp32
+    denom = (g * np.float32(E2M1_MAX)).astype(np.float32)                # [H]
+    ratio = (ab / denom[None, :, None]).astype(np.float32)
+    sb = e4m3_rne_satfinite(ratio)                                       # e4m3 values
+    eb = (sb.astype(np.float32) * g[None, :, None]).astype(np.float32)   # effective scale
+    safe = np.where(eb > 0, eb, np.float32(1.0)).astype(np.float32)
+    y = (xb / safe[..., None]).astype(np.float32)
+    code = np.where(eb[..., None] > 0, e2m1_rne_satfinite(y), 0.0)
+    return code.reshape(T, H, D), sb, g
+
+
+def fp4_dequantize(code: np.ndarray, sb: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """Dequantise to BF16 on use: bf16(fp32(code * fp32(s_b * g)))."""
+    T, H, D = code.shape
+    eb = (np.asarray(sb, dtype=np.float32) * np.asarray(g, dtype=np.float32)[None, :, None]).astype(np.float32)
+    c = np.asarray(code, dtype=np.float32).reshape(T, H, D // FP4_BLOCK, FP4_BLOCK)
+    prod = (c * eb[..., None]).astype(np.float32)
+    return round_to_bf16(prod.astype(np.float64)).reshape(T, H, D)
 
 
 # --------------------------------------------------------------------------
@@ -242,6 +304,7 @@ class OracleConfig:
     mem_slots: int         # C, FIFO capacity of compressed slots
     theta: float = 1e4
     fp8: bool = False
+    fp4: bool = False      # NVFP4 storage (exclusive with fp8)
     split: Optional[Tuple[int, int, int]] = None
 
     @property
@@ -257,7 +320,8 @@ class _Frame:
     k: np.ndarray          # [T, H, D] float64 (stored values, as consumed)
     v: np.ndarray
     index: int             # stream frame index (window/current) or slot index (memory)
-    codes: Optional[tuple] = None   # fp8: (k codes, k scales, v codes, v scales)
+    codes: Optional[tuple] = None   # fp8: (k codes, k scales, v codes, v scales);
+                                    # fp4: scales are (block scales, tensor scales)
 
 
 @dataclass
@@ -283,8 +347,8 @@ class OracleStream:
         self.S = 0        # slots produced so far
         self.block = 0
         self.events: List[ConvEvent] = []
-        self.mem_scales: List[np.ndarray] = []  # fp8: per-slot [2, H] scales
-        self.frame_scales = {}                  # fp8: stream frame -> [2, H] scales
+        self.mem_scales: List[tuple] = []       # fp8/fp4: per-slot (K, V) scales
+        self.frame_scales = {}                  # fp8/fp4: stream frame -> (K, V) scales
         self.sink: List[_Frame] = []            # reference-image frames, never evicted
 
     # -- reference-image partition -------------------------------------------
@@ -301,7 +365,7 @@ class OracleStream:
         cfg = self.cfg
         self.block += 1
         # (i) the previous current block joins the window
-        promoted = self.current_q8 if cfg.fp8 else self.current
+        promoted = self.current_q8 if (cfg.fp8 or cfg.fp4) else self.current
         self.window.extend(promoted)
         self.P += len(promoted)
         self.current, self.current_q8 = [], []
@@ -312,11 +376,9 @@ class OracleStream:
             kc = conv_compress(np.stack([f.k for f in group]), self.w[0])
             vc = conv_compress(np.stack([f.v for f in group]), self.w[1])
             codes = None
-            if cfg.fp8:
-                ck, sk = fp8_encode(kc)
-                cv, sv = fp8_encode(vc)
-                kc, vc = fp8_dequantize(ck, sk), fp8_dequantize(cv, sv)
-                scales = np.stack([sk, sv])
+            if cfg.fp8 or cfg.fp4:
+                (kc, ck, sk), (vc, cv, sv) = self._quantize(kc), self._quantize(vc)
+                scales = (sk, sv)
                 codes = (ck, sk, cv, sv)
             else:
                 kc, vc = round_to_bf16(kc), round_to_bf16(vc)
@@ -338,12 +400,20 @@ class OracleStream:
             kf = np.asarray(k[f], dtype=np.float64)
             vf = np.asarray(v[f], dtype=np.float64)
             self.current.append(_Frame(kf, vf, idx))
-            if cfg.fp8:
-                ck, sk = fp8_encode(kf)
-                cv, sv = fp8_encode(vf)
-                self.current_q8.append(_Frame(fp8_dequantize(ck, sk), fp8_dequantize(cv, sv), idx, (ck, sk, cv, sv)))
-                self.frame_scales[idx] = np.stack([sk, sv])
+            if cfg.fp8 or cfg.fp4:
+                (kq, ck, sk), (vq, cv, sv) = self._quantize(kf), self._quantize(vf)
+                self.current_q8.append(_Frame(kq, vq, idx, (ck, sk, cv, sv)))
+                self.frame_scales[idx] = (sk, sv)
         return new_events
+
+    def _quantize(self, x: np.ndarray):
+        """(values as consumed, codes, scales) of one frame or slot in the cache's
+        low-precision format; fp4 scales are (block scales, tensor scales)."""
+        if self.cfg.fp4:
+            code, sb, g = fp4_encode(x)
+            return fp4_dequantize(code, sb, g), code, (sb, g)
+        code, scale = fp8_encode(x)
+        return fp8_dequantize(code, scale), code, scale
 
     # -- layout ------------------------------------------------------------
     def key_frames(self) -> List[Tuple[int, _Frame, int]]:

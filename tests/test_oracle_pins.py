@@ -235,8 +235,8 @@ def test_attention_key_permutation_invariance():
 
 # ---------------------------------------------------------------- stream bookkeeping
 
-def _tiny_stream(W, C, blocks, b=2, b1=None, fp8=False, H=2, D=64, gh=4, gw=4, seed=0):
-    cfg = O.OracleConfig(H=H, D=D, grid_h=gh, grid_w=gw, window=W, mem_slots=C, fp8=fp8)
+def _tiny_stream(W, C, blocks, b=2, b1=None, fp8=False, H=2, D=64, gh=4, gw=4, seed=0, fp4=False):
+    cfg = O.OracleConfig(H=H, D=D, grid_h=gh, grid_w=gw, window=W, mem_slots=C, fp8=fp8, fp4=fp4)
     rng = np.random.default_rng(seed)
     w = rng.standard_normal((2, H, D, D, 5)) / math.sqrt(5 * D)
     st = O.OracleStream(cfg, w)
@@ -444,3 +444,76 @@ def test_sink_partition_equals_full_attention_over_concatenated_keys():
         ref = torch.nn.functional.scaled_dot_product_attention(
             torch.from_numpy(qr)[None], torch.from_numpy(kr)[None], torch.from_numpy(vall)[None])[0].numpy()
         np.testing.assert_allclose(o[:, h], ref, atol=1e-12)
+
+
+# -- NVFP4 (e2m1 values, e4m3 block scales per 16 channels, fp32 scale per frame and head)
+
+def test_e2m1_hand_table():
+    """The e2m1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}: nearest value, ties to the even
+    mantissa, saturation at 6 (values written out by hand from the format)."""
+    x = [0.0, 0.1, 0.25, 0.2500001, 0.5, 0.74, 0.75, 0.76, 1.0, 1.24, 1.25, 1.26, 1.5, 1.75, 2.0,
+         2.49, 2.5, 2.51, 3.0, 3.5, 4.0, 4.99, 5.0, 5.01, 6.0, 7.0, 100.0, -0.75, -5.0, -7.0, -0.25]
+    want = [0.0, 0.0, 0.0, 0.5, 0.5, 0.5, 1.0, 1.0, 1.0, 1.0, 1.0, 1.5, 1.5, 2.0, 2.0,
+            2.0, 2.0, 3.0, 3.0, 4.0, 4.0, 4.0, 4.0, 6.0, 6.0, 6.0, 6.0, -1.0, -4.0, -6.0, -0.0]
+    got = O.e2m1_rne_satfinite(np.array(x, dtype=np.float32))
+    np.testing.assert_array_equal(got, np.array(want))
+
+
+def test_e2m1_matches_brute_force_nearest():
+    """Against a search over the 15 finite values: nearest, and on a tie the one whose
+    mantissa bit is 0 (code index even)."""
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.uniform(-8, 8, 20000), (np.arange(-16, 17) / 4.0)]).astype(np.float32)
+    ref = np.empty(len(x))
+    for i, v in enumerate(x.astype(np.float64)):
+        a = min(abs(v), 6.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        j = best[0] if len(best) == 1 else [c for c in best if c % 2 == 0][0]
+        ref[i] = math.copysign(mags[j], v) if mags[j] != 0 else 0.0
+    np.testing.assert_array_equal(np.abs(O.e2m1_rne_satfinite(x)), np.abs(ref))
+
+
+def test_fp4_encode_grid_values_round_trip():
+    """Hand example.  Block 0 holds e2m1 grid values with max 6 = the frame's amax:
+    g = fp32(6 / 2688), s_0 = e4m3(6 / fp32(6 g)) = 448, e_0 = fp32(448 g) = 1, so the
+    codes are the values themselves.  Block 1 holds half-grid values with max 3:
+    s_1 = e4m3(3 / fp32(6 g)) = 224, e_1 = 1/2, codes = 2x.  Both dequantise exactly."""
+    b0 = [6.0, -3.0, 1.5, 0.5, 0.0, 4.0, -6.0, 2.0, 1.0, -1.5, 3.0, -0.5, 0.0, -4.0, 2.0, 1.0]
+    b1 = [v / 2 for v in b0]
+    x = np.array(b0 + b1, dtype=np.float64).reshape(1, 1, 32)
+    code, sb, g = O.fp4_encode(x)
+    assert g.dtype == np.float32 and g[0] == np.float32(6.0) / np.float32(2688.0)
+    np.testing.assert_array_equal(sb[0, 0], [448.0, 224.0])
+    np.testing.assert_array_equal(code[0, 0, :16], b0)
+    np.testing.assert_array_equal(code[0, 0, 16:], [2 * v for v in b1])
+    np.testing.assert_array_equal(O.fp4_dequantize(code, sb, g), x)
+
+
+def test_fp4_zero_block_and_error_bound():
+    rng = np.random.default_rng(9)
+    x = O.round_to_bf16(rng.standard_normal((8, 3, 64)))
+    x[2, 1, 16:32] = 0.0                                   # an all-zero block
+    code, sb, g = O.fp4_encode(x)
+    assert sb[2, 1, 1] == 0 and np.all(code[2, 1, 16:32] == 0)
+    np.testing.assert_array_equal(O.e2m1_rne_satfinite(code.astype(np.float32)), code)   # codes on the grid
+    np.testing.assert_array_equal(O.e4m3_rne_satfinite(sb.astype(np.float32)), sb)      # scales on the grid
+    dq = O.fp4_dequantize(code, sb, g)
+    eb = (sb * g[None, :, None]).repeat(16, axis=2)
+    # |x/e - code| <= 1 (largest half-quantum, at |x/e| in [4, 6]) plus the bf16 rounding
+    assert np.all(np.abs(dq - x) <= eb * 1.0 + np.abs(x) * 2.0 ** -8 + 1e-30)
+
+
+def test_fp4_stream_window_is_quantised_current_is_exact():
+    for st, (q, k, v), _ in _tiny_stream(W=4, C=3, blocks=5, fp4=True, seed=17):
+        pass
+    np.testing.assert_array_equal(st.current[0].k, k[0])
+    assert len(st.memory) > 0 and len(st.window) > 0
+    for f in st.window + st.memory:
+        ck, (bk, gk), cv, (bv, gv) = f.codes
+        np.testing.assert_array_equal(O.e2m1_rne_satfinite(ck.astype(np.float32)), ck)
+        np.testing.assert_array_equal(f.k, O.fp4_dequantize(ck, bk, gk))
+        np.testing.assert_array_equal(f.v, O.fp4_dequantize(cv, bv, gv))
+    o, ps = st.attend(q)
+    np.testing.assert_allclose(ps, 1.0, atol=1e-12)
