@@ -39,9 +39,12 @@ def attention_flops(Nq, Nk, D, H, S=1):
     return 4.0 * Nq * Nk * D * H * S
 
 
-def attention_bytes(Nq, Nk, D, H, S=1, kv_bytes=2):
-    """Algorithmic HBM bytes of one attend: Q and O (bf16) plus every key's K and V."""
-    return (2.0 * Nq * H * D * 2 + 2.0 * Nk * H * D * kv_bytes) * S
+def attention_bytes(Nq, Nk, D, H, S=1, kv_bytes=2, Nk_bf16=None):
+    """Algorithmic HBM bytes of one attend: Q and O (bf16) plus every key's K and V, at
+    kv_bytes per element (e4m3 1, NVFP4 9/16 with its block scales) except the Nk_bf16
+    keys kept in bf16 (the current block and reference frames of the low-precision formats)."""
+    nb = Nk if Nk_bf16 is None else Nk_bf16
+    return (2.0 * Nq * H * D * 2 + 2.0 * nb * H * D * 2 + 2.0 * (Nk - nb) * H * D * kv_bytes) * S
 
 
 def measured_traffic(algorithmic_bytes):
@@ -338,13 +341,17 @@ def run_ours(args, w):
     att_avg_ms = statistics.mean(att_ms)
     att_achieved = statistics.mean(flops) / (att_avg_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
-    att_bytes = attention_bytes(b * T, statistics.mean(nk_list), D, H, S)
-    traffic = measured_traffic(att_bytes)
+    kvb = 9.0 / 16.0 if getattr(w, "fp4", False) else (1.0 if w.fp8 else 2.0)
+    att_bytes = attention_bytes(b * T, statistics.mean(nk_list), D, H, S, kv_bytes=kvb,
+                                Nk_bf16=(b + r) * T if kvb < 2 else None)
+    # the committed capture is of the bf16 instantiation; other formats run another kernel
+    traffic = measured_traffic(att_bytes) if kvb == 2.0 else None
     frames_per_s = K * b * S * world / (total_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
+        "dtype": "bf16" if not w.fp8 and not getattr(w, "fp4", False) else
+                 ("bf16 compute, e4m3 K/V cache" if w.fp8 else "bf16 compute, NVFP4 K/V cache"), "data": "synthetic (seeded Philox4x32-10, Irwin-Hall(12) unit-variance bf16 values)",
         "config": {"workload": f"{w.name} steady state (memory full), one layer state per GPU"
                                + (f", {r} reference-image frame(s) attended first" if r else "")
                                + (", mean memory (5-frame mean instead of the conv)" if mean else ""),

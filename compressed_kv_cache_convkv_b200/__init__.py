@@ -22,7 +22,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_BAD_ORDER, ERR_OOM, ERR_CUDA, ERR_DEVICE_TIMEOUT = -1, -2, -3, -4, -5, -6
 ERR_SCRATCH_LIMIT = -7
 NOALLOC_MAX_FRAME_HEADS = 4096
-KV_BF16, KV_FP8_E4M3 = 0, 1
+KV_BF16, KV_FP8_E4M3, KV_NVFP4 = 0, 1, 2
 COMPRESS_CONV, COMPRESS_MEAN = 0, 1
 FLAG_DRY_RUN, FLAG_HOST_IO = 1, 2
 PART_MEMORY, PART_WINDOW, PART_CURRENT = 0, 1, 2
@@ -311,28 +311,30 @@ class ConvKV:
         _lib().convkv_layout(self._h, rec.ctypes.data, n)
         return rec[:n]
 
-    def read_slot(self, state: int, kv: int, pos: int):
-        """(bf16 bits [T, H, D] as uint16 -- or e4m3 codes as uint8 in the fp8 format --,
-        scales[H] or None) of memory position `pos`."""
+    def _read(self, fn, name: str, state: int, kv: int, idx: int):
         import numpy as np
         cfg = self.cfg
+        T, H, D = cfg.T, cfg.heads, cfg.head_dim
+        sc = np.zeros(H, dtype=np.float32)
+        if cfg.kv_format == KV_NVFP4:
+            raw = np.zeros(T * H * D // 2 + T * H * D // 16, dtype=np.uint8)
+            self._check(fn(self._h, state, kv, idx, raw.ctypes.data, sc.ctypes.data), name)
+            n = T * H * D // 2
+            return raw[:n].reshape(T, H, D // 2), (raw[n:].reshape(T, H, D // 16), sc)
         dt = np.uint8 if cfg.kv_format == KV_FP8_E4M3 else np.uint16
-        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=dt)
-        sc = np.zeros(cfg.heads, dtype=np.float32)
-        self._check(_lib().convkv_read_slot(self._h, state, kv, pos, dst.ctypes.data, sc.ctypes.data),
-                    "convkv_read_slot")
+        dst = np.zeros((T, H, D), dtype=dt)
+        self._check(fn(self._h, state, kv, idx, dst.ctypes.data, sc.ctypes.data), name)
         return dst, (sc if cfg.kv_format == KV_FP8_E4M3 else None)
+
+    def read_slot(self, state: int, kv: int, pos: int):
+        """Memory position `pos`: (bf16 bits [T, H, D] as uint16, None); in the fp8 format
+        (e4m3 codes uint8 [T, H, D], scales[H]); in the NVFP4 format (e2m1 pairs uint8
+        [T, H, D/2], (e4m3 block scales uint8 [T, H, D/16], scales[H]))."""
+        return self._read(_lib().convkv_read_slot, "convkv_read_slot", state, kv, pos)
 
     def read_ring(self, state: int, kv: int, slot: int):
         """Same as read_slot for ring slot `slot`."""
-        import numpy as np
-        cfg = self.cfg
-        dt = np.uint8 if cfg.kv_format == KV_FP8_E4M3 else np.uint16
-        dst = np.zeros((cfg.T, cfg.heads, cfg.head_dim), dtype=dt)
-        sc = np.zeros(cfg.heads, dtype=np.float32)
-        self._check(_lib().convkv_read_ring(self._h, state, kv, slot, dst.ctypes.data, sc.ctypes.data),
-                    "convkv_read_ring")
-        return dst, (sc if cfg.kv_format == KV_FP8_E4M3 else None)
+        return self._read(_lib().convkv_read_ring, "convkv_read_ring", state, kv, slot)
 
     def status(self) -> int:
         return int(_lib().convkv_status(self._h))

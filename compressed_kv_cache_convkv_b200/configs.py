@@ -27,6 +27,7 @@ class Workload:
     seed: int
     fp8: bool = False
     num_states: int = 1
+    fp4: bool = False        # NVFP4 ring and memory
 
     @property
     def T(self) -> int:
@@ -43,11 +44,12 @@ class Workload:
         return sizes
 
     def config(self, **kw):
-        from . import Config, KV_BF16, KV_FP8_E4M3
+        from . import Config, KV_BF16, KV_FP8_E4M3, KV_NVFP4
+        fmt = KV_NVFP4 if self.fp4 else (KV_FP8_E4M3 if self.fp8 else KV_BF16)
         c = Config(heads=self.heads, head_dim=self.head_dim, grid_h=self.grid_h, grid_w=self.grid_w,
                    first_block_frames=self.first_block_frames, block_frames=self.block_frames,
                    window_frames=self.window_frames, mem_slots=self.mem_slots,
-                   kv_format=KV_FP8_E4M3 if self.fp8 else KV_BF16, num_states=self.num_states)
+                   kv_format=fmt, num_states=self.num_states)
         return c.with_(**kw) if kw else c
 
 
@@ -62,4 +64,6 @@ PRESETS = {
     "soak": Workload("soak", 40, 128, 32, 32, 6, 8, 10, 8, 18000, seed=3),
     # fp8 e4m3 window/memory at 480x832: 30x52 = 1560 tokens, blocks of 8, 40 states per call
     "fp8_480x832": Workload("fp8_480x832", 40, 128, 30, 52, 8, 8, 10, 8, 200, seed=4, fp8=True, num_states=40),
+    # the same shape with the NVFP4 window and memory (FP4 for B-series GPUs)
+    "nvfp4_480x832": Workload("nvfp4_480x832", 40, 128, 30, 52, 8, 8, 10, 8, 200, seed=5, num_states=40, fp4=True),
 }

@@ -52,7 +52,8 @@ struct convkv {
   int H = 0, D = 0, T = 0, gh = 0, gw = 0, b1 = 0, bn = 0, Bmax = 0, W = 0, C = 0, R = 0, S = 0, Rs = 0;
   int G = 1, g = 0;  // sequence-parallel group size and this handle's rank
   int PT = 0, PH = 0, PW = 0, tab_t_rows = 0;
-  bool dry = false, mean = false, fp8 = false, host_io = false, sink_set = false;
+  // fp8: the ring and memory are stored in a low-precision format (e4m3, or NVFP4 when fp4)
+  bool dry = false, mean = false, fp8 = false, fp4 = false, host_io = false, sink_set = false;
   // bookkeeping
   int64_t P = 0, E = 0, Sn = 0, blocks = 0;
   int bcur = 0, last_groups = 0;
@@ -63,6 +64,8 @@ struct convkv {
   // fp8 format: ringK/ringV/memK/memV hold e4m3 codes; scales per (state, K|V, slot, head)
   float *ring_scale = nullptr, *mem_scale = nullptr;
   void *stageK = nullptr, *stageV = nullptr;  // bf16 copy of the current block
+  // NVFP4: ringK/ringV/memK/memV hold e2m1 pairs; e4m3 block scales per 16 channels
+  uint8_t *ringBK = nullptr, *ringBV = nullptr, *memBK = nullptr, *memBV = nullptr;
   void *sinkK = nullptr, *sinkV = nullptr;    // bf16 reference frames, both formats
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
   float4* tables = nullptr;
@@ -123,7 +126,8 @@ int validate(const convkv_cfg* c) {
     return CONVKV_ERR_INVALID_ARG;
   if (c->evict_frames != kEvict) return CONVKV_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return CONVKV_ERR_UNSUPPORTED;
-  if (c->kv_format != CONVKV_KV_BF16 && c->kv_format != CONVKV_KV_FP8_E4M3) return CONVKV_ERR_INVALID_ARG;
+  if (c->kv_format != CONVKV_KV_BF16 && c->kv_format != CONVKV_KV_FP8_E4M3 && c->kv_format != CONVKV_KV_NVFP4)
+    return CONVKV_ERR_INVALID_ARG;
   if (c->compress_mode != CONVKV_COMPRESS_CONV && c->compress_mode != CONVKV_COMPRESS_MEAN)
     return CONVKV_ERR_INVALID_ARG;
   if (c->flags & ~(CONVKV_FLAG_DRY_RUN | CONVKV_FLAG_HOST_IO)) return CONVKV_ERR_INVALID_ARG;
@@ -143,7 +147,7 @@ int validate(const convkv_cfg* c) {
   const int64_t tab_units = (int64_t(c->sink_frames) + c->mem_slots + c->window_frames + Bmax) * rope_units(0, pt) +
                             int64_t(c->grid_h) * rope_units(pt, ph) + int64_t(c->grid_w) * rope_units(pt + ph, ph);
   if (tab_units * 16 > 256 * 1024) return CONVKV_ERR_UNSUPPORTED;  // RoPE tables stay cache-resident
-  if (c->kv_format == CONVKV_KV_FP8_E4M3 && c->compress_mode == CONVKV_COMPRESS_MEAN) return CONVKV_ERR_UNSUPPORTED;
+  if (c->kv_format != CONVKV_KV_BF16 && c->compress_mode == CONVKV_COMPRESS_MEAN) return CONVKV_ERR_UNSUPPORTED;
   if (c->compress_mode == CONVKV_COMPRESS_CONV && !(c->flags & CONVKV_FLAG_DRY_RUN) && !c->conv_weight)
     return CONVKV_ERR_INVALID_ARG;
   return CONVKV_OK;
@@ -234,7 +238,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->dry = (cfg->flags & CONVKV_FLAG_DRY_RUN) != 0;
   h->host_io = (cfg->flags & CONVKV_FLAG_HOST_IO) != 0;
   h->mean = cfg->compress_mode == CONVKV_COMPRESS_MEAN;
-  h->fp8 = cfg->kv_format == CONVKV_KV_FP8_E4M3;
+  h->fp8 = cfg->kv_format != CONVKV_KV_BF16;
+  h->fp4 = cfg->kv_format == CONVKV_KV_NVFP4;
   h->stream = static_cast<cudaStream_t>(cfg->stream);
   h->cfg.conv_weight = nullptr;
   if (h->dry) {
@@ -243,9 +248,12 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   }
 
   const size_t fe = static_cast<size_t>(h->frame_elems());
-  const size_t esz = h->fp8 ? 1 : 2;  // bytes per cached element
-  const size_t ring_b = static_cast<size_t>(h->S) * h->R * fe * esz;
-  const size_t mem_b = static_cast<size_t>(h->S) * h->C * fe * esz;
+  // bytes of one cached frame: bf16 2 per element, e4m3 1, NVFP4 1/2 (+ 1/16 of block scales)
+  const size_t fbytes = h->fp4 ? fe / 2 : (h->fp8 ? fe : 2 * fe);
+  const size_t ring_b = static_cast<size_t>(h->S) * h->R * fbytes;
+  const size_t mem_b = static_cast<size_t>(h->S) * h->C * fbytes;
+  const size_t rbs_b = h->fp4 ? static_cast<size_t>(h->S) * h->R * fe / 16 : 0;
+  const size_t mbs_b = h->fp4 ? static_cast<size_t>(h->S) * h->C * fe / 16 : 0;
   const size_t rsc_b = h->fp8 ? static_cast<size_t>(h->S) * 2 * h->R * h->H * sizeof(float) : 0;
   const size_t msc_b = h->fp8 ? static_cast<size_t>(h->S) * 2 * h->C * h->H * sizeof(float) : 0;
   const size_t stg_b = h->fp8 ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
@@ -266,7 +274,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t o_rk = take(ring_b), o_rv = take(ring_b), o_mk = take(mem_b), o_mv = take(mem_b), o_w = take(w_b),
                o_tab = take(tab_b), o_st = take(sizeof(int)), o_q = take(io_b), o_k = take(io_b),
                o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
-               o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b);
+               o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b),
+               o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -289,6 +298,12 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->stageK = a + o_sk;
     h->stageV = a + o_sv;
     h->amax = reinterpret_cast<unsigned int*>(a + o_am);
+  }
+  if (h->fp4) {
+    h->ringBK = reinterpret_cast<uint8_t*>(a + o_rbk);
+    h->ringBV = reinterpret_cast<uint8_t*>(a + o_rbv);
+    h->memBK = reinterpret_cast<uint8_t*>(a + o_mbk);
+    h->memBV = reinterpret_cast<uint8_t*>(a + o_mbv);
   }
   if (h->Rs) {
     h->sinkK = a + o_rfk;
@@ -395,7 +410,11 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
       cp.ring_scale = h->ring_scale;
       cp.amax = h->amax;
       cp.mem_scale = h->mem_scale;
-      e = launch_conv_fp8(h->D, cp, h->mapW, h->stream);
+      cp.ring_bs[0] = h->ringBK;
+      cp.ring_bs[1] = h->ringBV;
+      cp.mem_bs[0] = h->memBK;
+      cp.mem_bs[1] = h->memBV;
+      e = h->fp4 ? launch_conv_fp4(h->D, cp, h->mapW, h->stream) : launch_conv_fp8(h->D, cp, h->mapW, h->stream);
       h->launches += 2;
     } else {
       e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
@@ -426,6 +445,9 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
     ap.ring8[0] = static_cast<uint8_t*>(h->ringK);
     ap.ring8[1] = static_cast<uint8_t*>(h->ringV);
     ap.ring_scale = h->ring_scale;
+    ap.ring_bs[0] = h->ringBK;
+    ap.ring_bs[1] = h->ringBV;
+    ap.fp4 = h->fp4 ? 1 : 0;
     ap.stage[0] = h->stageK;
     ap.stage[1] = h->stageV;
     ap.stage_frames = h->Bmax;
@@ -538,6 +560,10 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     ap.ring8[1] = static_cast<const uint8_t*>(h->ringV);
     ap.mem8[0] = static_cast<const uint8_t*>(h->memK);
     ap.mem8[1] = static_cast<const uint8_t*>(h->memV);
+    ap.ring_bs[0] = h->ringBK;
+    ap.ring_bs[1] = h->ringBV;
+    ap.mem_bs[0] = h->memBK;
+    ap.mem_bs[1] = h->memBV;
     km[0] = km[1] = km[2] = h->mapStageK;  // only staging and reference maps are used by TMA
     vm[0] = vm[1] = vm[2] = h->mapStageV;
   } else {
@@ -546,7 +572,7 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   }
   km[3] = r ? h->mapSinkK : km[2];
   vm[3] = r ? h->mapSinkV : vm[2];
-  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp8, h->stream);
+  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp4 ? 2 : (h->fp8 ? 1 : 0), h->stream);
   h->launches++;
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   return CONVKV_OK;
@@ -628,13 +654,17 @@ int convkv_counters(const convkv_t* h, int64_t out[8]) {
   return CONVKV_OK;
 }
 
-static int read_frame(const convkv_t* hc, const void* dev_base, int nslots, int state, int slot, void* host_dst,
-                      const float* scales, int kv, float* host_scales) {
+static int read_frame(const convkv_t* hc, const void* dev_base, const uint8_t* bs_base, int nslots, int state,
+                      int slot, void* host_dst, const float* scales, int kv, float* host_scales) {
   convkv_t* h = const_cast<convkv_t*>(hc);
-  const size_t fb = static_cast<size_t>(h->frame_elems()) * (h->fp8 ? 1 : 2);
+  const size_t fe = static_cast<size_t>(h->frame_elems());
+  const size_t fb = h->fp4 ? fe / 2 : fe * (h->fp8 ? 1 : 2);
   const char* src = static_cast<const char*>(dev_base) + (static_cast<size_t>(state) * nslots + slot) * fb;
   cudaError_t e = cudaStreamSynchronize(h->stream);
   if (e == cudaSuccess) e = cudaMemcpy(host_dst, src, fb, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && h->fp4)  // NVFP4: the block scales follow the codes
+    e = cudaMemcpy(static_cast<char*>(host_dst) + fb, bs_base + (static_cast<size_t>(state) * nslots + slot) * (fe / 16),
+                   fe / 16, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && h->fp8 && host_scales)
     e = cudaMemcpy(host_scales, scales + ((static_cast<size_t>(state) * 2 + kv) * nslots + slot) * h->H,
                    sizeof(float) * h->H, cudaMemcpyDeviceToHost);
@@ -646,14 +676,16 @@ int convkv_read_slot(const convkv_t* h, int state, int kv, int pos, void* host_d
   if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || pos < 0 || pos >= h->C)
     return CONVKV_ERR_INVALID_ARG;
   if (h->dry) return CONVKV_ERR_BAD_ORDER;
-  return read_frame(h, kv ? h->memV : h->memK, h->C, state, pos, host_dst, h->mem_scale, kv, host_scales);
+  return read_frame(h, kv ? h->memV : h->memK, kv ? h->memBV : h->memBK, h->C, state, pos, host_dst, h->mem_scale, kv,
+                    host_scales);
 }
 
 int convkv_read_ring(const convkv_t* h, int state, int kv, int slot, void* host_dst, float* host_scales) {
   if (!h || !host_dst || state < 0 || state >= h->S || (kv != 0 && kv != 1) || slot < 0 || slot >= h->R)
     return CONVKV_ERR_INVALID_ARG;
   if (h->dry) return CONVKV_ERR_BAD_ORDER;
-  return read_frame(h, kv ? h->ringV : h->ringK, h->R, state, slot, host_dst, h->ring_scale, kv, host_scales);
+  return read_frame(h, kv ? h->ringV : h->ringK, kv ? h->ringBV : h->ringBK, h->R, state, slot, host_dst,
+                    h->ring_scale, kv, host_scales);
 }
 
 int convkv_status(convkv_t* h) {

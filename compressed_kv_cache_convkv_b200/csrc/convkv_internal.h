@@ -73,6 +73,10 @@ struct AttnParams {
   const float* mem_scale;   // fp8: [S][2][C][H]
   const uint8_t* ring8[2];  // fp8: e4m3 K, V rings [S][R*T][H][D]
   const uint8_t* mem8[2];   // fp8: e4m3 K, V memory [S][C*T][H][D]
+  // NVFP4: ring8 / mem8 hold e2m1 code pairs [..][D/2], these the e4m3 block scales
+  // [..][D/16]; ring_scale / mem_scale the fp32 scales per (frame or slot, head)
+  const uint8_t* ring_bs[2];
+  const uint8_t* mem_bs[2];
   int R, C;
   int* status;
   // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
@@ -99,6 +103,9 @@ struct ConvParams {
   const float* ring_scale;    // [S][2][R][H]
   unsigned int* amax;         // [S][2][ngroups][H] fp32 bit patterns (scratch, zeroed before pass 1)
   float* mem_scale;           // [S][2][C][H]
+  // NVFP4 format: ring8 / memK / memV hold e2m1 code pairs [..][D/2], scales as below
+  const uint8_t* ring_bs[2];  // e4m3 block scales of the ring [S][R*T][H][D/16]
+  uint8_t* mem_bs[2];         // e4m3 block scales of the memory [S][C*T][H][D/16]
 };
 
 struct AppendParams {
@@ -109,6 +116,8 @@ struct AppendParams {
   unsigned int* amax;         // [S][2][b][H] fp32 bit patterns (scratch, zeroed before the amax pass)
   uint8_t* ring8[2];          // e4m3 K, V rings
   float* ring_scale;          // [S][2][R][H]
+  uint8_t* ring_bs[2];        // NVFP4: e4m3 block scales [S][R*T][H][D/16] (ring8 then holds e2m1 pairs)
+  int fp4;                    // 1: NVFP4 format
   void* stage[2];             // bf16 K, V current-block staging [S][stage_frames*T][H][D]
   int stage_frames;           // frames per state in the staging buffers (max block)
   // sequence-sharded K, V (sv.G > 0): the block's rows are gathered from the G ranks'
@@ -126,10 +135,12 @@ int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const
                      const CUtensorMap& wmap, cudaStream_t s);
 int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s);
 int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
+int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s);
 // k, v: tensor maps of buffers 0..3 (ring, memory, staging, reference frames)
+// fmt: 0 bf16, 1 e4m3, 2 NVFP4 (ring and memory segments)
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k,
-                  const CUtensorMap* v, int S, bool fp8, cudaStream_t s);
+                  const CUtensorMap* v, int S, int fmt, cudaStream_t s);
 size_t attend_smem_bytes(int D, const AttnParams& p);
 size_t conv_smem_bytes(int D);
 

@@ -28,6 +28,7 @@
 // records CONVKV_ERR_DEVICE_TIMEOUT in the status word.
 #include "convkv_internal.h"
 #include "sm100.cuh"
+#include "nvfp4.cuh"
 
 namespace ckv {
 namespace {
@@ -201,7 +202,36 @@ __device__ __forceinline__ void dequant_row(uint8_t* tile, int row, const uint8_
   }
 }
 
-template <int D, bool FP8>
+// NVFP4 row: D/2 code bytes (e2m1 pairs) and D/16 e4m3 block scales at the row's
+// offsets, fp32 scale g; bf16 value code * fp32(s_b * g), rotated (ROTATE) and
+// stored swizzled like dequant_row.  Rows past the segment store zeros.
+template <int D, bool ROTATE>
+__device__ __forceinline__ void dequant_row_fp4(uint8_t* tile, int row, const uint8_t* codes, const uint8_t* bs,
+                                                float g, bool valid, const RopeRow& rr) {
+  using C = AttnCfg<D>;
+  uint8_t* rowp = tile + row * 128;
+  const int sw = row & 7;
+  uint4 raw[D / 32];
+  uint32_t sraw[D / 64];
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) raw[k] = valid ? __ldg(reinterpret_cast<const uint4*>(codes) + k) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int k = 0; k < D / 64; ++k) sraw[k] = valid ? __ldg(reinterpret_cast<const uint32_t*>(bs) + k) : 0u;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 r4 = raw[c >> 2];
+    const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
+    const int b = c >> 1;  // block of 16 channels
+    const float e_b = __fmul_rn(fp4::e4m3_to_f32(sraw[b >> 2] >> (8 * (b & 3))), g);
+    uint32_t o[4];
+    fp4::decode8(word, e_b, o);
+    if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
+    *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// QF: storage of the ring and memory segments, 0 bf16, 1 e4m3, 2 NVFP4
+template <int D, int QF>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                 const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
@@ -209,6 +239,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                 const __grid_constant__ CUtensorMap tmV2, const __grid_constant__ CUtensorMap tmK3,
                 const __grid_constant__ CUtensorMap tmV3, const AttnParams p) {
   using C = AttnCfg<D>;
+  constexpr bool FP8 = QF != 0;  // low-precision ring and memory, dequantised in the kernel
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -420,8 +451,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             const int f = valid ? lr / p.T : 0;
             const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
             const float sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-            dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid,
-                                  RopeRow{nullptr, nullptr, nullptr});
+            if constexpr (QF == 2) {
+              const uint8_t* bsb = sg.buf == 1 ? p.mem_bs[1] : p.ring_bs[1];
+              dequant_row_fp4<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * (D / 2),
+                                        bsb + (grow * p.H + head) * (D / 16), sc, valid,
+                                        RopeRow{nullptr, nullptr, nullptr});
+            } else {
+              dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid,
+                                    RopeRow{nullptr, nullptr, nullptr});
+            }
           }
           fence_proxy_async_smem();
         }
@@ -592,7 +630,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
         const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
         const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-        dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, rr);
+        if constexpr (QF == 2) {
+          const uint8_t* bsb = sg.buf == 1 ? p.mem_bs[0] : p.ring_bs[0];
+          dequant_row_fp4<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * (D / 2),
+                                   bsb + (grow * p.H + head) * (D / 16), sc, valid, rr);
+        } else {
+          dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, rr);
+        }
       } else if (valid) {
         rope_row<D, false>(sK + ks * C::TILE, r, rr, 1.0f);
       }
@@ -618,11 +662,11 @@ size_t smem_for(const AttnParams&) {
   return C::FIXED > 120 * 1024 ? C::FIXED : 120 * 1024;
 }
 
-template <int D, bool FP8>
+template <int D, int QF>
 int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v, int S,
              cudaStream_t s) {
   const size_t smem = smem_for<D>(p);
-  auto kern = attn_kernel<D, FP8>;
+  auto kern = attn_kernel<D, QF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid((p.Nq + 255) / 256, p.H, S);
@@ -635,9 +679,15 @@ int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, co
 size_t attend_smem_bytes(int D, const AttnParams& p) { return D == 128 ? smem_for<128>(p) : smem_for<64>(p); }
 
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v,
-                  int S, bool fp8, cudaStream_t s) {
-  if (D == 128) return fp8 ? launch_t<128, true>(p, q, k, v, S, s) : launch_t<128, false>(p, q, k, v, S, s);
-  if (D == 64) return fp8 ? launch_t<64, true>(p, q, k, v, S, s) : launch_t<64, false>(p, q, k, v, S, s);
+                  int S, int fmt, cudaStream_t s) {
+  if (D == 128) {
+    if (fmt == 2) return launch_t<128, 2>(p, q, k, v, S, s);
+    return fmt ? launch_t<128, 1>(p, q, k, v, S, s) : launch_t<128, 0>(p, q, k, v, S, s);
+  }
+  if (D == 64) {
+    if (fmt == 2) return launch_t<64, 2>(p, q, k, v, S, s);
+    return fmt ? launch_t<64, 1>(p, q, k, v, S, s) : launch_t<64, 0>(p, q, k, v, S, s);
+  }
   return static_cast<int>(cudaErrorInvalidValue);
 }
 

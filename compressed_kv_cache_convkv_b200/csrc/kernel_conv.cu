@@ -15,6 +15,7 @@
 // K=16 steps) and owns the TMEM accumulator, warps 2-5 drain it.
 #include "convkv_internal.h"
 #include "sm100.cuh"
+#include "nvfp4.cuh"
 
 namespace ckv {
 namespace {
@@ -175,7 +176,9 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 // per (slot, head) = amax / 448 over the slot's [T, D] values, so the launch
 // runs twice: pass 1 only reduces amax (atomicMax on the fp32 bit pattern,
 // values are non-negative), pass 2 recomputes the same tiles and quantises
-// with that scale (round-to-nearest-even, saturating to +-448).
+// with that scale (round-to-nearest-even, saturating to +-448).  FMT 2 is the
+// NVFP4 format: e2m1 codes with an e4m3 scale per 16 channels and the fp32
+// scale per (frame or slot, head) of the same two-pass rule (nvfp4.cuh).
 __device__ __forceinline__ void e4m3x2_to_f32_c(uint32_t two, float& lo, float& hi) {
   uint32_t h2;
   asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
@@ -189,7 +192,7 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3(float lo, float hi) {
   return r;
 }
 
-template <int D, int PASS>
+template <int D, int PASS, int FMT>
 __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
     conv_fp8_kernel(const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
   using C = ConvCfg<D>;
@@ -295,10 +298,25 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
       }
       const int slot = p.grp[g].ring_slot[j];
       const float sc = __ldg(&p.ring_scale[((static_cast<int64_t>(state) * 2 + kv) * p.R + slot) * p.H + head]);
-      const uint8_t* src =
-          p.ring8[kv] + ((static_cast<int64_t>(state) * p.R * p.T + static_cast<int64_t>(slot) * p.T + token) * p.H + head) * D;
+      const int64_t grow = (static_cast<int64_t>(state) * p.R * p.T + static_cast<int64_t>(slot) * p.T + token) * p.H + head;
       uint8_t* rowp = stages + st * C::STAGE_BYTES + r * 128;
       const int sw = r & 7;
+      if (FMT == 2) {
+        // e2m1 pairs: 4 bytes per 8 channels, one e4m3 block scale per 16 channels
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.ring8[kv] + grow * (D / 2));
+        const uint8_t* bs = p.ring_bs[kv] + grow * (D / 16);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          uint32_t o[4] = {0, 0, 0, 0};
+          if (valid) {
+            const float e_b = __fmul_rn(fp4::e4m3_to_f32(__ldg(bs + (c >> 1))), sc);
+            fp4::decode8(__ldg(src + c), e_b, o);
+          }
+          *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
+              make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+      const uint8_t* src = p.ring8[kv] + grow * D;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint4 raw = valid ? __ldg(reinterpret_cast<const uint4*>(src) + k) : make_uint4(0, 0, 0, 0);
@@ -317,6 +335,7 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
           *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
               make_uint4(o[0], o[1], o[2], o[3]);
         }
+      }
       }
       fence_proxy_async_smem();
       mbar_arrive(&a_full[st]);
@@ -338,6 +357,36 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == 0) atomicMax(red, __float_as_uint(mx));
+      } else if (FMT == 2) {
+        const float gs = fp4::tensor_scale(__uint_as_float(p.amax[aidx]));
+        const int64_t row = ((static_cast<int64_t>(state) * p.C + p.grp[g].mem_pos) * p.T + token) * p.H + head;
+        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(kv ? p.memV : p.memK) + row * (D / 2));
+        uint8_t* bs = p.mem_bs[kv] + row * (D / 16);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            float xs[fp4::kBlock];
+            float a_b = 0.0f;
+#pragma unroll
+            for (int e = 0; e < fp4::kBlock; ++e) {
+              xs[e] = __uint_as_float(v[hb * 16 + e]);
+              a_b = fmaxf(a_b, fabsf(xs[e]));
+            }
+            float e_b;
+            const uint32_t sc = fp4::block_scale(a_b, gs, e_b);
+            const uint2 cw = fp4::encode_block(xs, e_b);
+            if (valid) {
+              dst[2 * c + hb] = cw;
+              bs[2 * c + hb] = static_cast<uint8_t>(sc);
+            }
+          }
+        }
+        if (mt == 0 && r == 0)
+          p.mem_scale[((static_cast<int64_t>(state) * 2 + kv) * p.C + p.grp[g].mem_pos) * p.H + head] = gs;
       } else {
         const float amax = __uint_as_float(p.amax[aidx]);
         const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
@@ -383,29 +432,39 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 
 }  // namespace
 
-int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
-  if (p.ngroups <= 0) return 0;
+namespace {
+
+template <int D, int FMT>
+int launch_lowp(const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+  using C = ConvCfg<D>;
   dim3 grid((p.T + 127) / 128, p.H, p.ngroups * p.S * 2);
+  auto k1 = conv_fp8_kernel<D, 1, FMT>;
+  auto k2 = conv_fp8_kernel<D, 2, FMT>;
+  cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  k1<<<grid, C::THREADS, C::SMEM, s>>>(wmap, p);
+  k2<<<grid, C::THREADS, C::SMEM, s>>>(wmap, p);
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <int FMT>
+int launch_lowp_d(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+  if (p.ngroups <= 0) return 0;
   cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(unsigned int) * p.S * 2 * p.ngroups * p.H, s);
   if (e != cudaSuccess) return static_cast<int>(e);
-  if (D == 128) {
-    auto k1 = conv_fp8_kernel<128, 1>;
-    auto k2 = conv_fp8_kernel<128, 2>;
-    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<128>::SMEM);
-    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<128>::SMEM);
-    k1<<<grid, ConvCfg<128>::THREADS, ConvCfg<128>::SMEM, s>>>(wmap, p);
-    k2<<<grid, ConvCfg<128>::THREADS, ConvCfg<128>::SMEM, s>>>(wmap, p);
-  } else if (D == 64) {
-    auto k1 = conv_fp8_kernel<64, 1>;
-    auto k2 = conv_fp8_kernel<64, 2>;
-    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<64>::SMEM);
-    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<64>::SMEM);
-    k1<<<grid, ConvCfg<64>::THREADS, ConvCfg<64>::SMEM, s>>>(wmap, p);
-    k2<<<grid, ConvCfg<64>::THREADS, ConvCfg<64>::SMEM, s>>>(wmap, p);
-  } else {
-    return static_cast<int>(cudaErrorInvalidValue);
-  }
-  return static_cast<int>(cudaGetLastError());
+  if (D == 128) return launch_lowp<128, FMT>(p, wmap, s);
+  if (D == 64) return launch_lowp<64, FMT>(p, wmap, s);
+  return static_cast<int>(cudaErrorInvalidValue);
+}
+
+}  // namespace
+
+int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+  return launch_lowp_d<1>(D, p, wmap, s);
+}
+
+int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+  return launch_lowp_d<2>(D, p, wmap, s);
 }
 
 

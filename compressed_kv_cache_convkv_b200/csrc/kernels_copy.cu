@@ -3,6 +3,7 @@
 // compression variant.  All HBM-bound: 16-byte vector accesses, grids sized as
 // a multiple of the SM count.
 #include "convkv_internal.h"
+#include "nvfp4.cuh"
 
 namespace ckv {
 namespace {
@@ -193,6 +194,52 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
   }
 }
 
+// NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
+// e2m1 codes into the ring, the bf16 values into staging, the tensor scale once.
+__global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
+  const int nb = p.D / fp4::kBlock;                           // blocks per token-head
+  const int64_t T = p.frame_elems / (static_cast<int64_t>(p.H) * p.D);
+  const int64_t per_frame = T * p.H * nb;
+  const int64_t per_kv = static_cast<int64_t>(p.S) * p.b * per_frame;
+  const int64_t fv = p.frame_elems / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * per_kv; i += stride) {
+    const int kv = static_cast<int>(i / per_kv);
+    const int64_t ib = i - kv * per_kv;
+    const int64_t sf = ib / per_frame;                         // s * b + f
+    const int64_t rb = ib - sf * per_frame;                    // (token * H + h) * nb + blk
+    const int s = static_cast<int>(sf / p.b);
+    const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
+    const int64_t th = rb / nb;                                // token * H + h
+    const int blk = static_cast<int>(rb - th * nb);
+    const int h = static_cast<int>(th % p.H);
+    const int64_t e0 = th * (p.D / 8) + blk * 2;               // first 16-byte vector of the block
+    const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
+    const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
+    uint4* st = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv + e0;
+    st[0] = x0;
+    st[1] = x1;
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float xs[fp4::kBlock];
+    float a_b = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      xs[2 * q] = __uint_as_float(w[q] << 16);
+      xs[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+      a_b = fmaxf(a_b, fmaxf(fabsf(xs[2 * q]), fabsf(xs[2 * q + 1])));
+    }
+    const float g = fp4::tensor_scale(__uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]));
+    float e_b;
+    const uint32_t sc = fp4::block_scale(a_b, g, e_b);
+    int slot = p.slot0 + f;
+    if (slot >= p.R) slot -= p.R;
+    const int64_t row = (static_cast<int64_t>(s) * p.R + slot) * T * p.H + th;   // token-head row in the ring
+    reinterpret_cast<uint2*>(p.ring8[kv])[row * nb + blk] = fp4::encode_block(xs, e_b);
+    p.ring_bs[kv][row * nb + blk] = static_cast<uint8_t>(sc);
+    if (th < p.H && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
+  }
+}
+
 }  // namespace
 
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
@@ -229,6 +276,12 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
                                                                  static_cast<const uint4*>(v), p, rows_per_block);
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
+  if (p.fp4) {
+    const int64_t blocks = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / fp4::kBlock);
+    append_quant_fp4_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(static_cast<const uint4*>(k),
+                                                                   static_cast<const uint4*>(v), p);
+    return static_cast<int>(cudaGetLastError());
+  }
   const int64_t total = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
   append_quant_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());

@@ -52,6 +52,9 @@ extern "C" {
 
 #define CONVKV_KV_BF16 0               /* cache stored in bf16 */
 #define CONVKV_KV_FP8_E4M3 1           /* window + memory stored e4m3 with per-(head, frame) fp32 scale */
+#define CONVKV_KV_NVFP4 2              /* window + memory stored NVFP4: e2m1 pairs, an e4m3 scale per 16
+                                          channels, an fp32 scale per (head, frame) (model card, open-source
+                                          plan: FP4 for B-series GPUs, read as NVFP4) */
 
 #define CONVKV_COMPRESS_CONV 0         /* 1D conv, kernel 5, stride 5 (the method) */
 #define CONVKV_COMPRESS_MEAN 1         /* mean of the 5 evicted frames (--mean_memory option) */
@@ -71,7 +74,7 @@ typedef struct convkv_cfg {
   int mem_slots;           /* C >= 1: FIFO capacity of compressed slots */
   int rope_t, rope_h, rope_w; /* RoPE channels per axis (even, sum = D); all 0 -> D-4*floor(D/6), 2*floor(D/6), 2*floor(D/6) */
   double rope_theta;       /* RoPE base, e.g. 1e4 */
-  int kv_format;           /* CONVKV_KV_BF16 or CONVKV_KV_FP8_E4M3 */
+  int kv_format;           /* CONVKV_KV_BF16, CONVKV_KV_FP8_E4M3 or CONVKV_KV_NVFP4 */
   int compress_mode;       /* CONVKV_COMPRESS_CONV or CONVKV_COMPRESS_MEAN */
   int num_states;          /* independent states advanced together (>= 1) */
   int flags;               /* CONVKV_FLAG_* */
@@ -187,8 +190,10 @@ int convkv_counters(const convkv_t* h, int64_t out[8]);
 
 /* Copy one stored memory slot (memory position `pos` in [0, C)) of one state
  * and one of K (kv = 0) or V (kv = 1) to host memory: [T][H][D] bf16, or e4m3
- * bytes in the fp8 format with scales[H] fp32 written to host_scales (may be
- * NULL for bf16).  Synchronises the stream.  Errors: INVALID_ARG, BAD_ORDER, CUDA. */
+ * bytes in the fp8 format, or in the NVFP4 format [T][H][D/2] bytes of e2m1 pairs
+ * (even channel in the low nibble) followed by [T][H][D/16] e4m3 block scales;
+ * the fp32 scales[H] of the low-precision formats go to host_scales (may be
+ * NULL).  Synchronises the stream.  Errors: INVALID_ARG, BAD_ORDER, CUDA. */
 int convkv_read_slot(const convkv_t* h, int state, int kv, int pos, void* host_dst, float* host_scales);
 
 /* Copy one ring frame slot (`slot` in [0, W + max(b1, b))) the same way. */

@@ -23,7 +23,7 @@ FP8_MAX = 5e-2
 
 def oracle_for(w, state: int = 0, conv_w: Optional[np.ndarray] = None, mean: bool = False) -> O.OracleStream:
     cfg = O.OracleConfig(H=w.heads, D=w.head_dim, grid_h=w.grid_h, grid_w=w.grid_w, window=w.window_frames,
-                         mem_slots=w.mem_slots, fp8=w.fp8)
+                         mem_slots=w.mem_slots, fp8=w.fp8, fp4=getattr(w, "fp4", False))
     if mean:
         wts = np.zeros((2, w.heads, w.head_dim, w.head_dim, 5))
         for o in range(w.head_dim):
@@ -148,3 +148,58 @@ def check_codes(gpu_bytes: np.ndarray, gpu_scales: np.ndarray, ref_codes: np.nda
         step = np.exp2(np.maximum(ex - 1.0, -6.0) - 3.0)      # e4m3 quantum at the reference value
         assert np.all(np.abs(g[diff] - ref_codes[diff]) <= step * 2 + 1e-30), (what, "code step")
     return {"mismatch": frac}
+
+
+# -- NVFP4 ------------------------------------------------------------------
+
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_pairs_to_f64(pairs: np.ndarray) -> np.ndarray:
+    """bytes [..., D/2] of e2m1 pairs (even channel in the low nibble) -> values [..., D]."""
+    b = np.asarray(pairs, dtype=np.uint8)
+    nib = np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], b.shape[-1] * 2)
+    val = E2M1_VALUES[nib & 7]
+    return np.where(nib & 8, -val, val)
+
+
+def fp4_values(codes: np.ndarray, bs: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """code * fp32(s_b * g) in fp32, for values [T, H, D], block scales [T, H, D/16], g[H]."""
+    T, H, D = codes.shape
+    eb = (np.asarray(bs, np.float32) * np.asarray(g, np.float32)[None, :, None]).astype(np.float32)
+    return (codes.astype(np.float32).reshape(T, H, D // 16, 16) * eb[..., None]).astype(np.float32).reshape(T, H, D)
+
+
+def check_codes_fp4(gpu, ref, exact: bool, what: str = "", max_frac: float = 0.0) -> dict:
+    """gpu = (e2m1 pair bytes [T, H, D/2], (e4m3 block scale bytes [T, H, D/16], g[H]));
+    ref = (code values [T, H, D], (block scale values [T, H, D/16], g[H])) from the oracle.
+
+    exact: every code, block scale and tensor scale equal.  Otherwise (quantised conv
+    outputs: fp32 accumulation on the GPU against fp64 in the oracle) tensor scales
+    within 1e-5 relative, and the fraction of channels whose dequantised value differs
+    by more than that at most max_frac; such a value is within one e2m1 step at the
+    larger of the two block scales (values next to a rounding boundary, of a code or
+    of its block's scale)."""
+    gc, (gb, gg) = gpu
+    rc, (rb, rg) = ref
+    gcv = e2m1_pairs_to_f64(gc)
+    gbv = e4m3_bytes_to_f64(gb)
+    if exact:
+        assert np.array_equal(gg, np.asarray(rg, np.float32)), (what, "tensor scales")
+        assert np.array_equal(gbv, rb), (what, "block scales", int(np.sum(gbv != rb)))
+        assert np.array_equal(gcv, rc), (what, "codes", int(np.sum(gcv != rc)))
+        return {"mismatch": 0.0}
+    rs = np.abs(gg.astype(np.float64) / np.asarray(rg, np.float64) - 1).max()
+    assert rs <= 1e-5, (what, "tensor scale", rs)
+    gv, rv = fp4_values(gcv, gbv, gg), fp4_values(rc, rb, rg)
+    # same code and block scale: the values differ only through g (<= 1e-5 relative)
+    diff = np.abs(gv.astype(np.float64) - rv) > 2e-5 * np.abs(rv)
+    frac = float(diff.mean())
+    assert frac <= max_frac, (what, "value mismatch fraction", frac)
+    if diff.any():
+        T, H, D = rc.shape
+        eg = (gbv.astype(np.float32) * gg[None, :, None]).repeat(16, axis=2)
+        er = (rb.astype(np.float32) * np.asarray(rg, np.float32)[None, :, None]).repeat(16, axis=2)
+        step = 2.0 * np.maximum(eg, er)                      # the largest e2m1 step is 2 (between 4 and 6)
+        assert np.all(np.abs(gv - rv)[diff] <= step[diff] * 1.0001 + 1e-30), (what, "value step")
+    return {"mismatch": frac, "block_scale_mismatch": float((gbv != rb).mean())}

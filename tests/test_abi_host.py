@@ -53,6 +53,10 @@ def test_invalid_configs_rejected():
         (base.with_(rope_theta=0.0), ckv.ERR_INVALID_ARG),
         (base.with_(grid_h=4096, grid_w=4096), ckv.ERR_UNSUPPORTED),
         (base.with_(sink_frames=-1), ckv.ERR_INVALID_ARG),
+        (base.with_(kv_format=3), ckv.ERR_INVALID_ARG),
+        (base.with_(kv_format=ckv.KV_NVFP4, compress_mode=ckv.COMPRESS_MEAN), ckv.ERR_UNSUPPORTED),
+        (base.with_(sp_ranks=9), ckv.ERR_INVALID_ARG),
+        (base.with_(sp_ranks=2, sp_rank=2), ckv.ERR_INVALID_ARG),
         (base.with_(sink_frames=100000), ckv.ERR_UNSUPPORTED),   # RoPE time table too large
     ]
     for cfg, code in bad:
@@ -88,7 +92,7 @@ def _oracle_layout(st):
     return [(int(p), int(s), int(t)) for p, s, t in st.layout()]
 
 
-@pytest.mark.parametrize("name", ["tiny", "512x512", "720x416", "fp8_480x832"])
+@pytest.mark.parametrize("name", ["tiny", "512x512", "720x416", "fp8_480x832", "nvfp4_480x832"])
 def test_bookkeeping_matches_oracle_every_block(name):
     w = PRESETS[name]
     h = _dry(w)
@@ -105,7 +109,7 @@ def test_bookkeeping_matches_oracle_every_block(name):
         assert [tuple(r) for r in lay[:, [0, 1, 3]]] == _oracle_layout(st)
         # physical slots: memory position = slot mod C, ring slot = frame mod R
         for part, src, phys, _ in lay:
-            if part == 2 and w.fp8:      # fp8: the current block sits in bf16 staging
+            if part == 2 and (w.fp8 or w.fp4):   # low precision: the current block sits in bf16 staging
                 assert phys == src - st.P
             else:
                 assert phys == (src % w.mem_slots if part == 0 else src % R)

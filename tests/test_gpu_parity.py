@@ -12,8 +12,12 @@ import seeded_inputs as si
 from compressed_kv_cache_convkv_b200.configs import PRESETS, Workload
 from dataclasses import replace
 
-from streams import (attention_errors, bf16_tensor_to_f64, check_attention, check_codes, check_slot, device_frames,
-                     device_weights, host_frames, oracle_for, sample_rows)
+from streams import (attention_errors, bf16_tensor_to_f64, check_attention, check_codes, check_codes_fp4, check_slot,
+                     device_frames, device_weights, host_frames, oracle_for, sample_rows)
+
+# NVFP4 conv outputs: fraction of channels allowed to sit one step apart (a code or its
+# block scale next to a rounding boundary; 8e-6 at most on the 480x832 stream)
+FP4_VALUE_MISMATCH = 1e-4
 
 pytestmark = pytest.mark.gpu
 
@@ -193,7 +197,8 @@ def test_720_stream_ragged(torch):
 
 
 def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, ring_frames=None, sink=0):
-    """fp8 format: window codes bit-exact, memory codes within one step, attention <= 5e-2."""
+    """Low-precision formats (e4m3, or NVFP4 when w.fp4): window codes and scales bit-exact,
+    memory codes within one step, attention <= 5e-2."""
     ckv = _ckv()
     weights = device_weights(w, torch)
     cfg = w.config(sink_frames=sink)
@@ -216,20 +221,28 @@ def _run_fp8(torch, w: Workload, states=(0,), attend_blocks=None, rows=None, rin
                 lay = h.layout()
                 assert [tuple(r) for r in lay[:, [0, 1, 3]]] == [tuple(r) for r in st.layout()], f"block {n}"
                 assert [int(x) for x in lay[lay[:, 0] == 2, 2]] == list(range(b))  # staging slots
-            # the new block's e4m3 ring codes and scales: bit-exact
+            # the new block's ring codes and scales: bit-exact
             frames = range(b) if ring_frames is None else [x for x in ring_frames if x < b]
             for f in frames:
                 ck, sk, cv, sv = st.current_q8[f].codes
                 for kv, (rc, rsc) in enumerate(((ck, sk), (cv, sv))):
                     gb, gs = h.read_ring(s, kv, (F + f) % R)
-                    check_codes(gb, gs, rc, rsc, exact=True, what=f"state {s} frame {F + f} kv {kv}")
+                    what = f"state {s} frame {F + f} kv {kv}"
+                    if w.fp4:
+                        check_codes_fp4((gb, gs), (rc, rsc), exact=True, what=what)
+                    else:
+                        check_codes(gb, gs, rc, rsc, exact=True, what=what)
             # new memory slots: codes within one step of the oracle's
             for e in ev[-cfg.mem_slots:]:
                 age = st.m - (st.S - e.slot)
                 ck, sk, cv, sv = st.memory[age].codes
                 for kv, (rc, rsc) in enumerate(((ck, sk), (cv, sv))):
                     gb, gs = h.read_slot(s, kv, e.slot % cfg.mem_slots)
-                    check_codes(gb, gs, rc, rsc, exact=False, what=f"state {s} slot {e.slot} kv {kv}")
+                    what = f"state {s} slot {e.slot} kv {kv}"
+                    if w.fp4:
+                        check_codes_fp4((gb, gs), (rc, rsc), exact=False, what=what, max_frac=FP4_VALUE_MISMATCH)
+                    else:
+                        check_codes(gb, gs, rc, rsc, exact=False, what=what)
             if attend_blocks is None or n in attend_blocks:
                 qh = host_frames(w, si.Q, s, F, b)
                 r = sample_rows(w, b, rows or b * w.T, rng)
@@ -281,3 +294,15 @@ def test_tiny_fp8_reference_frames_two_states(torch):
     """fp8 window/memory with bf16 reference frames, one per state."""
     w = replace(PRESETS["tiny"], fp8=True, num_states=2, name="tiny_fp8")
     _run_fp8(torch, w, states=(0, 1), sink=1)
+
+
+# -- NVFP4 window and memory -------------------------------------------------
+
+def test_tiny_nvfp4_two_states(torch):
+    w = replace(PRESETS["tiny"], fp4=True, num_states=2, name="tiny_nvfp4")
+    _run_fp8(torch, w, states=(0, 1))
+
+
+def test_nvfp4_480x832_40_states(torch):
+    _run_fp8(torch, PRESETS["nvfp4_480x832"], states=(0, 39), attend_blocks={1, 2, 5, 9, 17, 25}, rows=32,
+             ring_frames=[0, 7])
