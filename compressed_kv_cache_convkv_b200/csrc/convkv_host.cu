@@ -11,6 +11,13 @@
 //   attend:    keys = the r reference frames at time 0..r-1 (r = sink_frames, given
 //              once, never evicted), stored slots S-m .. S-1 (m = min(S, C)) at
 //              time r..r+m-1, then frames E .. P+b-1 at time r + m + (f - E).
+//
+// RoPE is relative, so the time table of a step may hold any common shift of these
+// indices.  Each append rebuilds it for absolute positions B0 + i, B0 = E - r - m
+// (+ t_offset): table row i then serves reset time index i, and a window or
+// current frame's row is its stream index q - B0, so a key rotated at append time
+// at stream position q stays valid at every later attend (bf16 format: the ring
+// keeps an un-rotated K for the conv and a rotated copy for the attention).
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -53,7 +60,7 @@ struct convkv {
   int G = 1, g = 0;  // sequence-parallel group size and this handle's rank
   int PT = 0, PH = 0, PW = 0, tab_t_rows = 0;
   // fp8: the ring and memory are stored in a low-precision format (e4m3, or NVFP4 when fp4)
-  bool dry = false, mean = false, fp8 = false, fp4 = false, host_io = false, sink_set = false;
+  bool dry = false, mean = false, fp8 = false, fp4 = false, host_io = false, sink_set = false, prerot = false;
   // bookkeeping
   int64_t P = 0, E = 0, Sn = 0, blocks = 0;
   int bcur = 0, last_groups = 0;
@@ -61,6 +68,8 @@ struct convkv {
   void* arena = nullptr;
   size_t arena_bytes = 0;
   void *ringK = nullptr, *ringV = nullptr, *memK = nullptr, *memV = nullptr, *weights = nullptr;
+  void* ringKr = nullptr;           // bf16 format: K of the ring rotated at its stream position
+  std::vector<float4> tab_t_host;   // time table rows of the current step (host copy)
   // fp8 format: ringK/ringV/memK/memV hold e4m3 codes; scales per (state, K|V, slot, head)
   float *ring_scale = nullptr, *mem_scale = nullptr;
   void *stageK = nullptr, *stageV = nullptr;  // bf16 copy of the current block
@@ -71,7 +80,7 @@ struct convkv {
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
-  CUtensorMap mapRingK{}, mapRingV{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
+  CUtensorMap mapRingK{}, mapRingV{}, mapRingKr{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
       mapSinkV{};
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
@@ -164,30 +173,31 @@ ShardView make_view(const convkv* h, int frames) {
   return v;
 }
 
-void build_tables(const convkv* h, std::vector<float4>& out) {
-  // axis with global pairs [g, g + n), positions 0..rows-1 (+offset): for pair i of the
-  // axis the angle is pos * theta^(-2i/(2n)); units pack the pairs 2k, 2k+1 as
-  // (cos, cos, sin, sin), zero for a pair outside the axis
-  auto axis = [&](int rows, int g, int n, int offset) {
-    const int units = rope_units(g, n);
-    for (int r = 0; r < rows; ++r)
-      for (int u = 0; u < units; ++u) {
-        float c[2] = {0.f, 0.f}, sn[2] = {0.f, 0.f};
-        for (int q = 0; q < 2; ++q) {
-          const int gp = 2 * (g / 2 + u) + q;  // global pair
-          if (gp < g || gp >= g + n) continue;
-          const int i = gp - g;
-          const double freq = std::pow(h->cfg.rope_theta, -2.0 * i / (2.0 * n));
-          const double ang = static_cast<double>(r + offset) * freq;
-          c[q] = static_cast<float>(std::cos(ang));
-          sn[q] = static_cast<float>(std::sin(ang));
-        }
-        out.push_back(make_float4(c[0], c[1], sn[0], sn[1]));
+// axis with global pairs [g, g + n), positions offset .. offset+rows-1: for pair i of the
+// axis the angle is pos * theta^(-2i/(2n)); units pack the pairs 2k, 2k+1 as
+// (cos, cos, sin, sin), zero for a pair outside the axis
+void table_axis(const convkv* h, std::vector<float4>& out, int rows, int g, int n, int64_t offset) {
+  const int units = rope_units(g, n);
+  for (int r = 0; r < rows; ++r)
+    for (int u = 0; u < units; ++u) {
+      float c[2] = {0.f, 0.f}, sn[2] = {0.f, 0.f};
+      for (int q = 0; q < 2; ++q) {
+        const int gp = 2 * (g / 2 + u) + q;  // global pair
+        if (gp < g || gp >= g + n) continue;
+        const int i = gp - g;
+        const double freq = std::pow(h->cfg.rope_theta, -2.0 * i / (2.0 * n));
+        const double ang = static_cast<double>(r + offset) * freq;
+        c[q] = static_cast<float>(std::cos(ang));
+        sn[q] = static_cast<float>(std::sin(ang));
       }
-  };
-  axis(h->tab_t_rows, 0, h->PT, h->cfg.t_offset);
-  axis(h->gh, h->PT, h->PH, 0);
-  axis(h->gw, h->PT + h->PH, h->PW, 0);
+      out.push_back(make_float4(c[0], c[1], sn[0], sn[1]));
+    }
+}
+
+void build_tables(const convkv* h, std::vector<float4>& out) {
+  table_axis(h, out, h->tab_t_rows, 0, h->PT, h->cfg.t_offset);
+  table_axis(h, out, h->gh, h->PT, h->PH, 0);
+  table_axis(h, out, h->gw, h->PT + h->PH, h->PW, 0);
 }
 
 }  // namespace
@@ -240,6 +250,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->mean = cfg->compress_mode == CONVKV_COMPRESS_MEAN;
   h->fp8 = cfg->kv_format != CONVKV_KV_BF16;
   h->fp4 = cfg->kv_format == CONVKV_KV_NVFP4;
+  h->prerot = !h->fp8;
   h->stream = static_cast<cudaStream_t>(cfg->stream);
   h->cfg.conv_weight = nullptr;
   if (h->dry) {
@@ -265,6 +276,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t tab_b = tab.size() * sizeof(float4);
   const size_t io_b = h->host_io ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
   const size_t sink_b = static_cast<size_t>(h->S) * h->Rs * fe * 2;
+  const size_t rkr_b = h->prerot ? ring_b : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -275,7 +287,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
                o_tab = take(tab_b), o_st = take(sizeof(int)), o_q = take(io_b), o_k = take(io_b),
                o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
                o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b),
-               o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b);
+               o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b),
+               o_rkr = take(rkr_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -305,6 +318,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->memBK = reinterpret_cast<uint8_t*>(a + o_mbk);
     h->memBV = reinterpret_cast<uint8_t*>(a + o_mbv);
   }
+  if (h->prerot) h->ringKr = a + o_rkr;
   if (h->Rs) {
     h->sinkK = a + o_rfk;
     h->sinkV = a + o_rfv;
@@ -333,6 +347,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     if (!rc) rc = encode_4d(&h->mapStageV, h->stageV, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
   } else {
     rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapRingKr, h->ringKr, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapRingV, h->ringV, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
@@ -423,7 +438,16 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
     }
     if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   }
-  // 3. the new block becomes the current block: copy into ring slots (P + f) mod R
+  // 3. the time table of this step: absolute positions B0 + i, B0 = E - r - m (+ t_offset)
+  {
+    h->tab_t_host.clear();
+    const int64_t B0 = h->E - h->Rs - h->m() + h->cfg.t_offset;
+    table_axis(h, h->tab_t_host, h->tab_t_rows, 0, h->PT, B0);
+    cudaError_t e = cudaMemcpyAsync(h->tables, h->tab_t_host.data(), h->tab_t_host.size() * sizeof(float4),
+                                    cudaMemcpyHostToDevice, h->stream);
+    if (e != cudaSuccess) return h->cuda_fail(e);
+  }
+  // 4. the new block becomes the current block: copy into ring slots (P + f) mod R
   AppendParams ap{};
   ap.S = h->S;
   ap.b = frames;
@@ -432,6 +456,14 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
   ap.frame_elems = h->frame_elems();
   ap.H = h->H;
   ap.D = h->D;
+  if (h->prerot) {
+    ap.ringKr = h->ringKr;
+    ap.tables = h->tables;
+    ap.tab_t_rows = h->tab_t_rows;
+    ap.tab_h_rows = h->gh;
+    ap.t_row0 = h->Rs + h->m() + h->w();
+    ap.grid_w = h->gw;
+  }
   if (k_sh) {
     ap.sv = make_view(h, frames);
     for (int r = 0; r < h->G; ++r) {
@@ -510,6 +542,7 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     s.t0 = t0;
     s.tile0 = tiles;
     s.fp8 = (h->fp8 && buf < 2) ? 1 : 0;
+    s.prerot = (h->prerot && buf == 0) ? 1 : 0;
     s.slot0 = frame0;
     tiles += (s.nrows + 127) / 128;
   };
@@ -567,7 +600,7 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     km[0] = km[1] = km[2] = h->mapStageK;  // only staging and reference maps are used by TMA
     vm[0] = vm[1] = vm[2] = h->mapStageV;
   } else {
-    km[0] = h->mapRingK; km[1] = h->mapMemK; km[2] = h->mapRingK;
+    km[0] = h->mapRingKr; km[1] = h->mapMemK; km[2] = h->mapRingK;
     vm[0] = h->mapRingV; vm[1] = h->mapMemV; vm[2] = h->mapRingV;
   }
   km[3] = r ? h->mapSinkK : km[2];

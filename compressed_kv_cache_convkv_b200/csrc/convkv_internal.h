@@ -31,7 +31,7 @@ struct KeySeg {
   int tile0;   // index of the segment's first 128-row key tile in the attend's tile list
   int fp8;     // 1 if the rows are e4m3 with per-(frame, head) fp32 scales
   int slot0;   // ring slot or memory position of the segment's first frame (row0 / T)
-  int pad;
+  int prerot;  // 1 if the K rows are stored already rotated (window and current block, bf16)
 };
 
 // A block's rows (frames * T tokens) split into G contiguous sequence shards, one
@@ -125,6 +125,11 @@ struct AppendParams {
   ShardView sv;
   const void* k_sh[kMaxRanks];
   const void* v_sh[kMaxRanks];
+  // bf16 format: K is also stored rotated (ringKr) with the RoPE tables of the step;
+  // frame f of the block sits at table row t_row0 + f, token s at (s / grid_w, s % grid_w)
+  void* ringKr;
+  const float4* tables;
+  int tab_t_rows, tab_h_rows, t_row0, grid_w;
 };
 
 // Kernel launchers (return cudaError_t of the launch).

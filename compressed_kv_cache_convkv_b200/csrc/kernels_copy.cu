@@ -4,6 +4,7 @@
 // a multiple of the SM count.
 #include "convkv_internal.h"
 #include "nvfp4.cuh"
+#include "rope.cuh"
 
 namespace ckv {
 namespace {
@@ -37,12 +38,20 @@ __device__ __forceinline__ const uint4* block_vec(const void* plain, const void*
 
 // Append (SoulX-LiveAct blog, "ConvKV Memory": append-only KV -- only the new
 // tokens' K/V are written, cached entries are never recomputed).
-// k, v: [S][b*T][H][D] bf16 -> ring slot (slot0 + f) % R of each state.
+// k, v: [S][b*T][H][D] bf16 -> ring slot (slot0 + f) % R of each state.  K is also
+// written rotated into ringKr at the same place: a window or current-block key
+// keeps its RoPE position relative to every later query (both are stream
+// positions), so it is rotated once here instead of at every attend.
+template <int D>
 __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                    uint4* __restrict__ ringK, uint4* __restrict__ ringV, AppendParams p) {
+  using RC = RopeCfg<D>;
   const int64_t fv = p.frame_elems / 8;  // 16-byte vectors per frame
+  const int vpr = p.H * D / 8;           // vectors per token
   const int64_t total = static_cast<int64_t>(p.S) * p.b * fv;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
+  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     const int64_t sf = i / fv;               // state * b + f
     const int64_t e = i - sf * fv;
@@ -55,6 +64,16 @@ __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __r
     const uint4 vv = __ldcs(block_vec(v, p.v_sh, p, s, f, e));
     ringK[dst] = kv;
     ringV[dst] = vv;
+    if (p.ringKr) {
+      const int tok = static_cast<int>(e / vpr);
+      const int c = static_cast<int>(e % (D / 8));  // chunk of 8 channels within the head
+      const int y = tok / p.grid_w, x = tok - (tok / p.grid_w) * p.grid_w;
+      const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.t_row0 + f) * RC::UT, tab_h + y * RC::UH,
+                            tab_w + x * RC::UW};
+      uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+      dev::rope_chunk<D, false>(w, c, rr, 1.0f);
+      static_cast<uint4*>(p.ringKr)[dst] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
@@ -245,8 +264,9 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
                        cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
-  append_bf16_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
-                                                          static_cast<uint4*>(ringK), static_cast<uint4*>(ringV), p);
+  auto kern = p.D == 128 ? append_bf16_kernel<128> : append_bf16_kernel<64>;
+  kern<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                                            static_cast<uint4*>(ringK), static_cast<uint4*>(ringV), p);
   return static_cast<int>(cudaGetLastError());
 }
 
