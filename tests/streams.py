@@ -14,7 +14,7 @@ import numpy as np
 import seeded_inputs as si
 from oracle import convkv_oracle as O
 
-# tolerances (spec bounds; relative form for compressed K/V of magnitude > 1,
+# tolerances (the target bounds; relative form for compressed K/V of magnitude > 1,
 # plus a relative-L2 gate on attention outputs whose magnitude is ~1e-2)
 ATT_MAX, ATT_MEAN, ATT_REL_L2 = 1e-2, 1e-3, 1e-2
 SLOT_MAX_REL, SLOT_MEAN = 1e-2, 1e-3
