@@ -174,3 +174,40 @@ def test_first_conv_at_block_3_for_512():
         h.dry_append(b)
         groups.append(h.counters()["groups"])
     assert groups[:3] == [0, 0, 1]
+
+
+def test_sequence_parallel_argument_checks():
+    """Host-side checks of the sequence-parallel forms (no CUDA call is reached)."""
+    lib = ckv.library()
+    w = PRESETS["tiny"]
+    plain = _dry(w)
+    two = (ctypes.c_void_p * 2)(1, 2)
+    # the SP forms need a handle created with sp_ranks >= 2
+    assert lib.convkv_append_block_sp(plain._h, two, two, 2) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_attend_sp(plain._h, two, two) == ckv.ERR_INVALID_ARG
+    sp = _dry(w, heads=1, sp_ranks=2, sp_rank=1)
+    assert lib.convkv_attend_sp(sp._h, two, two) == ckv.ERR_BAD_ORDER      # nothing appended yet
+    assert lib.convkv_append_block_sp(sp._h, two, two, 0) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_append_block_sp(sp._h, two, two, 2) == ckv.OK        # dry run: bookkeeping only
+    assert lib.convkv_attend_sp(sp._h, two, two) == ckv.OK
+    assert sp.counters()["b"] == 2
+    # the IPC helpers reject null arguments before touching CUDA
+    assert lib.convkv_ipc_export(None, None, None) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_ipc_open(None, None) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_ipc_close(None) == ckv.ERR_INVALID_ARG
+
+
+def test_low_precision_formats_share_the_bookkeeping():
+    """e4m3 and NVFP4 handles keep the bf16 bookkeeping; only the current block's
+    physical slots (staging) differ."""
+    w = PRESETS["fp8_480x832"]
+    hs = {fmt: _dry(w, kv_format=fmt) for fmt in (ckv.KV_BF16, ckv.KV_FP8_E4M3, ckv.KV_NVFP4)}
+    for b in w.block_sizes()[:12]:
+        for h in hs.values():
+            h.dry_append(b)
+        lays = {fmt: h.layout() for fmt, h in hs.items()}
+        ref = lays[ckv.KV_BF16]
+        for fmt in (ckv.KV_FP8_E4M3, ckv.KV_NVFP4):
+            assert np.array_equal(lays[fmt][:, [0, 1, 3]], ref[:, [0, 1, 3]])
+            cur = lays[fmt][:, 0] == 2
+            assert list(lays[fmt][cur, 2]) == list(range(int(cur.sum())))
