@@ -194,7 +194,7 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3(float lo, float hi) {
 
 template <int D, int PASS, int FMT>
 __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
-    conv_fp8_kernel(const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
+    conv_lowp_kernel(const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
   using C = ConvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -438,8 +438,8 @@ template <int D, int FMT>
 int launch_lowp(const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
   using C = ConvCfg<D>;
   dim3 grid((p.T + 127) / 128, p.H, p.ngroups * p.S * 2);
-  auto k1 = conv_fp8_kernel<D, 1, FMT>;
-  auto k2 = conv_fp8_kernel<D, 2, FMT>;
+  auto k1 = conv_lowp_kernel<D, 1, FMT>;
+  auto k2 = conv_lowp_kernel<D, 2, FMT>;
   cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   k1<<<grid, C::THREADS, C::SMEM, s>>>(wmap, p);
