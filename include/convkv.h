@@ -66,7 +66,8 @@ extern "C" {
 typedef struct convkv_cfg {
   int heads;               /* H */
   int head_dim;            /* D: 64 or 128 */
-  int grid_h, grid_w;      /* tokens per latent frame T = grid_h * grid_w (each <= 255) */
+  int grid_h, grid_w;      /* tokens per latent frame T = grid_h * grid_w; UNSUPPORTED when the RoPE
+                              tables exceed 256 KB or T * max(ring frames, mem_slots) > 2^30 */
   int first_block_frames;  /* b1: frames of the first block */
   int block_frames;        /* b : frames of later blocks; any append may carry 1..max(b1, b) frames */
   int window_frames;       /* W >= 4: past-block frames kept exact */
