@@ -50,6 +50,7 @@ _SIGNATURES = {
     "convkv_status": (ctypes.c_int, [_P]),
     "convkv_launch_count": (ctypes.c_int64, [_P]),
     "convkv_last_cuda_error": (ctypes.c_int, [_P]),
+    "convkv_debug_fail_step": (ctypes.c_int, [_P, ctypes.c_int]),
     "convkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "convkv_quantize_e4m3_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_int, _P]),

@@ -85,10 +85,26 @@ struct convkv {
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
   int last_cuda = 0;
+  // host-side failure injection (tests): the fail_at-th launch step of the next
+  // append reports a launch failure instead of running
+  int fail_at = -1, steps = 0;
+  // set when an append failed after rolling back its counters: a conv of that call
+  // may already have rewritten a memory position, so attends wait for the next
+  // successful append
+  bool need_append = false;
 
   int cuda_fail(cudaError_t e) {
     last_cuda = static_cast<int>(e);
     return CONVKV_ERR_CUDA;
+  }
+  // Called before every launch step of an append (also in dry-run mode, where the
+  // step itself is skipped); returns the injected error once when armed.
+  cudaError_t step_gate() {
+    if (fail_at >= 0 && steps++ == fail_at) {
+      fail_at = -1;
+      return cudaErrorLaunchFailure;
+    }
+    return cudaSuccess;
   }
   int64_t frame_elems() const { return static_cast<int64_t>(T) * H * D; }
   int m() const { return static_cast<int>(Sn < C ? Sn : C); }
@@ -384,8 +400,10 @@ int64_t convkv_launch_count(const convkv_t* h) { return h ? h->launches : 0; }
 
 int convkv_last_cuda_error(const convkv_t* h) { return h ? h->last_cuda : 0; }
 
-static int append_impl(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
-                       const void* const* v_sh, int frames) {
+// The steps of one append.  Advances the counters first (the launches read the new
+// ones); append_impl restores them when a step fails.
+static int append_steps(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
+                        const void* const* v_sh, int frames) {
   // 1. the previous current block joins the window
   h->P += h->bcur;
   // 2. evict groups of 5 while the window holds more than W frames
@@ -400,46 +418,49 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
   const size_t first = groups.size() > static_cast<size_t>(h->C) ? groups.size() - h->C : 0;
   h->bcur = frames;
   h->blocks += 1;
-  if (h->dry) return CONVKV_OK;
 
   if (groups.size() > first) {
-    ConvParams cp{};
-    cp.H = h->H;
-    cp.T = h->T;
-    cp.S = h->S;
-    cp.C = h->C;
-    cp.R = h->R;
-    cp.ngroups = static_cast<int>(groups.size() - first);
-    for (size_t g = first; g < groups.size(); ++g) {
-      ConvGroup& cg = cp.grp[g - first];
-      for (int j = 0; j < kEvict; ++j) cg.ring_slot[j] = static_cast<int>((groups[g].first + j) % h->R);
-      cg.mem_pos = static_cast<int>(groups[g].second % h->C);
+    if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
+    if (!h->dry) {
+      ConvParams cp{};
+      cp.H = h->H;
+      cp.T = h->T;
+      cp.S = h->S;
+      cp.C = h->C;
+      cp.R = h->R;
+      cp.ngroups = static_cast<int>(groups.size() - first);
+      for (size_t g = first; g < groups.size(); ++g) {
+        ConvGroup& cg = cp.grp[g - first];
+        for (int j = 0; j < kEvict; ++j) cg.ring_slot[j] = static_cast<int>((groups[g].first + j) % h->R);
+        cg.mem_pos = static_cast<int>(groups[g].second % h->C);
+      }
+      cp.memK = h->memK;
+      cp.memV = h->memV;
+      cp.status = h->status;
+      int e;
+      if (h->fp8) {
+        cp.ring8[0] = static_cast<const uint8_t*>(h->ringK);
+        cp.ring8[1] = static_cast<const uint8_t*>(h->ringV);
+        cp.ring_scale = h->ring_scale;
+        cp.amax = h->amax;
+        cp.mem_scale = h->mem_scale;
+        cp.ring_bs[0] = h->ringBK;
+        cp.ring_bs[1] = h->ringBV;
+        cp.mem_bs[0] = h->memBK;
+        cp.mem_bs[1] = h->memBV;
+        e = h->fp4 ? launch_conv_fp4(h->D, cp, h->mapW, h->stream) : launch_conv_fp8(h->D, cp, h->mapW, h->stream);
+        h->launches += 2;
+      } else {
+        e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
+                    : launch_conv_bf16(h->D, cp, h->mapRingK, h->mapRingV, h->mapW, h->stream);
+        h->launches++;
+      }
+      if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
     }
-    cp.memK = h->memK;
-    cp.memV = h->memV;
-    cp.status = h->status;
-    int e;
-    if (h->fp8) {
-      cp.ring8[0] = static_cast<const uint8_t*>(h->ringK);
-      cp.ring8[1] = static_cast<const uint8_t*>(h->ringV);
-      cp.ring_scale = h->ring_scale;
-      cp.amax = h->amax;
-      cp.mem_scale = h->mem_scale;
-      cp.ring_bs[0] = h->ringBK;
-      cp.ring_bs[1] = h->ringBV;
-      cp.mem_bs[0] = h->memBK;
-      cp.mem_bs[1] = h->memBV;
-      e = h->fp4 ? launch_conv_fp4(h->D, cp, h->mapW, h->stream) : launch_conv_fp8(h->D, cp, h->mapW, h->stream);
-      h->launches += 2;
-    } else {
-      e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
-                  : launch_conv_bf16(h->D, cp, h->mapRingK, h->mapRingV, h->mapW, h->stream);
-      h->launches++;
-    }
-    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   }
   // 3. the time table of this step: absolute positions B0 + i, B0 = E - r - m (+ t_offset)
-  {
+  if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
+  if (!h->dry) {
     h->tab_t_host.clear();
     const int64_t B0 = h->E - h->Rs - h->m() + h->cfg.t_offset;
     table_axis(h, h->tab_t_host, h->tab_t_rows, 0, h->PT, B0);
@@ -448,6 +469,8 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
     if (e != cudaSuccess) return h->cuda_fail(e);
   }
   // 4. the new block becomes the current block: copy into ring slots (P + f) mod R
+  if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
+  if (h->dry) return CONVKV_OK;
   AppendParams ap{};
   ap.S = h->S;
   ap.b = frames;
@@ -490,6 +513,35 @@ static int append_impl(convkv_t* h, const void* k, const void* v, const void* co
     h->launches++;
   }
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  return CONVKV_OK;
+}
+
+// One append, all or nothing on the host side: when a launch step fails, the
+// counters go back to their values before the call.  A conv that already ran for
+// the call may have rewritten a memory position (with the new slot, made from ring
+// frames that no later step of the call touches), so until an append succeeds the
+// handle refuses attends; the next append recomputes that slot from the same frames.
+static int append_impl(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
+                       const void* const* v_sh, int frames) {
+  const int64_t P = h->P, E = h->E, Sn = h->Sn, blocks = h->blocks;
+  const int bcur = h->bcur, last_groups = h->last_groups;
+  h->steps = 0;
+  const int rc = append_steps(h, k, v, k_sh, v_sh, frames);
+  h->need_append = rc != CONVKV_OK;
+  if (rc != CONVKV_OK) {
+    h->P = P;
+    h->E = E;
+    h->Sn = Sn;
+    h->blocks = blocks;
+    h->bcur = bcur;
+    h->last_groups = last_groups;
+  }
+  return rc;
+}
+
+int convkv_debug_fail_step(convkv_t* h, int step) {
+  if (!h || step < -1) return CONVKV_ERR_INVALID_ARG;
+  h->fail_at = step;
   return CONVKV_OK;
 }
 
@@ -613,7 +665,7 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
 
 int convkv_attend(convkv_t* h, const void* q, void* out) {
   if (!h || (!h->dry && (!q || !out))) return CONVKV_ERR_INVALID_ARG;
-  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
+  if (h->blocks < 1 || h->need_append || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
   if (h->dry) return CONVKV_OK;
   return attend_impl(h, q, out, nullptr, nullptr);
 }
@@ -622,7 +674,7 @@ int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_
   if (!h || h->G < 2) return CONVKV_ERR_INVALID_ARG;
   if (!h->dry && !shards_ok(h, q_shards, reinterpret_cast<const void* const*>(out_shards)))
     return CONVKV_ERR_INVALID_ARG;
-  if (h->blocks < 1 || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
+  if (h->blocks < 1 || h->need_append || (h->Rs > 0 && !h->sink_set)) return CONVKV_ERR_BAD_ORDER;
   if (h->dry) return CONVKV_OK;
   return attend_impl(h, nullptr, nullptr, q_shards, out_shards);
 }
@@ -639,7 +691,7 @@ int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host
 
 int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
   if (!h || !q_host || !out_host) return CONVKV_ERR_INVALID_ARG;
-  if (!h->host_io || h->dry || h->blocks < 1) return CONVKV_ERR_BAD_ORDER;
+  if (!h->host_io || h->dry || h->blocks < 1 || h->need_append) return CONVKV_ERR_BAD_ORDER;
   const size_t bytes = static_cast<size_t>(h->S) * h->bcur * h->frame_elems() * 2;
   cudaError_t e = cudaMemcpyAsync(h->io_q, q_host, bytes, cudaMemcpyHostToDevice, h->stream);
   if (e != cudaSuccess) return h->cuda_fail(e);

@@ -105,6 +105,10 @@ extern "C" int convkv_quantize_e4m3_noalloc(const void* x, void* codes, float* s
                                             int heads, int head_dim, void* stream) {
   if (!x || !codes || !scales || frames < 1 || tokens < 1 || heads < 1 || head_dim < 8 || head_dim % 8)
     return CONVKV_ERR_INVALID_ARG;
+  // the kernels read x in 16-byte vectors, write codes in 8-byte vectors and scales as fp32
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
+      (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return CONVKV_ERR_INVALID_ARG;
   if (static_cast<int64_t>(frames) * heads > kMaxFrameHeads) return CONVKV_ERR_SCRATCH_LIMIT;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -112,7 +116,9 @@ extern "C" int convkv_quantize_e4m3_noalloc(const void* x, void* codes, float* s
   if (dev < 0 || dev >= kMaxDevices) return CONVKV_ERR_UNSUPPORTED;
   unsigned int* amax = nullptr;
   {
-    // first call on this device: resolve the array's device address (with this device current)
+    // first call on this device: resolve the array's device address (with this device
+    // current); the address stays valid for the life of the primary context, so a
+    // cudaDeviceReset after this call is not supported
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_amax_addr[dev]) {
       void* p = nullptr;

@@ -107,7 +107,11 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out);
  * k, v: DEVICE pointers, [num_states][frames*T][H][D] bf16; the copy is
  * asynchronous on the handle's stream, so keep them unchanged until it passes.
  * frames: 1 .. max(b1, b).  Errors: INVALID_ARG, BAD_ORDER (dry-run with
- * non-null pointers is fine), CUDA. */
+ * non-null pointers is fine), CUDA.
+ * A CUDA error leaves the counters (and so the layout) as they were before the
+ * call; a compression that already ran for the call may have rewritten one
+ * memory position, so attends return BAD_ORDER until an append succeeds, and
+ * that append recomputes the position from the same ring frames. */
 int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames);
 
 /* Attention of the current block's queries over [memory | window | current]
@@ -115,7 +119,8 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames);
  * indices reset to start at 0 (memory slot i -> r + i, window frame j -> r + m +
  * j, current frame f -> r + m + w + f, r = sink_frames), spatial indices
  * unchanged, softmax scale 1/sqrt(D), no mask inside the attended set.
- * BAD_ORDER also when sink_frames > 0 and convkv_set_sink was not called.
+ * BAD_ORDER also when sink_frames > 0 and convkv_set_sink was not called, and
+ * after an append that failed, until an append succeeds.
  * q, out: DEVICE pointers, [num_states][frames*T][H][D] bf16 with `frames` of
  * the last append.  Does not change the state (may be repeated).
  * Errors: INVALID_ARG, BAD_ORDER, CUDA. */
@@ -216,6 +221,12 @@ int64_t convkv_launch_count(const convkv_t* h);
  * stays usable.  Errors: INVALID_ARG, CUDA. */
 int convkv_selftest_wait_timeout(int* dev_status, long long budget_clocks, void* stream);
 
+/* Failure injection for tests, on the host: the `step`-th launch step (0-based,
+ * counted per call: conv, time-table upload, ring append; in dry-run handles the
+ * steps are counted but not run) of the next append reports cudaErrorLaunchFailure
+ * instead of running, once; -1 disarms.  Errors: INVALID_ARG. */
+int convkv_debug_fail_step(convkv_t* h, int step);
+
 /* cudaError_t of the last failing CUDA call made through this handle (0 if none). */
 int convkv_last_cuda_error(const convkv_t* h);
 
@@ -237,17 +248,25 @@ const char* convkv_strerror(int code);
  * [frames][heads]), asynchronously on `stream` (cudaStream_t, NULL = legacy
  * default).  The caller owns all three buffers.
  *
- * No device memory is allocated: the only scratch, one amax per (frame, head),
- * is a fixed array of CONVKV_NOALLOC_MAX_FRAME_HEADS entries (16 KiB) inside
- * the library, kept on every GPU that loads the library until the process
- * exits.  frames * heads above that limit returns CONVKV_ERR_SCRATCH_LIMIT.
- * The first call on a device resolves the array's address there (with that
- * device current); make that first call before any stream capture.  Every call
- * shares the array and it keeps the last call's contents (each call clears the
- * part it uses), so calls whose work overlaps on the GPU -- on different
- * streams, or from several host threads at once -- race and give wrong results.
- * head_dim must be a multiple of 8.  Errors: INVALID_ARG, SCRATCH_LIMIT,
- * UNSUPPORTED (device ordinal >= 128), CUDA. */
+ * Alignment: x on 16 bytes, codes on 8, scales on 4 (a misaligned pointer
+ * returns INVALID_ARG before anything runs).
+ *
+ * No device memory is allocated by a call: the only scratch, one amax per
+ * (frame, head), is a fixed array of CONVKV_NOALLOC_MAX_FRAME_HEADS entries
+ * (16 KiB) inside the library, kept on every GPU that loads the library until
+ * the process exits.  frames * heads above that limit returns
+ * CONVKV_ERR_SCRATCH_LIMIT.  The first call on a device resolves the array's
+ * address there (with that device current); with lazy module loading that
+ * first call may also make the driver load this part of the library's device
+ * code, the array included.  So make the first call once during set-up, before
+ * any stream capture and outside any window in which allocation is forbidden.
+ * The resolved address is kept for the life of the process: calling
+ * cudaDeviceReset on a device after its first call is not supported.  Every
+ * call shares the array and it keeps the last call's contents (each call
+ * clears the part it uses), so calls whose work overlaps on the GPU -- on
+ * different streams, or from several host threads at once -- race and give
+ * wrong results.  head_dim must be a multiple of 8.  Errors: INVALID_ARG,
+ * SCRATCH_LIMIT, UNSUPPORTED (device ordinal >= 128), CUDA. */
 #define CONVKV_NOALLOC_MAX_FRAME_HEADS 4096
 int convkv_quantize_e4m3_noalloc(const void* x, void* codes, float* scales, int frames, int tokens, int heads,
                                  int head_dim, void* stream);

@@ -211,3 +211,44 @@ def test_low_precision_formats_share_the_bookkeeping():
             assert np.array_equal(lays[fmt][:, [0, 1, 3]], ref[:, [0, 1, 3]])
             cur = lays[fmt][:, 0] == 2
             assert list(lays[fmt][cur, 2]) == list(range(int(cur.sum())))
+
+
+@pytest.mark.parametrize("step", [0, 1, 2])
+def test_failed_append_leaves_the_state_unchanged(step):
+    """A launch failure injected on the host at one step of an append (conv, time-table
+    upload, ring append) leaves counters and layout as they were; attends are refused
+    until an append succeeds, and the stream then continues exactly like a stream that
+    never failed."""
+    w = PRESETS["512x512"]
+    h, ref = _dry(w), _dry(w)
+    lib = ckv.library()
+    sizes = w.block_sizes()
+    # blocks 1..2 need no conv; block 3 runs the first one (step 0 is then the conv)
+    n_before = 2 if step == 0 else 4
+    for b in sizes[:n_before]:
+        h.dry_append(b)
+        ref.dry_append(b)
+    before = (h.counters(), h.layout().tolist())
+    assert lib.convkv_debug_fail_step(h._h, step) == ckv.OK
+    rc = lib.convkv_append_block(h._h, None, None, sizes[n_before])
+    assert rc == ckv.ERR_CUDA
+    assert lib.convkv_last_cuda_error(h._h) != 0
+    assert (h.counters(), h.layout().tolist()) == before
+    assert lib.convkv_attend(h._h, None, None) == ckv.ERR_BAD_ORDER
+    for b in sizes[n_before:n_before + 6]:
+        h.dry_append(b)
+        ref.dry_append(b)
+        assert h.counters() == ref.counters()
+        assert h.layout().tolist() == ref.layout().tolist()
+    assert lib.convkv_attend(h._h, None, None) == ckv.OK
+    assert lib.convkv_debug_fail_step(h._h, -2) == ckv.ERR_INVALID_ARG
+
+
+def test_noalloc_quantiser_rejects_misaligned_pointers_before_any_work():
+    """x is read in 16-byte vectors, codes written in 8-byte vectors, scales as fp32:
+    a misaligned pointer returns INVALID_ARG before any CUDA call (the addresses
+    here are never dereferenced)."""
+    lib = ckv.library()
+    good = 1 << 20
+    for x, c, s in [(good + 8, good, good), (good, good + 4, good), (good, good, good + 2)]:
+        assert lib.convkv_quantize_e4m3_noalloc(x, c, s, 1, 16, 2, 64, None) == ckv.ERR_INVALID_ARG

@@ -15,7 +15,8 @@ import pytest
 import seeded_inputs as si
 from compressed_kv_cache_convkv_b200.configs import PRESETS
 from compressed_kv_cache_convkv_b200.sp import head_range, shard_rows, split_block
-from streams import bf16_tensor_to_f64, check_attention, device_frames, device_weights, host_frames, oracle_for
+from streams import (bf16_tensor_to_f64, check_attention, device_frames, device_weights, host_frames, oracle_for,
+                     select_heads)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +31,7 @@ def torch():
     return t
 
 
-def _run_sp(torch, w, G, max_blocks=None, oracle_blocks=(), sink=0, rows=64):
+def _run_sp(torch, w, G, max_blocks=None, oracle_blocks=(), sink=0, rows=64, heads=None):
     import compressed_kv_cache_convkv_b200 as ckv
     H, T = w.heads, w.T
     weights = device_weights(w, torch)
@@ -41,15 +42,15 @@ def _run_sp(torch, w, G, max_blocks=None, oracle_blocks=(), sink=0, rows=64):
         hr = head_range(H, G, g)
         ranks.append((hr, ckv.ConvKV(cfg.with_(heads=len(hr), sp_ranks=G, sp_rank=g),
                                      weights[:, :, hr.start:hr.stop].contiguous())))
-    st = oracle_for(w) if oracle_blocks else None
+    st = oracle_for(w, heads=heads) if oracle_blocks else None
     if sink:
         rk, rv = device_frames(w, si.RK, 0, sink, torch), device_frames(w, si.RV, 0, sink, torch)
         plain.set_sink(rk, rv)
         for hr, hd in ranks:
             hd.set_sink(rk[:, :, hr.start:hr.stop].contiguous(), rv[:, :, hr.start:hr.stop].contiguous())
         if st is not None:
-            st.set_sink(si.bf16_bits_to_f64(host_frames(w, si.RK, 0, 0, sink)),
-                        si.bf16_bits_to_f64(host_frames(w, si.RV, 0, 0, sink)))
+            st.set_sink(si.bf16_bits_to_f64(host_frames(w, si.RK, 0, 0, sink, heads)),
+                        si.bf16_bits_to_f64(host_frames(w, si.RV, 0, 0, sink, heads)))
     rng = np.random.default_rng(w.seed)
     R = cfg.ring_frames
     F = 0
@@ -76,13 +77,13 @@ def _run_sp(torch, w, G, max_blocks=None, oracle_blocks=(), sink=0, rows=64):
                 assert np.array_equal(gk, pk.reshape(T, H, -1)[:, hr.start:hr.stop].reshape(gk.shape)), n
                 assert np.array_equal(gv, pv.reshape(T, H, -1)[:, hr.start:hr.stop].reshape(gv.shape)), n
         if st is not None:
-            kh, vh, qh = (host_frames(w, t, 0, F, b) for t in (si.K, si.V, si.Q))
+            kh, vh, qh = (host_frames(w, t, 0, F, b, heads) for t in (si.K, si.V, si.Q))
             st.append(si.bf16_bits_to_f64(kh), si.bf16_bits_to_f64(vh))
             if n in oracle_blocks:
                 r = np.sort(rng.choice(b * T, size=min(rows, b * T), replace=False))
                 o, _ = st.attend(si.bf16_bits_to_f64(qh), rows=r)
-                check_attention(bf16_tensor_to_f64(out[0][torch.as_tensor(r, device="cuda")]), o,
-                                what=f"{w.name} G={G} block {n}")
+                check_attention(select_heads(bf16_tensor_to_f64(out[0][torch.as_tensor(r, device="cuda")]), heads),
+                                o, what=f"{w.name} G={G} block {n}")
         F += b
     assert plain.status() == 0 and all(hd.status() == 0 for _, hd in ranks)
     plain.close()
@@ -95,7 +96,7 @@ def test_sp_tiny_two_ranks(torch):
 
 
 def test_sp_512_four_ranks(torch):
-    _run_sp(torch, PRESETS["512x512"], 4, max_blocks=6, oracle_blocks={6})
+    _run_sp(torch, PRESETS["512x512"], 4, max_blocks=6, oracle_blocks={6}, heads=(0, 9, 10, 19, 20, 29, 30, 39))
 
 
 def test_sp_720_eight_ranks_uneven_rows_with_reference(torch):

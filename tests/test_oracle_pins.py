@@ -517,3 +517,34 @@ def test_fp4_stream_window_is_quantised_current_is_exact():
         np.testing.assert_array_equal(f.v, O.fp4_dequantize(cv, bv, gv))
     o, ps = st.attend(q)
     np.testing.assert_allclose(ps, 1.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "fp4"])
+def test_low_precision_memory_slot_is_encoded_conv_of_dequantised_group(fmt):
+    """A stored memory slot in the low-precision formats is the conv of its group's five
+    frames as the cache holds them (each quantised when it joined the window, then
+    dequantised to BF16 on use), encoded once more in the cache's format: slot k covers
+    stream frames [5k, 5k+5).  Codes and scales must match that composition exactly, and
+    the slot's values must be their dequantisation (model card, --fp8_kv_cache: stored
+    in FP8, dequantised to BF16 on use)."""
+    fp4 = fmt == "fp4"
+    enc = (lambda x: (lambda c, sb, g: (c, (sb, g)))(*O.fp4_encode(x))) if fp4 else O.fp8_encode
+    deq = (lambda c, s: O.fp4_dequantize(c, s[0], s[1])) if fp4 else O.fp8_dequantize
+    hist = []
+    for st, (q, k, v), _ in _tiny_stream(W=4, C=3, blocks=12, fp8=not fp4, fp4=fp4, seed=29):
+        hist.append((k, v))
+    K = np.concatenate([h[0] for h in hist])
+    V = np.concatenate([h[1] for h in hist])
+    assert st.S > st.m == 3          # the FIFO has dropped slots
+    for age, slot in enumerate(st.memory):
+        f0 = 5 * slot.index
+        for kv, (X, got_val, got_codes) in enumerate(((K, slot.k, slot.codes[:2]), (V, slot.v, slot.codes[2:]))):
+            group = np.stack([deq(*enc(X[f])) for f in range(f0, f0 + 5)])
+            code, scales = enc(O.conv_compress(group, st.w[kv]))
+            np.testing.assert_array_equal(got_codes[0], code)
+            if fp4:
+                np.testing.assert_array_equal(got_codes[1][0], scales[0])
+                np.testing.assert_array_equal(got_codes[1][1], scales[1])
+            else:
+                np.testing.assert_array_equal(got_codes[1], scales)
+            np.testing.assert_array_equal(got_val, deq(code, scales))
