@@ -496,12 +496,17 @@ def main(argv=None):
                     help="memory compression: the learned 1D conv (default) or the 5-frame mean")
     ap.add_argument("--sink-frames", type=int, default=0,
                     help="reference-image frames attended first by every block (default none)")
+    ap.add_argument("--states", type=int, default=0,
+                    help="layer states per call (default: the workload's own; fewer make a small profiling case)")
     args = ap.parse_args(argv)
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         # one process per GPU: start the ranks here and pass their output through
         return subprocess.call(rank_launch_command(args.gpus, argv))
+    from dataclasses import replace
     from compressed_kv_cache_convkv_b200.configs import PRESETS
     w = PRESETS[args.workload]
+    if args.states:
+        w = replace(w, num_states=args.states)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -69,6 +69,12 @@ struct convkv {
   size_t arena_bytes = 0;
   void *ringK = nullptr, *ringV = nullptr, *memK = nullptr, *memV = nullptr, *weights = nullptr;
   void* ringKr = nullptr;           // bf16 format: K of the ring rotated at its stream position
+  // rotated copies of the keys whose RoPE positions move with every eviction: the
+  // memory slots (bf16 format) and the reference frames (both formats), refreshed by
+  // the append whenever the time table's base moves
+  void *memKr = nullptr, *sinkKr = nullptr;
+  int64_t rot_B0 = INT64_MIN;       // table base the rotated copies were made with
+  bool rot_sink_stale = false;      // reference frames given since the last rotation
   std::vector<float4> tab_t_host;   // time table rows of the current step (host copy)
   // fp8 format: ringK/ringV/memK/memV hold e4m3 codes; scales per (state, K|V, slot, head)
   float *ring_scale = nullptr, *mem_scale = nullptr;
@@ -82,6 +88,9 @@ struct convkv {
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
   CUtensorMap mapRingK{}, mapRingV{}, mapRingKr{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
       mapSinkV{};
+  // e4m3 / NVFP4: code tiles of the ring and memory, staged by the attention kernel
+  CUtensorMap mapRingCK{}, mapRingCV{}, mapMemCK{}, mapMemCV{};
+  CUtensorMap mapMemKr{}, mapSinkKr{};
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
   int last_cuda = 0;
@@ -125,6 +134,25 @@ int encode_4d(CUtensorMap* map, void* ptr, int D, int H, int64_t rows, int S) {
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVKV_OK : CONVKV_ERR_CUDA;
+}
+
+// Codes of the e4m3 / NVFP4 cache [S][rows][H][cb] bytes: one box is 128 rows of one
+// head's cb code bytes, written with the cb-byte swizzle (cb = 128, 64 or 32).
+int encode_codes(CUtensorMap* map, void* ptr, int cb, int H, int64_t rows, int S) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return CONVKV_ERR_CUDA;
+  const CUtensorMapSwizzle sw = cb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                          : (cb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  if (cb != 128 && cb != 64 && cb != 32) return CONVKV_ERR_UNSUPPORTED;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(cb), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(S)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(cb), static_cast<cuuint64_t>(H) * cb,
+                           static_cast<cuuint64_t>(rows) * H * cb};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(cb), 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? CONVKV_OK : CONVKV_ERR_CUDA;
 }
 
@@ -293,6 +321,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t io_b = h->host_io ? static_cast<size_t>(h->S) * h->Bmax * fe * 2 : 0;
   const size_t sink_b = static_cast<size_t>(h->S) * h->Rs * fe * 2;
   const size_t rkr_b = h->prerot ? ring_b : 0;
+  const size_t mkr_b = h->prerot ? mem_b : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -304,7 +333,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
                o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
                o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b),
                o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b),
-               o_rkr = take(rkr_b);
+               o_rkr = take(rkr_b), o_mkr = take(mkr_b), o_skr = take(sink_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -334,10 +363,14 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->memBK = reinterpret_cast<uint8_t*>(a + o_mbk);
     h->memBV = reinterpret_cast<uint8_t*>(a + o_mbv);
   }
-  if (h->prerot) h->ringKr = a + o_rkr;
+  if (h->prerot) {
+    h->ringKr = a + o_rkr;
+    h->memKr = a + o_mkr;
+  }
   if (h->Rs) {
     h->sinkK = a + o_rfk;
     h->sinkV = a + o_rfv;
+    h->sinkKr = a + o_skr;
   }
   if (h->host_io) {
     h->io_q = a + o_q;
@@ -357,17 +390,24 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   }
   if ((e = cudaStreamSynchronize(h->stream)) != cudaSuccess) goto fail_cuda;
   if (h->fp8) {
-    // e4m3 ring and memory are read by the kernels' own dequantising loads; TMA only
-    // serves the bf16 staging of the current block
+    // the attention stages the ring's and memory's code tiles with TMA and expands
+    // them itself; the bf16 staging of the current block is loaded as is
+    const int cb = h->fp4 ? h->D / 2 : h->D;
     rc = encode_4d(&h->mapStageK, h->stageK, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapStageV, h->stageV, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
+    if (!rc) rc = encode_codes(&h->mapRingCK, h->ringK, cb, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+    if (!rc) rc = encode_codes(&h->mapRingCV, h->ringV, cb, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
+    if (!rc) rc = encode_codes(&h->mapMemCK, h->memK, cb, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+    if (!rc) rc = encode_codes(&h->mapMemCV, h->memV, cb, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
   } else {
     rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapRingKr, h->ringKr, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapRingV, h->ringV, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapMemK, h->memK, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapMemV, h->memV, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+    if (!rc) rc = encode_4d(&h->mapMemKr, h->memKr, h->D, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
   }
+  if (!rc && h->Rs) rc = encode_4d(&h->mapSinkKr, h->sinkKr, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && h->Rs) rc = encode_4d(&h->mapSinkK, h->sinkK, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && h->Rs) rc = encode_4d(&h->mapSinkV, h->sinkV, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && w_b) rc = encode_weights(&h->mapW, h->weights, h->D, h->H, h->S);
@@ -399,6 +439,34 @@ size_t convkv_state_bytes(const convkv_t* h) { return h ? h->arena_bytes : 0; }
 int64_t convkv_launch_count(const convkv_t* h) { return h ? h->launches : 0; }
 
 int convkv_last_cuda_error(const convkv_t* h) { return h ? h->last_cuda : 0; }
+
+// Rotated copies of the reference frames and memory slots for the time table of the
+// step (base B0): RoPE Reset moves their positions with every eviction, so they are
+// rotated again whenever B0 moves, or the reference frames were given anew.
+static int rotate_moving_keys(convkv_t* h, int64_t B0) {
+  RotateParams rp{};
+  rp.S = h->S;
+  rp.r = h->Rs;
+  rp.m = h->prerot ? h->m() : 0;
+  rp.C = h->C;
+  rp.pos0 = static_cast<int>((h->Sn - h->m()) % h->C);
+  rp.frame_vecs = h->frame_elems() / 8;
+  rp.H = h->H;
+  rp.grid_w = h->gw;
+  rp.sink_src = h->sinkK;
+  rp.sink_dst = h->sinkKr;
+  rp.mem_src = h->memK;
+  rp.mem_dst = h->memKr;
+  rp.tables = h->tables;
+  rp.tab_t_rows = h->tab_t_rows;
+  rp.tab_h_rows = h->gh;
+  const int e = launch_rotate_keys(h->D, rp, h->stream);
+  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  if (rp.r + rp.m > 0) h->launches++;
+  h->rot_B0 = B0;
+  h->rot_sink_stale = false;
+  return CONVKV_OK;
+}
 
 // The steps of one append.  Advances the counters first (the launches read the new
 // ones); append_impl restores them when a step fails.
@@ -448,7 +516,8 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
         cp.ring_bs[1] = h->ringBV;
         cp.mem_bs[0] = h->memBK;
         cp.mem_bs[1] = h->memBV;
-        e = h->fp4 ? launch_conv_fp4(h->D, cp, h->mapW, h->stream) : launch_conv_fp8(h->D, cp, h->mapW, h->stream);
+        e = h->fp4 ? launch_conv_fp4(h->D, cp, h->mapRingCK, h->mapRingCV, h->mapW, h->stream)
+                   : launch_conv_fp8(h->D, cp, h->mapRingCK, h->mapRingCV, h->mapW, h->stream);
         h->launches += 2;
       } else {
         e = h->mean ? launch_mean_bf16(h->D, cp, h->ringK, h->ringV, h->stream)
@@ -459,14 +528,24 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
     }
   }
   // 3. the time table of this step: absolute positions B0 + i, B0 = E - r - m (+ t_offset)
+  const int64_t B0 = h->E - h->Rs - h->m() + h->cfg.t_offset;
   if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
   if (!h->dry) {
     h->tab_t_host.clear();
-    const int64_t B0 = h->E - h->Rs - h->m() + h->cfg.t_offset;
     table_axis(h, h->tab_t_host, h->tab_t_rows, 0, h->PT, B0);
     cudaError_t e = cudaMemcpyAsync(h->tables, h->tab_t_host.data(), h->tab_t_host.size() * sizeof(float4),
                                     cudaMemcpyHostToDevice, h->stream);
     if (e != cudaSuccess) return h->cuda_fail(e);
+  }
+  // 3b. memory slots (bf16 format) and reference frames rotated for this table
+  if ((h->prerot || h->Rs) && (B0 != h->rot_B0 || h->rot_sink_stale)) {
+    if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
+    if (!h->dry) {
+      if (int rc = rotate_moving_keys(h, B0)) return rc;
+    } else {
+      h->rot_B0 = B0;
+      h->rot_sink_stale = false;
+    }
   }
   // 4. the new block becomes the current block: copy into ring slots (P + f) mod R
   if (cudaError_t g = h->step_gate()) return h->cuda_fail(g);
@@ -479,8 +558,10 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
   ap.frame_elems = h->frame_elems();
   ap.H = h->H;
   ap.D = h->D;
-  if (h->prerot) {
-    ap.ringKr = h->ringKr;
+  if (h->prerot || h->fp8) {
+    // bf16: K is also written rotated into ringKr; e4m3 / NVFP4: the current block's
+    // bf16 staging copy of K is written rotated
+    ap.ringKr = h->prerot ? h->ringKr : nullptr;
     ap.tables = h->tables;
     ap.tab_t_rows = h->tab_t_rows;
     ap.tab_h_rows = h->gh;
@@ -573,6 +654,16 @@ int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
     if (e == cudaSuccess) e = cudaMemcpyAsync(h->sinkV, v, bytes, cudaMemcpyDeviceToDevice, h->stream);
     if (e != cudaSuccess) return h->cuda_fail(e);
   }
+  h->rot_sink_stale = true;
+  // after the first append the step's table exists: rotate the new frames now (before
+  // that, the first append does it)
+  if (h->blocks > 0 && !h->need_append) {
+    if (!h->dry) {
+      if (int rc = rotate_moving_keys(h, h->rot_B0)) return rc;
+    } else {
+      h->rot_sink_stale = false;
+    }
+  }
   h->sink_set = true;
   return CONVKV_OK;
 }
@@ -594,7 +685,9 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     s.t0 = t0;
     s.tile0 = tiles;
     s.fp8 = (h->fp8 && buf < 2) ? 1 : 0;
-    s.prerot = (h->prerot && buf == 0) ? 1 : 0;
+    // keys stored rotated: the bf16 ring's K (window and current) and the bf16
+    // staging of the current block in the e4m3 / NVFP4 formats
+    s.prerot = ((h->prerot && buf <= 1) || (h->fp8 && buf == 2) || buf == 3) ? 1 : 0;
     s.slot0 = frame0;
     tiles += (s.nrows + 127) / 128;
   };
@@ -616,6 +709,9 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     if (h->fp8) add(2, 0, b, r + m + w);
   }
   ap.ntiles = tiles;
+  ap.all_prerot = 1;
+  for (int i = 0; i < ap.nseg; ++i)
+    if (!ap.seg[i].prerot || ap.seg[i].fp8) ap.all_prerot = 0;
   ap.tab_t_rows = h->tab_t_rows;
   ap.tab_h_rows = h->gh;
   ap.tab_w_rows = h->gw;
@@ -649,13 +745,14 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     ap.ring_bs[1] = h->ringBV;
     ap.mem_bs[0] = h->memBK;
     ap.mem_bs[1] = h->memBV;
-    km[0] = km[1] = km[2] = h->mapStageK;  // only staging and reference maps are used by TMA
-    vm[0] = vm[1] = vm[2] = h->mapStageV;
+    // ring and memory: code tiles (expanded by the kernel); staging: bf16 tiles
+    km[0] = h->mapRingCK; km[1] = h->mapMemCK; km[2] = h->mapStageK;
+    vm[0] = h->mapRingCV; vm[1] = h->mapMemCV; vm[2] = h->mapStageV;
   } else {
-    km[0] = h->mapRingKr; km[1] = h->mapMemK; km[2] = h->mapRingK;
+    km[0] = h->mapRingKr; km[1] = h->mapMemKr; km[2] = h->mapRingK;
     vm[0] = h->mapRingV; vm[1] = h->mapMemV; vm[2] = h->mapRingV;
   }
-  km[3] = r ? h->mapSinkK : km[2];
+  km[3] = r ? h->mapSinkKr : km[2];
   vm[3] = r ? h->mapSinkV : vm[2];
   int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp4 ? 2 : (h->fp8 ? 1 : 0), h->stream);
   h->launches++;

@@ -78,6 +78,7 @@ struct AttnParams {
   const uint8_t* ring_bs[2];
   const uint8_t* mem_bs[2];
   int R, C;
+  int all_prerot;         // every key segment is stored rotated: no RoPE work on K tiles
   int* status;
   // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
   // and written to the G ranks' shards (peer memory on a multi-GPU node)
@@ -132,15 +133,35 @@ struct AppendParams {
   int tab_t_rows, tab_h_rows, t_row0, grid_w;
 };
 
+// Rotation of the cached keys that are not stored rotated at append: the r reference
+// frames and the m stored memory slots, whose RoPE positions move with every eviction
+// (RoPE Reset).  Frame i < r is reference frame i (table row i); frame i >= r is the
+// memory position (pos0 + i - r) mod C (table row i).  src/dst: [S][frames*T][H][D] bf16.
+struct RotateParams {
+  int S, r, m, C, pos0;
+  int64_t frame_vecs;          // 16-byte vectors per frame (T * H * D / 8)
+  int H, grid_w;
+  const void* sink_src;
+  void* sink_dst;
+  const void* mem_src;
+  void* mem_dst;
+  const float4* tables;
+  int tab_t_rows, tab_h_rows;
+};
+
 // Kernel launchers (return cudaError_t of the launch).
+int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s);
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
                        cudaStream_t s);
 int launch_permute_weights(const void* src, void* dst, int S, int H, int D, cudaStream_t s);
 int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const CUtensorMap& ringV,
                      const CUtensorMap& wmap, cudaStream_t s);
 int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s);
-int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
-int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s);
+// codesK, codesV: TMA maps of the ring's code tiles (one head's 128 rows of codes)
+int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
+                    const CUtensorMap& wmap, cudaStream_t s);
+int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
+                    const CUtensorMap& wmap, cudaStream_t s);
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s);
 // k, v: tensor maps of buffers 0..3 (ring, memory, staging, reference frames)
 // fmt: 0 bf16, 1 e4m3, 2 NVFP4 (ring and memory segments)

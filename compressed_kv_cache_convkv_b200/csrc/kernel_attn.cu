@@ -20,8 +20,14 @@
 //               thread per query row; online softmax in fp32 registers with a
 //               lazily rescaled running max (the O rescale is only done when
 //               the max grows by more than 2^8); P written back over S as bf16
-//   warps 12-15 RoPE of each landed K tile, in place in shared memory
-//               (cos/sin tables read through the read-only data cache)
+//   warps 12-15 RoPE of each landed K tile that is not stored rotated, in place
+//               in shared memory (cos/sin tables read through the read-only data
+//               cache); with every key stored rotated (bf16 cache) they are idle and
+//               the MMA issuer takes K tiles straight from TMA
+//   warps 2-3   (e4m3 / NVFP4 cache only) dequantisation of V tiles
+// In the e4m3 / NVFP4 formats the producer stages each ring or memory tile's codes
+// with TMA in the upper half of its stage buffer; the RoPE warpgroup (K) and warps
+// 2-3 (V) turn them into bf16 rows in place.
 // TMEM: S_0 | S_1 | O_0 | O_1 = 128 | 128 | D | D columns of 512.
 // Every barrier wait is bounded; on expiry the CTA raises an abort flag, skips
 // the remaining work, drains its outstanding copies and MMAs, frees TMEM and
@@ -109,64 +115,105 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi
   hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
 
-// Dequantise one e4m3 row (D codes at src, scale s) to bf16 value x*s, rotate it
-// (ROTATE) and store it as row `row` of a 128-byte-swizzled bf16 tile.  Rows
-// past the segment store zeros (valid == false) so masked columns stay finite.
-template <int D, bool ROTATE>
-__device__ __forceinline__ void dequant_row(uint8_t* tile, int row, const uint8_t* src, float sc, bool valid,
-                                            const RopeRow& rr) {
-  using C = AttnCfg<D>;
-  uint8_t* rowp = tile + row * 128;
-  const int sw = row & 7;
-  uint4 raw[D / 16];
+// Code tiles of the e4m3 / NVFP4 cache, staged by TMA: 128 rows of CB bytes (the
+// codes of one head's row), written with the CB-byte swizzle into the upper half of
+// a stage buffer, and turned into the bf16 tile in place.
+template <int D, int QF>
+struct CodeCfg {
+  static constexpr int CB = QF == 2 ? D / 2 : D;   // code bytes per row
+  static constexpr int BYTES = 128 * CB;
+  static constexpr int OFF = AttnCfg<D>::TILE / 2;  // 1024-aligned
+  static constexpr int NCH = CB / 16;               // 16-byte chunks per row
+  static constexpr uint32_t MASK = CB == 128 ? 7u : (CB == 64 ? 3u : 1u);
+  // e4m3 at D = 128: a row's codes lie inside the bytes of its own bf16 output (the
+  // second 64-channel box), so each thread converts its rows with no barrier.
+  // Otherwise the codes of one row sit under other rows' output: the converting
+  // threads read all their codes, meet at a barrier, then write.
+  static constexpr bool SELF = QF == 1 && D == 128;
+  static constexpr int SCALE_WORDS = QF == 2 ? (D / 16 + 3) / 4 : 0;  // NVFP4 block-scale words per row
+};
+
+// 16-byte chunk c of row r of a staged code tile (the TMA swizzle XORs address bits
+// [4, 7) with bits [7, 10), masked to the swizzle span).
+template <int CB, uint32_t MASK>
+__device__ __forceinline__ uint4 code_chunk(const uint8_t* codes, int r, int c) {
+  const uint32_t logical = static_cast<uint32_t>(r * CB + c * 16);
+  const uint32_t phys = logical ^ (((logical >> 7) & MASK) << 4);
+  return *reinterpret_cast<const uint4*>(codes + phys);
+}
+
+// The codes of one row (zeros for rows past the segment) and, for NVFP4, its block
+// scales from global memory.
+template <int D, int QF>
+struct RowCodes {
+  uint4 raw[CodeCfg<D, QF>::NCH];
+  uint32_t bs[CodeCfg<D, QF>::SCALE_WORDS > 0 ? CodeCfg<D, QF>::SCALE_WORDS : 1];
+
+  __device__ __forceinline__ void load(const uint8_t* codes, int r, bool valid, const uint8_t* bs_row) {
+    using CC = CodeCfg<D, QF>;
 #pragma unroll
-  for (int k = 0; k < D / 16; ++k) raw[k] = valid ? __ldg(reinterpret_cast<const uint4*>(src) + k) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < CC::NCH; ++k)
+      raw[k] = valid ? code_chunk<CC::CB, CC::MASK>(codes, r, k) : make_uint4(0, 0, 0, 0);
+    if constexpr (QF == 2) {
+      if constexpr (D / 16 >= 4) {
 #pragma unroll
-  for (int k = 0; k < D / 16; ++k) {
-    const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        for (int k = 0; k < CC::SCALE_WORDS; ++k) bs[k] = valid ? __ldg(reinterpret_cast<const uint32_t*>(bs_row) + k) : 0u;
+      } else {
+        // D / 16 block scales per row, fewer than four: byte loads
+        uint32_t w = 0;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {  // two bf16 chunks of 8 channels
-      const int c = 2 * k + u;
+        for (int k = 0; k < D / 16; ++k) w |= valid ? static_cast<uint32_t>(__ldg(bs_row + k)) << (8 * k) : 0u;
+        bs[0] = w;
+      }
+    }
+  }
+
+  // Dequantise to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale = fp32(s_b * g)),
+  // rotate (ROTATE) and store as row `row` of the 128-byte-swizzled bf16 tile.
+  template <bool ROTATE>
+  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr) const {
+    using C = AttnCfg<D>;
+    uint8_t* rowp = tile + row * 128;
+    const int sw = row & 7;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
       uint32_t o[4];
+      if constexpr (QF == 2) {
+        const uint4 r4 = raw[c >> 2];
+        const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
+        const int b = c >> 1;  // block of 16 channels
+        const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), sc);
+        fp4::decode8(word, e_b, o);
+      } else {
+        const uint4 r4 = raw[c >> 1];
+        const uint32_t w0 = (c & 1) ? r4.z : r4.x, w1 = (c & 1) ? r4.w : r4.y;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t word = w[2 * u + (q >> 1)];
-        float a, b;
-        e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
-        o[q] = pack_bf16x2(a * sc, b * sc);  // dequantised to bf16 on use
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t word = q < 2 ? w0 : w1;
+          float a, b;
+          e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
+          o[q] = pack_bf16x2(a * sc, b * sc);
+        }
       }
       if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
       *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-}
+};
 
-// NVFP4 row: D/2 code bytes (e2m1 pairs) and D/16 e4m3 block scales at the row's
-// offsets, fp32 scale g; bf16 value code * fp32(s_b * g), rotated (ROTATE) and
-// stored swizzled like dequant_row.  Rows past the segment store zeros.
-template <int D, bool ROTATE>
-__device__ __forceinline__ void dequant_row_fp4(uint8_t* tile, int row, const uint8_t* codes, const uint8_t* bs,
-                                                float g, bool valid, const RopeRow& rr) {
-  using C = AttnCfg<D>;
-  uint8_t* rowp = tile + row * 128;
-  const int sw = row & 7;
-  uint4 raw[D / 32];
-  uint32_t sraw[D / 64];
-#pragma unroll
-  for (int k = 0; k < D / 32; ++k) raw[k] = valid ? __ldg(reinterpret_cast<const uint4*>(codes) + k) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int k = 0; k < D / 64; ++k) sraw[k] = valid ? __ldg(reinterpret_cast<const uint32_t*>(bs) + k) : 0u;
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 r4 = raw[c >> 2];
-    const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
-    const int b = c >> 1;  // block of 16 channels
-    const float e_b = __fmul_rn(fp4::e4m3_to_f32(sraw[b >> 2] >> (8 * (b & 3))), g);
-    uint32_t o[4];
-    fp4::decode8(word, e_b, o);
-    if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
-    *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
+// AND of `v` over the `nthreads` threads (whole warps) that meet at named barrier `id`.
+__device__ __forceinline__ bool bar_all(int id, int nthreads, bool v) {
+  uint32_t r;
+  __syncwarp();  // the barrier is warp-aligned: reconverge first
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // QF: storage of the ring and memory segments, 0 bf16, 1 e4m3, 2 NVFP4
@@ -266,7 +313,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int ks = j % C::KST;
         if (j >= C::KST && !mbar_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
         if (FP8 && sg.fp8) {
-          mbar_arrive(&k_full[ks]);  // stage free: the RoPE warpgroup loads and dequantises it
+          // the tile's codes into the upper half of the stage; the RoPE warpgroup expands them
+          mbar_expect_tx(&k_full[ks], CodeCfg<D, QF>::BYTES);
+          tma_load_4d(sK + ks * C::TILE + CodeCfg<D, QF>::OFF, kmap(sg.buf), &k_full[ks], 0, head, row, state);
         } else {
           mbar_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
@@ -277,7 +326,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int vs = j % C::VST;
         if (j >= C::VST && !mbar_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, abort_flag)) break;
         if (FP8 && sg.fp8) {
-          mbar_arrive(&v_full[vs]);  // stage free: warps 2-3 load and dequantise it
+          // the tile's codes into the upper half of the stage; warps 2-3 expand them
+          mbar_expect_tx(&v_full[vs], CodeCfg<D, QF>::BYTES);
+          tma_load_4d(sV + vs * C::TILE + CodeCfg<D, QF>::OFF, vmap(sg.buf), &v_full[vs], 0, head, row, state);
         } else {
           mbar_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll
@@ -324,9 +375,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      // K tiles that are all stored rotated go from TMA straight to the tensor cores
+      uint64_t* kr = p.all_prerot ? k_full : k_ready;
       do {
         if (!mbar_wait(q_ready, 0, abort_flag)) break;
-        if (!mbar_wait(&k_ready[0], 0, abort_flag)) break;
+        if (!mbar_wait(&kr[0], 0, abort_flag)) break;
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(&s_full[0]);
@@ -346,7 +399,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             if (i == 1) tc_commit(&v_empty[vs]);
             if (has_next) {
               if (i == 0) {
-                if (!mbar_wait(&k_ready[ksn], ((j + 1) / C::KST) & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&kr[ksn], ((j + 1) / C::KST) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
               }
               issue_s(i, ksn);
@@ -367,40 +420,55 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
   } else if (FP8 && (warp == 2 || warp == 3)) {
       // ---------------------------------------------------------- V dequantisation
+      using CC = CodeCfg<D, QF>;
       const int r0 = (warp - 2) * 32 + lane;  // rows r0 and r0 + 64 of each V tile
       TileCursor cur;
       for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
         const int vs = j % C::VST;
-        if (!mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag)) break;
+        bool ok = mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag);
         const KeySeg& sg = seg[cur.s];
-        if (sg.fp8) {
-          const uint8_t* base = p.ring8[1];
-          const float* scl = p.ring_scale;
-          int nsl = p.R;
-          if (sg.buf == 1) {
-            base = p.mem8[1];
-            scl = p.mem_scale;
-            nsl = p.C;
-          }
+        uint8_t* tile = sV + vs * C::TILE;
+        const uint8_t* codes = tile + CC::OFF;
+        const bool mem = sg.buf == 1;
+        const int nsl = mem ? p.C : p.R;
+        const float* scl = mem ? p.mem_scale : p.ring_scale;
+        const uint8_t* bsb = mem ? p.mem_bs[1] : p.ring_bs[1];
+        RowCodes<D, QF> rc[2];
+        float sc[2];
+        auto load = [&](int u) {
+          const int r = r0 + 64 * u;
+          const int lr = cur.jt * C::BN + r;
+          const bool valid = lr < sg.nrows;
+          const int f = valid ? lr / p.T : 0;
+          const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
+          sc[u] = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
+          rc[u].load(codes, r, valid, bsb + (grow * p.H + head) * (D / 16));
+        };
+        if constexpr (CC::SELF) {
+          if (!ok) break;
+          if (sg.fp8) {
+            // each row's codes sit under its own output: convert row by row
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int r = r0 + 64 * u;
-            const int lr = cur.jt * C::BN + r;
-            const bool valid = lr < sg.nrows;
-            const int f = valid ? lr / p.T : 0;
-            const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
-            const float sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-            if constexpr (QF == 2) {
-              const uint8_t* bsb = sg.buf == 1 ? p.mem_bs[1] : p.ring_bs[1];
-              dequant_row_fp4<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * (D / 2),
-                                        bsb + (grow * p.H + head) * (D / 16), sc, valid,
-                                        RopeRow{nullptr, nullptr, nullptr});
-            } else {
-              dequant_row<D, false>(sV + vs * C::TILE, r, base + (grow * p.H + head) * D, sc, valid,
-                                    RopeRow{nullptr, nullptr, nullptr});
+            for (int u = 0; u < 2; ++u) {
+              load(u);
+              rc[u].template store<false>(tile, r0 + 64 * u, sc[u], RopeRow{nullptr, nullptr, nullptr});
             }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
+        } else {
+          if (ok && sg.fp8) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) load(u);
+          }
+          // every code of the tile is in registers before any row is written (and a
+          // timeout anywhere in the group stops all of it together)
+          if (!bar_all(2, 64, ok)) break;
+          if (sg.fp8) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              rc[u].template store<false>(tile, r0 + 64 * u, sc[u], RopeRow{nullptr, nullptr, nullptr});
+            fence_proxy_async_smem();
+          }
         }
         mbar_arrive(&v_ready[vs]);
       }
@@ -544,11 +612,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   } else {
     regs_dec<C::REG_ROPE>();
     // ------------------------------------------------------------ K RoPE
+    using CC = CodeCfg<D, QF>;
+    // staged codes that lie under other rows' output: the warpgroup meets at a barrier
+    // on every tile (uniformly, so a timeout anywhere stops all of it together)
+    constexpr bool VOTE = FP8 && !CC::SELF;
     const int r = threadIdx.x - 384;
     TileCursor cur;
-    for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
+    for (int j = 0; j < (p.all_prerot ? 0 : p.ntiles); ++j, cur.next(seg)) {
       const int ks = j % C::KST;
-      if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
+      bool ok = mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag);
       const KeySeg& sg = seg[cur.s];
       const int lr = cur.jt * C::BN + r;
       const bool valid = lr < sg.nrows;
@@ -558,26 +630,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int y = s / p.grid_w;
       const int x = s - y * p.grid_w;
       const RopeRow rr{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW};
+      uint8_t* tile = sK + ks * C::TILE;
       if (FP8 && sg.fp8) {
-        const uint8_t* base = p.ring8[0];
-        const float* scl = p.ring_scale;
-        int nsl = p.R;
-        if (sg.buf == 1) {
-          base = p.mem8[0];
-          scl = p.mem_scale;
-          nsl = p.C;
-        }
+        // e4m3 / NVFP4 codes staged by TMA: dequantise, rotate, write the bf16 row
+        const bool mem = sg.buf == 1;
+        const int nsl = mem ? p.C : p.R;
+        const float* scl = mem ? p.mem_scale : p.ring_scale;
         const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
         const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-        if constexpr (QF == 2) {
-          const uint8_t* bsb = sg.buf == 1 ? p.mem_bs[0] : p.ring_bs[0];
-          dequant_row_fp4<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * (D / 2),
-                                   bsb + (grow * p.H + head) * (D / 16), sc, valid, rr);
-        } else {
-          dequant_row<D, true>(sK + ks * C::TILE, r, base + (grow * p.H + head) * D, sc, valid, rr);
-        }
-      } else if (valid && !sg.prerot) {
-        rope_row<D, false>(sK + ks * C::TILE, r, rr, 1.0f);
+        RowCodes<D, QF> rc;
+        if (ok) rc.load(tile + CC::OFF, r, valid, (mem ? p.mem_bs[0] : p.ring_bs[0]) + (grow * p.H + head) * (D / 16));
+        if constexpr (VOTE) ok = bar_all(1, 128, ok);
+        if (!ok) break;
+        rc.template store<true>(tile, r, sc, rr);
+      } else {
+        if constexpr (VOTE) ok = bar_all(1, 128, ok);
+        if (!ok) break;
+        if (valid && !sg.prerot) rope_row<D, false>(tile, r, rr, 1.0f);
       }
       fence_proxy_async_smem();
       mbar_arrive(&k_ready[ks]);

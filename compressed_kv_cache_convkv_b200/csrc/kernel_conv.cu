@@ -8,11 +8,13 @@
 // i.e. one GEMM per (group, K|V, head): [T x 5D] . [5D x D], accumulated in
 // fp32 in tensor memory and rounded to bf16 into the memory slot.
 //
-// One CTA computes a 128-token x D tile: five k-blocks (one per evicted frame),
+// One work unit is a 128-token x D tile: five k-blocks (one per evicted frame),
 // each a TMA box of the frame's rows for this head (ring slots may wrap; each
 // k-block is its own load, so wrap costs nothing) and the matching D x D
 // weight block.  Warp 0 issues TMA, warp 1 issues tcgen05.mma (M=128, N=D,
-// K=16 steps) and owns the TMEM accumulator, warps 2-5 drain it.
+// K=16 steps) and owns the TMEM accumulators, warps 2-5 drain them.  The bf16
+// kernel is persistent (one CTA per SM walking the units); the low-precision one
+// keeps one unit per CTA.
 #include "convkv_internal.h"
 #include "sm100.cuh"
 #include "nvfp4.cuh"
@@ -35,41 +37,62 @@ struct ConvCfg {
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
 };
 
+// One work unit = (128-token tile mt, head, K|V, state, group); units are numbered
+// with mt fastest, so consecutive units of a CTA share the head's weights in L2.
+struct ConvUnit {
+  int mt, head, kv, state, g;
+};
+__device__ __forceinline__ ConvUnit conv_unit(int u, int MT, const ConvParams& p) {
+  ConvUnit c;
+  c.mt = u % MT;
+  int rest = u / MT;
+  c.head = rest % p.H;
+  rest /= p.H;
+  c.kv = rest & 1;
+  const int sg = rest >> 1;
+  c.state = sg % p.S;
+  c.g = sg / p.S;
+  return c;
+}
+
+// Persistent: each CTA walks units blockIdx.x, blockIdx.x + gridDim.x, ...  The
+// producer streams the units' k-blocks through a 3-stage ring without pausing
+// between units; the accumulator is double-buffered in TMEM, so the epilogue of one
+// unit overlaps the loads and MMAs of the next.
 template <int D>
 __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
     conv_bf16_kernel(const __grid_constant__ CUtensorMap tmRingK, const __grid_constant__ CUtensorMap tmRingV,
-                     const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
+                     const __grid_constant__ CUtensorMap tmW, const ConvParams p, int MT, int units) {
   using C = ConvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::STAGES * C::STAGE_BYTES);
-  uint64_t* full = bars;                 // [STAGES]
-  uint64_t* empty = bars + C::STAGES;    // [STAGES]
-  uint64_t* acc_full = bars + 2 * C::STAGES;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* full = bars;                    // [STAGES]
+  uint64_t* empty = bars + C::STAGES;       // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, head = blockIdx.y;
-  const int kv = blockIdx.z & 1;
-  const int sg = blockIdx.z >> 1;
-  const int state = sg % p.S;
-  const int g = sg / p.S;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -79,24 +102,33 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const CUtensorMap* ring = kv ? &tmRingV : &tmRingK;
-      tma_prefetch_desc(ring);
+      tma_prefetch_desc(&tmRingK);
+      tma_prefetch_desc(&tmRingV);
       tma_prefetch_desc(&tmW);
       int issued[C::STAGES] = {};
-      for (int j = 0; j < kEvict; ++j) {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(&empty[st], ((j / C::STAGES) - 1) & 1, abort_flag)) break;
-        uint8_t* a = stages + st * C::STAGE_BYTES;
-        uint8_t* b = a + C::A_BYTES;
-        mbar_expect_tx(&full[st], C::STAGE_BYTES);
-        const int row = p.grp[g].ring_slot[j] * p.T + mt * C::BM;
-        const int wrow = ((kv * p.H + head) * kEvict + j) * D;
+      int it = 0;  // k-blocks issued by this CTA
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const ConvUnit cu = conv_unit(u, MT, p);
+        const CUtensorMap* ring = cu.kv ? &tmRingV : &tmRingK;
+        for (int j = 0; j < kEvict; ++j, ++it) {
+          const int st = it % C::STAGES;
+          if (it >= C::STAGES && !mbar_wait(&empty[st], ((it / C::STAGES) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a = stages + st * C::STAGE_BYTES;
+          uint8_t* b = a + C::A_BYTES;
+          mbar_expect_tx(&full[st], C::STAGE_BYTES);
+          const int row = p.grp[cu.g].ring_slot[j] * p.T + cu.mt * C::BM;
+          const int wrow = ((cu.kv * p.H + cu.head) * kEvict + j) * D;
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx) {
-          tma_load_4d(a + bx * (C::BM * 128), ring, &full[st], bx * 64, head, row, state);
-          tma_load_3d(b + bx * (D * 128), &tmW, &full[st], bx * 64, wrow, state);
+          for (int bx = 0; bx < C::NBOX; ++bx) {
+            tma_load_4d(a + bx * (C::BM * 128), ring, &full[st], bx * 64, cu.head, row, cu.state);
+            tma_load_3d(b + bx * (D * 128), &tmW, &full[st], bx * 64, wrow, cu.state);
+          }
+          ++issued[st];
         }
-        ++issued[st];
       }
       // drain: every load issued must have landed before the CTA may exit
       for (int st = 0; st < C::STAGES; ++st) {
@@ -109,24 +141,34 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, D, false, false);
-      bool any = false;
-      for (int j = 0; j < kEvict; ++j) {
-        const int st = j % C::STAGES;
-        if (!mbar_wait(&full[st], (j / C::STAGES) & 1, abort_flag)) break;
+      bool any = false, ok = true;
+      int it = 0, n = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++n) {
+        const int ab = n & 1;
+        if (n >= 2 && !mbar_wait(&acc_empty[ab], ((n >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(stages + st * C::STAGE_BYTES);
-        const uint32_t b = a + C::A_BYTES;
+        const uint32_t acc = tmem + ab * C::TMEM_COLS;
+        for (int j = 0; j < kEvict; ++j, ++it) {
+          const int st = it % C::STAGES;
+          if (!mbar_wait(&full[st], (it / C::STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(stages + st * C::STAGE_BYTES);
+          const uint32_t b = a + C::A_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks & 3) * 32;
-          const uint64_t ad = sdesc_sw128(a + (ks >> 2) * (C::BM * 128) + koff, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b + (ks >> 2) * (D * 128) + koff, 16, 1024);
-          mma_ss(tmem, ad, bd, idesc, (j | ks) != 0);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t koff = (ks & 3) * 32;
+            const uint64_t ad = sdesc_sw128(a + (ks >> 2) * (C::BM * 128) + koff, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b + (ks >> 2) * (D * 128) + koff, 16, 1024);
+            mma_ss(acc, ad, bd, idesc, (j | ks) != 0);
+          }
+          any = true;
+          tc_commit(&empty[st]);
         }
-        any = true;
-        tc_commit(&empty[st]);
+        if (ok) tc_commit(&acc_full[ab]);
       }
-      tc_commit(acc_full);
       if (any) {
         volatile int no_abort = 0;
         tc_commit(drain);
@@ -134,19 +176,24 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
       }
     }
   } else {
-    // epilogue: warps 2..5 -> TMEM lanes 32*(warp%4) .. +31
+    // epilogue: warps 2..5 -> TMEM lanes 32*(warp%4) .. +31, one token row each
     const int lane_base = (warp & 3) * 32;
     const int r = lane_base + lane;
-    const int token = mt * C::BM + r;
-    if (mbar_wait_warp(acc_full, 0, abort_flag)) {
+    int n = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
+      const int ab = n & 1;
+      if (!mbar_wait_warp(&acc_full[ab], (n >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      __nv_bfloat16* dst_base = static_cast<__nv_bfloat16*>(kv ? p.memV : p.memK);
-      const int64_t row = (static_cast<int64_t>(state) * p.C + p.grp[g].mem_pos) * p.T + token;
-      uint4* dst = reinterpret_cast<uint4*>(dst_base + (row * p.H + head) * D);
+      const ConvUnit cu = conv_unit(u, MT, p);
+      const int token = cu.mt * C::BM + r;
+      __nv_bfloat16* dst_base = static_cast<__nv_bfloat16*>(cu.kv ? p.memV : p.memK);
+      const int64_t row = (static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token;
+      uint4* dst = reinterpret_cast<uint4*>(dst_base + (row * p.H + cu.head) * D);
+      const uint32_t tacc = tmem + ab * C::TMEM_COLS + (static_cast<uint32_t>(lane_base) << 16);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+        tmem_ld32(tacc + c * 32, v);
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
@@ -156,6 +203,9 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
           for (int q = 0; q < 4; ++q) dst[c * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
+      // the accumulator may be overwritten once every row of it has been read
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
     }
   }
 
@@ -163,7 +213,7 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, kStatusTimeout);
 }
@@ -171,8 +221,8 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 
 // ---------------------------------------------------------------------------
 // fp8 (e4m3) format.  The evicted frames are e4m3 with one fp32 scale per
-// (frame, head); the A operand is dequantised to bf16 (x * scale) in shared
-// memory by warps 2-5 instead of TMA.  The slot is stored e4m3 with one scale
+// (frame, head); the A operand's codes arrive by TMA and are dequantised to bf16
+// (x * scale) in shared memory by warps 6-9.  The slot is stored e4m3 with one scale
 // per (slot, head) = amax / 448 over the slot's [T, D] values, so the launch
 // runs twice: pass 1 only reduces amax (atomicMax on the fp32 bit pattern,
 // values are non-negative), pass 2 recomputes the same tiles and quantises
@@ -192,44 +242,80 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3(float lo, float hi) {
   return r;
 }
 
+// Low-precision A operand: the evicted frame's code tile (128 token rows of CB code
+// bytes of one head) is staged by TMA into the upper half of the A stage, with the
+// CB-byte swizzle, and expanded in place into the bf16 tile by warps 6-9 (one row
+// each).  For e4m3 at D = 128 a row's codes lie under its own output only; otherwise
+// the converting threads read their codes, meet at a barrier, then write.
+template <int D, int FMT>
+struct LowpA {
+  static constexpr int CB = FMT == 2 ? D / 2 : D;
+  static constexpr int BYTES = 128 * CB;
+  static constexpr int OFF = ConvCfg<D>::A_BYTES / 2;
+  static constexpr int NCH = CB / 16;
+  static constexpr uint32_t MASK = CB == 128 ? 7u : (CB == 64 ? 3u : 1u);
+  static constexpr bool SELF = FMT == 1 && D == 128;
+};
+
+__device__ __forceinline__ bool conv_bar_all(int id, int nthreads, bool v) {
+  uint32_t r;
+  __syncwarp();
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+template <int D>
+struct LowpCfg {
+  static constexpr int THREADS = 320;  // producer, MMA, 4 epilogue warps, 4 converter warps
+};
+
+// Persistent like the bf16 kernel: CTAs walk the units, the accumulator is double-
+// buffered in TMEM.  PASS 1 reduces each slot's amax; PASS 2 recomputes the same
+// tiles and quantises with it.
 template <int D, int PASS, int FMT>
-__global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
-    conv_lowp_kernel(const __grid_constant__ CUtensorMap tmW, const ConvParams p) {
+__global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
+    conv_lowp_kernel(const __grid_constant__ CUtensorMap tmCodesK, const __grid_constant__ CUtensorMap tmCodesV,
+                     const __grid_constant__ CUtensorMap tmW, const ConvParams p, int MT, int units) {
   using C = ConvCfg<D>;
+  using LA = LowpA<D, FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::STAGES * C::STAGE_BYTES);
-  uint64_t* b_full = bars;                    // [STAGES] weights landed (TMA)
-  uint64_t* a_full = bars + C::STAGES;        // [STAGES] A dequantised (128 threads)
-  uint64_t* empty = bars + 2 * C::STAGES;     // [STAGES]
-  uint64_t* acc_full = bars + 3 * C::STAGES;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* full = bars;                       // [STAGES] codes + weights landed (TMA)
+  uint64_t* a_ready = bars + C::STAGES;        // [STAGES] A expanded to bf16 (128 threads)
+  uint64_t* empty = bars + 2 * C::STAGES;      // [STAGES]
+  uint64_t* acc_full = bars + 3 * C::STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  unsigned int* red = reinterpret_cast<unsigned int*>(tmem_slot + 2);  // CTA amax
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, head = blockIdx.y;
-  const int kv = blockIdx.z & 1;
-  const int sg = blockIdx.z >> 1;
-  const int state = sg % p.S;
-  const int g = sg / p.S;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&b_full[i], 1);
-      mbar_init(&a_full[i], 128);
+      mbar_init(&full[i], 1);
+      mbar_init(&a_ready[i], 128);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *red = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_alloc(tmem_slot, 2 * C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -239,116 +325,164 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      tma_prefetch_desc(&tmCodesK);
+      tma_prefetch_desc(&tmCodesV);
       tma_prefetch_desc(&tmW);
       int issued[C::STAGES] = {};
-      for (int j = 0; j < kEvict; ++j) {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(&empty[st], ((j / C::STAGES) - 1) & 1, abort_flag)) break;
-        uint8_t* b = stages + st * C::STAGE_BYTES + C::A_BYTES;
-        mbar_expect_tx(&b_full[st], C::B_BYTES);
-        const int wrow = ((kv * p.H + head) * kEvict + j) * D;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const ConvUnit cu = conv_unit(u, MT, p);
+        const CUtensorMap* codes = cu.kv ? &tmCodesV : &tmCodesK;
+        for (int j = 0; j < kEvict; ++j, ++it) {
+          const int st = it % C::STAGES;
+          if (it >= C::STAGES && !mbar_wait(&empty[st], ((it / C::STAGES) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a = stages + st * C::STAGE_BYTES;
+          uint8_t* b = a + C::A_BYTES;
+          mbar_expect_tx(&full[st], LA::BYTES + C::B_BYTES);
+          const int row = p.grp[cu.g].ring_slot[j] * p.T + cu.mt * C::BM;
+          tma_load_4d(a + LA::OFF, codes, &full[st], 0, cu.head, row, cu.state);
+          const int wrow = ((cu.kv * p.H + cu.head) * kEvict + j) * D;
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx) tma_load_3d(b + bx * (D * 128), &tmW, &b_full[st], bx * 64, wrow, state);
-        ++issued[st];
+          for (int bx = 0; bx < C::NBOX; ++bx) tma_load_3d(b + bx * (D * 128), &tmW, &full[st], bx * 64, wrow, cu.state);
+          ++issued[st];
+        }
       }
-      volatile int no_abort = 0;
-      for (int st = 0; st < C::STAGES; ++st)
-        if (issued[st] > 0) mbar_wait(&b_full[st], (issued[st] - 1) & 1, &no_abort);
+      for (int st = 0; st < C::STAGES; ++st) {
+        if (issued[st] > 0) {
+          volatile int no_abort = 0;
+          mbar_wait(&full[st], (issued[st] - 1) & 1, &no_abort);
+        }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, D, false, false);
-      bool any = false;
-      for (int j = 0; j < kEvict; ++j) {
-        const int st = j % C::STAGES;
-        if (!mbar_wait(&a_full[st], (j / C::STAGES) & 1, abort_flag)) break;
-        if (!mbar_wait(&b_full[st], (j / C::STAGES) & 1, abort_flag)) break;
+      bool any = false, ok = true;
+      int it = 0, n = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++n) {
+        const int ab = n & 1;
+        if (n >= 2 && !mbar_wait(&acc_empty[ab], ((n >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(stages + st * C::STAGE_BYTES);
-        const uint32_t b = a + C::A_BYTES;
+        const uint32_t acc = tmem + ab * C::TMEM_COLS;
+        for (int j = 0; j < kEvict; ++j, ++it) {
+          const int st = it % C::STAGES;
+          // the weights' TMA (full) and the expanded A (a_ready) of the stage
+          if (!mbar_wait(&full[st], (it / C::STAGES) & 1, abort_flag) ||
+              !mbar_wait(&a_ready[st], (it / C::STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(stages + st * C::STAGE_BYTES);
+          const uint32_t b = a + C::A_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks & 3) * 32;
-          const uint64_t ad = sdesc_sw128(a + (ks >> 2) * (C::BM * 128) + koff, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b + (ks >> 2) * (D * 128) + koff, 16, 1024);
-          mma_ss(tmem, ad, bd, idesc, (j | ks) != 0);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t koff = (ks & 3) * 32;
+            const uint64_t ad = sdesc_sw128(a + (ks >> 2) * (C::BM * 128) + koff, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b + (ks >> 2) * (D * 128) + koff, 16, 1024);
+            mma_ss(acc, ad, bd, idesc, (j | ks) != 0);
+          }
+          any = true;
+          tc_commit(&empty[st]);
         }
-        any = true;
-        tc_commit(&empty[st]);
+        if (ok) tc_commit(&acc_full[ab]);
       }
-      tc_commit(acc_full);
       if (any) {
         volatile int no_abort = 0;
         tc_commit(drain);
         mbar_wait(drain, 0, &no_abort);
       }
     }
-  } else {
-    // warps 2..5: dequantise A (one token row per thread), then drain the accumulator
-    const int lane_base = (warp & 3) * 32;
-    const int r = lane_base + lane;
-    const int token = mt * C::BM + r;
-    const bool valid = token < p.T;
-    bool alive = true;
-    for (int j = 0; j < kEvict; ++j) {
-      const int st = j % C::STAGES;
-      if (j >= C::STAGES && !mbar_wait(&empty[st], ((j / C::STAGES) - 1) & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      const int slot = p.grp[g].ring_slot[j];
-      const float sc = __ldg(&p.ring_scale[((static_cast<int64_t>(state) * 2 + kv) * p.R + slot) * p.H + head]);
-      const int64_t grow = (static_cast<int64_t>(state) * p.R * p.T + static_cast<int64_t>(slot) * p.T + token) * p.H + head;
-      uint8_t* rowp = stages + st * C::STAGE_BYTES + r * 128;
-      const int sw = r & 7;
-      if (FMT == 2) {
-        // e2m1 pairs: 4 bytes per 8 channels, one e4m3 block scale per 16 channels
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.ring8[kv] + grow * (D / 2));
-        const uint8_t* bs = p.ring_bs[kv] + grow * (D / 16);
+  } else if (warp >= 6) {
+    // warps 6..9: expand each staged code tile to bf16 rows (bf16(fp32(code * scale)))
+    const int r = threadIdx.x - 192;
+    int it = 0;
+    bool live = true;
+    for (int u = blockIdx.x; u < units && live; u += gridDim.x) {
+      const ConvUnit cu = conv_unit(u, MT, p);
+      const int token = cu.mt * C::BM + r;
+      const bool valid = token < p.T;
+      for (int j = 0; j < kEvict; ++j, ++it) {
+        const int st = it % C::STAGES;
+        bool ok = mbar_wait(&full[st], (it / C::STAGES) & 1, abort_flag);
+        uint8_t* a = stages + st * C::STAGE_BYTES;
+        const int slot = p.grp[cu.g].ring_slot[j];
+        const float sc = __ldg(&p.ring_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.R + slot) * p.H + cu.head]);
+        const int64_t grow =
+            (static_cast<int64_t>(cu.state) * p.R * p.T + static_cast<int64_t>(slot) * p.T + token) * p.H + cu.head;
+        uint4 raw[LA::NCH];
+        uint32_t bsw[D / 64 > 0 ? D / 64 : 1];
+        if (ok) {
+#pragma unroll
+          for (int k = 0; k < LA::NCH; ++k) {
+            const uint32_t logical = static_cast<uint32_t>(r * LA::CB + k * 16);
+            const uint32_t phys = logical ^ (((logical >> 7) & LA::MASK) << 4);
+            raw[k] = valid ? *reinterpret_cast<const uint4*>(a + LA::OFF + phys) : make_uint4(0, 0, 0, 0);
+          }
+          if constexpr (FMT == 2) {
+            const uint32_t* bs = reinterpret_cast<const uint32_t*>(p.ring_bs[cu.kv] + grow * (D / 16));
+#pragma unroll
+            for (int k = 0; k < D / 64; ++k) bsw[k] = valid ? __ldg(bs + k) : 0u;
+          }
+        }
+        if constexpr (!LA::SELF) ok = conv_bar_all(1, 128, ok);
+        if (!ok) {
+          live = false;
+          break;
+        }
+        uint8_t* rowp = a + r * 128;
+        const int sw = r & 7;
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
-          uint32_t o[4] = {0, 0, 0, 0};
-          if (valid) {
-            const float e_b = __fmul_rn(fp4::e4m3_to_f32(__ldg(bs + (c >> 1))), sc);
-            fp4::decode8(__ldg(src + c), e_b, o);
-          }
-          *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
-              make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      } else {
-      const uint8_t* src = p.ring8[kv] + grow * D;
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint4 raw = valid ? __ldg(reinterpret_cast<const uint4*>(src) + k) : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 2 * k + u;
           uint32_t o[4];
+          if constexpr (FMT == 2) {
+            const uint4 r4 = raw[c >> 2];
+            const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
+            const int b = c >> 1;
+            const float e_b = __fmul_rn(fp4::e4m3_to_f32(bsw[b >> 2] >> (8 * (b & 3))), sc);
+            fp4::decode8(word, e_b, o);
+          } else {
+            const uint4 r4 = raw[c >> 1];
+            const uint32_t w0 = (c & 1) ? r4.z : r4.x, w1 = (c & 1) ? r4.w : r4.y;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t word = w[2 * u + (q >> 1)];
-            float a, b;
-            e4m3x2_to_f32_c((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
-            o[q] = pack_bf16x2(a * sc, b * sc);
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t word = q < 2 ? w0 : w1;
+              float x0, x1;
+              e4m3x2_to_f32_c((q & 1) ? (word >> 16) : (word & 0xFFFFu), x0, x1);
+              o[q] = pack_bf16x2(x0 * sc, x1 * sc);
+            }
           }
           *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
               make_uint4(o[0], o[1], o[2], o[3]);
         }
+        fence_proxy_async_smem();
+        mbar_arrive(&a_ready[st]);
       }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&a_full[st]);
     }
-    if (alive && mbar_wait_warp(acc_full, 0, abort_flag)) {
+  } else {
+    // warps 2..5: drain the accumulator -> amax (pass 1) or codes (pass 2)
+    const int lane_base = (warp & 3) * 32;
+    const int r = lane_base + lane;
+    int n = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
+      const int ab = n & 1;
+      if (!mbar_wait_warp(&acc_full[ab], (n >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      const int64_t aidx = ((static_cast<int64_t>(state) * 2 + kv) * p.ngroups + g) * p.H + head;
+      const ConvUnit cu = conv_unit(u, MT, p);
+      const int token = cu.mt * C::BM + r;
+      const bool valid = token < p.T;
+      const uint32_t tacc = tmem + ab * C::TMEM_COLS + (static_cast<uint32_t>(lane_base) << 16);
+      const int64_t aidx = ((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.ngroups + cu.g) * p.H + cu.head;
       if (PASS == 1) {
         float mx = 0.0f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+          tmem_ld32(tacc + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(__uint_as_float(v[e])));
@@ -356,16 +490,16 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
         if (!valid) mx = 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) atomicMax(red, __float_as_uint(mx));
+        if (lane == 0 && mx > 0.0f) atomicMax(&p.amax[aidx], __float_as_uint(mx));
       } else if (FMT == 2) {
         const float gs = fp4::tensor_scale(__uint_as_float(p.amax[aidx]));
-        const int64_t row = ((static_cast<int64_t>(state) * p.C + p.grp[g].mem_pos) * p.T + token) * p.H + head;
-        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(kv ? p.memV : p.memK) + row * (D / 2));
-        uint8_t* bs = p.mem_bs[kv] + row * (D / 16);
+        const int64_t row = ((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head;
+        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) + row * (D / 2));
+        uint8_t* bs = p.mem_bs[cu.kv] + row * (D / 16);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+          tmem_ld32(tacc + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int hb = 0; hb < 2; ++hb) {
@@ -385,17 +519,17 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
             }
           }
         }
-        if (mt == 0 && r == 0)
-          p.mem_scale[((static_cast<int64_t>(state) * 2 + kv) * p.C + p.grp[g].mem_pos) * p.H + head] = gs;
+        if (cu.mt == 0 && r == 0)
+          p.mem_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.C + p.grp[cu.g].mem_pos) * p.H + cu.head] = gs;
       } else {
         const float amax = __uint_as_float(p.amax[aidx]);
         const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        uint8_t* dst = static_cast<uint8_t*>(kv ? p.memV : p.memK) +
-                       (((static_cast<int64_t>(state) * p.C + p.grp[g].mem_pos) * p.T + token) * p.H + head) * D;
+        uint8_t* dst = static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) +
+                       (((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+          tmem_ld32(tacc + c * 32, v);
           tmem_ld_wait();
           uint32_t w[8];
 #pragma unroll
@@ -411,21 +545,19 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
             reinterpret_cast<uint4*>(dst)[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
           }
         }
-        if (mt == 0 && r == 0)
-          p.mem_scale[((static_cast<int64_t>(state) * 2 + kv) * p.C + p.grp[g].mem_pos) * p.H + head] = scale;
+        if (cu.mt == 0 && r == 0)
+          p.mem_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.C + p.grp[cu.g].mem_pos) * p.H + cu.head] = scale;
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (PASS == 1 && threadIdx.x == 64 && *red != 0) {
-    const int64_t aidx = ((static_cast<int64_t>(state) * 2 + kv) * p.ngroups + g) * p.H + head;
-    atomicMax(&p.amax[aidx], *red);
-  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 2 * C::TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, kStatusTimeout);
 }
@@ -435,36 +567,47 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 namespace {
 
 template <int D, int FMT>
-int launch_lowp(const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+int launch_lowp(const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV, const CUtensorMap& wmap,
+                cudaStream_t s) {
   using C = ConvCfg<D>;
-  dim3 grid((p.T + 127) / 128, p.H, p.ngroups * p.S * 2);
+  const int MT = (p.T + 127) / 128;
+  const int64_t units64 = static_cast<int64_t>(MT) * p.H * 2 * p.S * p.ngroups;
+  if (units64 > (int64_t(1) << 30)) return static_cast<int>(cudaErrorInvalidValue);
+  const int units = static_cast<int>(units64);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = units < sms ? units : sms;
   auto k1 = conv_lowp_kernel<D, 1, FMT>;
   auto k2 = conv_lowp_kernel<D, 2, FMT>;
   cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  k1<<<grid, C::THREADS, C::SMEM, s>>>(wmap, p);
-  k2<<<grid, C::THREADS, C::SMEM, s>>>(wmap, p);
+  k1<<<grid, LowpCfg<D>::THREADS, C::SMEM, s>>>(codesK, codesV, wmap, p, MT, units);
+  k2<<<grid, LowpCfg<D>::THREADS, C::SMEM, s>>>(codesK, codesV, wmap, p, MT, units);
   return static_cast<int>(cudaGetLastError());
 }
 
 template <int FMT>
-int launch_lowp_d(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
+int launch_lowp_d(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
+                  const CUtensorMap& wmap, cudaStream_t s) {
   if (p.ngroups <= 0) return 0;
   cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(unsigned int) * p.S * 2 * p.ngroups * p.H, s);
   if (e != cudaSuccess) return static_cast<int>(e);
-  if (D == 128) return launch_lowp<128, FMT>(p, wmap, s);
-  if (D == 64) return launch_lowp<64, FMT>(p, wmap, s);
+  if (D == 128) return launch_lowp<128, FMT>(p, codesK, codesV, wmap, s);
+  if (D == 64) return launch_lowp<64, FMT>(p, codesK, codesV, wmap, s);
   return static_cast<int>(cudaErrorInvalidValue);
 }
 
 }  // namespace
 
-int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
-  return launch_lowp_d<1>(D, p, wmap, s);
+int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
+                    const CUtensorMap& wmap, cudaStream_t s) {
+  return launch_lowp_d<1>(D, p, codesK, codesV, wmap, s);
 }
 
-int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& wmap, cudaStream_t s) {
-  return launch_lowp_d<2>(D, p, wmap, s);
+int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
+                    const CUtensorMap& wmap, cudaStream_t s) {
+  return launch_lowp_d<2>(D, p, codesK, codesV, wmap, s);
 }
 
 
@@ -473,15 +616,23 @@ size_t conv_smem_bytes(int D) { return D == 128 ? ConvCfg<128>::SMEM : ConvCfg<6
 int launch_conv_bf16(int D, const ConvParams& p, const CUtensorMap& ringK, const CUtensorMap& ringV,
                      const CUtensorMap& wmap, cudaStream_t s) {
   if (p.ngroups <= 0) return 0;
-  dim3 grid((p.T + 127) / 128, p.H, p.ngroups * p.S * 2);
+  const int MT = (p.T + 127) / 128;
+  const int64_t units64 = static_cast<int64_t>(MT) * p.H * 2 * p.S * p.ngroups;
+  if (units64 > (int64_t(1) << 30)) return static_cast<int>(cudaErrorInvalidValue);
+  const int units = static_cast<int>(units64);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // one persistent CTA per SM (the stage ring takes most of the shared memory)
+  const int grid = units < sms ? units : sms;
   if (D == 128) {
     auto k = conv_bf16_kernel<128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<128>::SMEM);
-    k<<<grid, ConvCfg<128>::THREADS, ConvCfg<128>::SMEM, s>>>(ringK, ringV, wmap, p);
+    k<<<grid, ConvCfg<128>::THREADS, ConvCfg<128>::SMEM, s>>>(ringK, ringV, wmap, p, MT, units);
   } else if (D == 64) {
     auto k = conv_bf16_kernel<64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ConvCfg<64>::SMEM);
-    k<<<grid, ConvCfg<64>::THREADS, ConvCfg<64>::SMEM, s>>>(ringK, ringV, wmap, p);
+    k<<<grid, ConvCfg<64>::THREADS, ConvCfg<64>::SMEM, s>>>(ringK, ringV, wmap, p, MT, units);
   } else {
     return static_cast<int>(cudaErrorInvalidValue);
   }

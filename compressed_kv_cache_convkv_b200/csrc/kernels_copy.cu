@@ -77,6 +77,47 @@ __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __r
   }
 }
 
+// Rotated copies of the reference frames and memory slots for the current time table
+// (bit-identical to rotating them tile by tile in the attention: same table, same
+// rounding).
+template <int D>
+__global__ void rotate_keys_kernel(RotateParams p) {
+  using RC = RopeCfg<D>;
+  const int nf = p.r + p.m;
+  const int64_t total = static_cast<int64_t>(p.S) * nf * p.frame_vecs;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int vpr = p.H * D / 8;
+  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
+  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int64_t sf = i / p.frame_vecs;   // state * nf + frame
+    const int64_t e = i - sf * p.frame_vecs;
+    const int s = static_cast<int>(sf / nf);
+    const int fi = static_cast<int>(sf - static_cast<int64_t>(s) * nf);
+    const uint4* src;
+    uint4* dst;
+    if (fi < p.r) {
+      const int64_t off = (static_cast<int64_t>(s) * p.r + fi) * p.frame_vecs + e;
+      src = static_cast<const uint4*>(p.sink_src) + off;
+      dst = static_cast<uint4*>(p.sink_dst) + off;
+    } else {
+      int pos = p.pos0 + fi - p.r;
+      if (pos >= p.C) pos -= p.C;
+      const int64_t off = (static_cast<int64_t>(s) * p.C + pos) * p.frame_vecs + e;
+      src = static_cast<const uint4*>(p.mem_src) + off;
+      dst = static_cast<uint4*>(p.mem_dst) + off;
+    }
+    const uint4 x = __ldg(src);
+    const int tok = static_cast<int>(e / vpr);
+    const int c = static_cast<int>(e % (D / 8));
+    const int y = tok / p.grid_w, xx = tok - (tok / p.grid_w) * p.grid_w;
+    const dev::RopeRow rr{p.tables + static_cast<int64_t>(fi) * RC::UT, tab_h + y * RC::UH, tab_w + xx * RC::UW};
+    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    dev::rope_chunk<D, false>(w, c, rr, 1.0f);
+    *dst = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // [S][2][H][D_out][D_in][5] -> [S][2][H][5][D_out][D_in]
 __global__ void permute_weights_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                                        int64_t n, int D) {
@@ -171,7 +212,29 @@ __global__ void append_amax_kernel(const uint4* __restrict__ k, const uint4* __r
     if (sh_amax[h]) atomicMax(&p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h], sh_amax[h]);
 }
 
-// pass 2: quantise into the ring, copy to staging, record the scales.
+// The block's K row chunk as written to staging: rotated at its stream position
+// (frame f of the block at time-table row t_row0 + f) when the tables are given --
+// the current block keeps its RoPE position relative to every later query, like
+// the pre-rotated ring of the bf16 format -- else as is.
+template <int D>
+__device__ __forceinline__ uint4 staged_k(uint4 x, const AppendParams& p, int f, int64_t e) {
+  if (!p.tables) return x;
+  using RC = RopeCfg<D>;
+  const int vpr = p.H * D / 8;
+  const int tok = static_cast<int>(e / vpr);
+  const int c = static_cast<int>(e % (D / 8));
+  const int y = tok / p.grid_w, xx = tok - (tok / p.grid_w) * p.grid_w;
+  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
+  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
+  const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.t_row0 + f) * RC::UT, tab_h + y * RC::UH,
+                        tab_w + xx * RC::UW};
+  uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  dev::rope_chunk<D, false>(w, c, rr, 1.0f);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// pass 2: quantise into the ring, copy to staging (K rotated), record the scales.
+template <int D>
 __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   const int64_t fv = p.frame_elems / 8;
   const int64_t per_kv = static_cast<int64_t>(p.S) * p.b * fv;
@@ -187,7 +250,8 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
     const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
     const int h = static_cast<int>((e % vec_per_row) * 8 / p.D);
     const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
-    reinterpret_cast<uint4*>(p.stage[kv])[(static_cast<int64_t>(s) * p.stage_frames + f) * fv + e] = x;
+    reinterpret_cast<uint4*>(p.stage[kv])[(static_cast<int64_t>(s) * p.stage_frames + f) * fv + e] =
+        kv == 0 ? staged_k<D>(x, p, f, e) : x;
     const float amax = __uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]);
     const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -214,7 +278,9 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
 }
 
 // NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
-// e2m1 codes into the ring, the bf16 values into staging, the tensor scale once.
+// e2m1 codes into the ring, the bf16 values into staging (K rotated), the tensor
+// scale once.
+template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   const int nb = p.D / fp4::kBlock;                           // blocks per token-head
   const int64_t T = p.frame_elems / (static_cast<int64_t>(p.H) * p.D);
@@ -236,8 +302,8 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
     const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
     const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
     uint4* st = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv + e0;
-    st[0] = x0;
-    st[1] = x1;
+    st[0] = kv == 0 ? staged_k<D>(x0, p, f, e0) : x0;
+    st[1] = kv == 0 ? staged_k<D>(x1, p, f, e0 + 1) : x1;
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
     float xs[fp4::kBlock];
     float a_b = 0.0f;
@@ -270,6 +336,14 @@ int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void
   return static_cast<int>(cudaGetLastError());
 }
 
+int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(p.S) * (p.r + p.m) * p.frame_vecs;
+  if (total == 0) return 0;
+  auto kern = D == 128 ? rotate_keys_kernel<128> : rotate_keys_kernel<64>;
+  kern<<<grid_for(total, 256), 256, 0, s>>>(p);
+  return static_cast<int>(cudaGetLastError());
+}
+
 int launch_permute_weights(const void* src, void* dst, int S, int H, int D, cudaStream_t s) {
   const int64_t n = static_cast<int64_t>(S) * 2 * H * kEvict * D * D;
   permute_weights_kernel<<<grid_for(n, 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src),
@@ -298,12 +372,13 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   if (e != cudaSuccess) return static_cast<int>(e);
   if (p.fp4) {
     const int64_t blocks = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / fp4::kBlock);
-    append_quant_fp4_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(static_cast<const uint4*>(k),
-                                                                   static_cast<const uint4*>(v), p);
+    auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
+    kern<<<grid_for(blocks, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
   const int64_t total = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
-  append_quant_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+  auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
+  kern<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }
 
