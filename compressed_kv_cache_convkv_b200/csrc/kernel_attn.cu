@@ -35,6 +35,7 @@
 #include "convkv_internal.h"
 #include "sm100.cuh"
 #include "nvfp4.cuh"
+#include "lowp_codes.cuh"
 #include "rope.cuh"
 
 namespace ckv {
@@ -169,12 +170,18 @@ struct RowCodes {
   }
 
   // Dequantise to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale = fp32(s_b * g)),
-  // rotate (ROTATE) and store as row `row` of the 128-byte-swizzled bf16 tile.
+  // rotate (ROTATE) and store as row `row` of the 128-byte-swizzled bf16 tile.  The
+  // codes are widened by moving bits (values times a power of two) and the scale
+  // carries the inverse power, so each product -- and its rounding -- is exactly
+  // code * scale; a scale too large for that fold takes the conversion instructions.
   template <bool ROTATE>
   __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr) const {
     using C = AttnCfg<D>;
     uint8_t* rowp = tile + row * 128;
     const int sw = row & 7;
+    const bool fold = QF == 2 ? (sc < kFp4FoldLimit) : (sc < kE4m3FoldLimit);
+    const float scf = sc * kTwo120;
+    const uint64_t sc2 = f2_make(scf, scf);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
       uint32_t o[4];
@@ -183,16 +190,25 @@ struct RowCodes {
         const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
         const int b = c >> 1;  // block of 16 channels
         const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), sc);
-        fp4::decode8(word, e_b, o);
+        if (fold && e_b < kFp4FoldLimit) {
+          const float ebf = e_b * kTwo112;
+          e2m1x8_to_bf16(word, f2_make(ebf, ebf), o);
+        } else {
+          fp4::decode8(word, e_b, o);
+        }
       } else {
         const uint4 r4 = raw[c >> 1];
         const uint32_t w0 = (c & 1) ? r4.z : r4.x, w1 = (c & 1) ? r4.w : r4.y;
+        if (fold) {
+          e4m3x8_to_bf16(w0, w1, sc2, o);
+        } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t word = q < 2 ? w0 : w1;
-          float a, b;
-          e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
-          o[q] = pack_bf16x2(a * sc, b * sc);
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t word = q < 2 ? w0 : w1;
+            float a, b;
+            e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
+            o[q] = pack_bf16x2(a * sc, b * sc);
+          }
         }
       }
       if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
