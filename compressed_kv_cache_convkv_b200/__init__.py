@@ -16,7 +16,9 @@ from typing import Optional, Tuple
 from .configs import PRESETS, Workload  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "lib", "libconvkv.so")
+# the in-tree build; CONVKV_LIB names another build of the same sources (a variant
+# compiled with other -D options), loaded in its place
+LIB_PATH = os.environ.get("CONVKV_LIB") or os.path.join(_HERE, "lib", "libconvkv.so")
 
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_BAD_ORDER, ERR_OOM, ERR_CUDA, ERR_DEVICE_TIMEOUT = -1, -2, -3, -4, -5, -6

@@ -108,14 +108,6 @@ __device__ __forceinline__ void load_row(uint8_t* tile, int row, const __nv_bflo
   }
 }
 
-// Two e4m3 codes (low byte first) -> two fp32 values (exact).
-__device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
-  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
-}
-
 // Code tiles of the e4m3 / NVFP4 cache, staged by TMA: 128 rows of CB bytes (the
 // codes of one head's row), written with the CB-byte swizzle into the upper half of
 // a stage buffer, and turned into the bf16 tile in place.
@@ -143,18 +135,27 @@ __device__ __forceinline__ uint4 code_chunk(const uint8_t* codes, int r, int c) 
   return *reinterpret_cast<const uint4*>(codes + phys);
 }
 
-// The codes of one row (zeros for rows past the segment) and, for NVFP4, its block
-// scales from global memory.
+// The codes of (part of) one row, zeros for rows past the segment, and for NVFP4 the
+// row's block scales from global memory.  For e4m3 at D = 128 a row is handled in two
+// halves of 64 channels (the second half's codes are read after the first half's
+// output, which does not cover them, is written), so at most 16 code registers are
+// live; otherwise the whole row's codes (at most 64 bytes) are held.
 template <int D, int QF>
 struct RowCodes {
-  uint4 raw[CodeCfg<D, QF>::NCH];
-  uint32_t bs[CodeCfg<D, QF>::SCALE_WORDS > 0 ? CodeCfg<D, QF>::SCALE_WORDS : 1];
+  using CC = CodeCfg<D, QF>;
+  static constexpr int NR = CC::SELF ? CC::NCH / 2 : CC::NCH;   // 16-byte code chunks held at once
+  static constexpr int CPR = QF == 2 ? 4 : 2;                    // 8-channel chunks per 16 code bytes
+  static constexpr int PARTS = CC::NCH / NR;                     // 2 (SELF) or 1 (used by the SELF paths)
+  static constexpr int CHUNKS = NR * CPR;                        // 8-channel chunks per part
+  uint4 raw[NR];
+  uint32_t bs[CC::SCALE_WORDS > 0 ? CC::SCALE_WORDS : 1];
 
-  __device__ __forceinline__ void load(const uint8_t* codes, int r, bool valid, const uint8_t* bs_row) {
-    using CC = CodeCfg<D, QF>;
+  __device__ __forceinline__ void load_codes(const uint8_t* codes, int r, bool valid, int part) {
 #pragma unroll
-    for (int k = 0; k < CC::NCH; ++k)
-      raw[k] = valid ? code_chunk<CC::CB, CC::MASK>(codes, r, k) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < NR; ++k)
+      raw[k] = valid ? code_chunk<CC::CB, CC::MASK>(codes, r, part * NR + k) : make_uint4(0, 0, 0, 0);
+  }
+  __device__ __forceinline__ void load_scales(const uint8_t* bs_row, bool valid) {
     if constexpr (QF == 2) {
       if constexpr (D / 16 >= 4) {
 #pragma unroll
@@ -169,47 +170,36 @@ struct RowCodes {
     }
   }
 
-  // Dequantise to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale = fp32(s_b * g)),
-  // rotate (ROTATE) and store as row `row` of the 128-byte-swizzled bf16 tile.  The
-  // codes are widened by moving bits (values times a power of two) and the scale
-  // carries the inverse power, so each product -- and its rounding -- is exactly
-  // code * scale; a scale too large for that fold takes the conversion instructions.
+  // Dequantise the held chunks to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale =
+  // fp32(s_b * g)), rotate them (ROTATE) and store them as row `row` of the 128-byte-
+  // swizzled bf16 tile; the first held chunk is chunk part * CHUNKS.  The codes are
+  // widened by moving bits to values times a power of two; the scale carries the
+  // inverse power (one product, exactly code * scale), or -- for a scale too large to
+  // carry it -- the power is multiplied out first (exact) and then the scale.
   template <bool ROTATE>
-  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr) const {
+  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr, int part) const {
     using C = AttnCfg<D>;
     uint8_t* rowp = tile + row * 128;
     const int sw = row & 7;
-    const bool fold = QF == 2 ? (sc < kFp4FoldLimit) : (sc < kE4m3FoldLimit);
-    const float scf = sc * kTwo120;
-    const uint64_t sc2 = f2_make(scf, scf);
+    constexpr float kPow = QF == 2 ? kTwo112 : kTwo120;
+    constexpr float kLim = QF == 2 ? kFp4FoldLimit : kE4m3FoldLimit;
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
+    for (int cc = 0; cc < CHUNKS; ++cc) {
+      const int c = part * CHUNKS + cc;
       uint32_t o[4];
       if constexpr (QF == 2) {
-        const uint4 r4 = raw[c >> 2];
-        const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
+        const uint4 r4 = raw[cc >> 2];
+        const uint32_t word = (cc & 3) == 0 ? r4.x : ((cc & 3) == 1 ? r4.y : ((cc & 3) == 2 ? r4.z : r4.w));
         const int b = c >> 1;  // block of 16 channels
         const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), sc);
-        if (fold && e_b < kFp4FoldLimit) {
-          const float ebf = e_b * kTwo112;
-          e2m1x8_to_bf16(word, f2_make(ebf, ebf), o);
-        } else {
-          fp4::decode8(word, e_b, o);
-        }
+        const bool fold = e_b < kLim;
+        const float m1 = fold ? e_b * kPow : kPow;
+        e2m1x8_to_bf16(word, f2_make(m1, m1), fold, f2_make(e_b, e_b), o);
       } else {
-        const uint4 r4 = raw[c >> 1];
-        const uint32_t w0 = (c & 1) ? r4.z : r4.x, w1 = (c & 1) ? r4.w : r4.y;
-        if (fold) {
-          e4m3x8_to_bf16(w0, w1, sc2, o);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t word = q < 2 ? w0 : w1;
-            float a, b;
-            e4m3x2_to_f32((q & 1) ? (word >> 16) : (word & 0xFFFFu), a, b);
-            o[q] = pack_bf16x2(a * sc, b * sc);
-          }
-        }
+        const bool fold = sc < kLim;
+        const float m1 = fold ? sc * kPow : kPow;
+        const uint4 r4 = raw[cc >> 1];
+        e4m3x8_to_bf16((cc & 1) ? r4.z : r4.x, (cc & 1) ? r4.w : r4.y, f2_make(m1, m1), fold, f2_make(sc, sc), o);
       }
       if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
       *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -230,6 +220,34 @@ __device__ __forceinline__ bool bar_all(int id, int nthreads, bool v) {
       : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
+}
+
+// One pair of 2^x (x <= 8) per kExp2PolyPeriod pairs of the softmax is computed on the
+// FMA pipe instead of the exponential unit: x = n + f with n = round(x) (the 1.5 * 2^23
+// rounding constant) and |f| <= 1/2, 2^f by a cubic fitted here for the smallest
+// relative error on [-1/2, 1/2] (Lawson iteration on Chebyshev points), then n added
+// to the exponent field.  Relative error <= 1.5e-4, far below the bf16 rounding of P.
+// x is clamped at -126 (2^-126 in place of smaller weights; masked columns, at -inf,
+// get 2^-126 against V rows that are zero).  0 keeps every exponential on the unit.
+#ifndef CKV_EXP2_POLY_PERIOD
+#define CKV_EXP2_POLY_PERIOD 0
+#endif
+constexpr int kExp2PolyPeriod = CKV_EXP2_POLY_PERIOD;
+
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  const uint64_t magic = f2_make(12582912.0f, 12582912.0f);
+  const uint64_t x = f2_make(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));
+  uint64_t p = f2_fma(f, f2_make(0.055171669626346814f, 0.055171669626346814f),
+                      f2_make(0.24261112621210384f, 0.24261112621210384f));
+  p = f2_fma(p, f, f2_make(0.6932609857037668f, 0.6932609857037668f));
+  p = f2_fma(p, f, f2_make(0.9999280733003428f, 0.9999280733003428f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // QF: storage of the ring and memory segments, 0 bf16, 1 e4m3, 2 NVFP4
@@ -449,40 +467,55 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int nsl = mem ? p.C : p.R;
         const float* scl = mem ? p.mem_scale : p.ring_scale;
         const uint8_t* bsb = mem ? p.mem_bs[1] : p.ring_bs[1];
-        RowCodes<D, QF> rc[2];
-        float sc[2];
-        auto load = [&](int u) {
+        const RopeRow none{nullptr, nullptr, nullptr};
+        // (row, valid, scale) of this thread's rows r0 and r0 + 64
+        auto row_of = [&](int u, bool& valid, float& sc, int64_t& grow) {
           const int r = r0 + 64 * u;
           const int lr = cur.jt * C::BN + r;
-          const bool valid = lr < sg.nrows;
+          valid = lr < sg.nrows;
           const int f = valid ? lr / p.T : 0;
-          const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
-          sc[u] = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-          rc[u].load(codes, r, valid, bsb + (grow * p.H + head) * (D / 16));
+          grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
+          sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
+          return r;
         };
         if constexpr (CC::SELF) {
           if (!ok) break;
           if (sg.fp8) {
-            // each row's codes sit under its own output: convert row by row
-#pragma unroll
+            // each row's codes sit under its own output: convert row by row, half by half
+#pragma unroll 1
             for (int u = 0; u < 2; ++u) {
-              load(u);
-              rc[u].template store<false>(tile, r0 + 64 * u, sc[u], RopeRow{nullptr, nullptr, nullptr});
+              bool valid;
+              float sc;
+              int64_t grow;
+              const int r = row_of(u, valid, sc, grow);
+              RowCodes<D, QF> rc;
+#pragma unroll 1
+              for (int part = 0; part < RowCodes<D, QF>::PARTS; ++part) {
+                rc.load_codes(codes, r, valid, part);
+                rc.template store<false>(tile, r, sc, none, part);
+              }
             }
             fence_proxy_async_smem();
           }
         } else {
+          RowCodes<D, QF> rc[2];
+          float sc[2];
           if (ok && sg.fp8) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) load(u);
+            for (int u = 0; u < 2; ++u) {
+              bool valid;
+              int64_t grow;
+              const int r = row_of(u, valid, sc[u], grow);
+              rc[u].load_codes(codes, r, valid, 0);
+              rc[u].load_scales(bsb + (grow * p.H + head) * (D / 16), valid);
+            }
           }
           // every code of the tile is in registers before any row is written (and a
           // timeout anywhere in the group stops all of it together)
           if (!bar_all(2, 64, ok)) break;
           if (sg.fp8) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
-              rc[u].template store<false>(tile, r0 + 64 * u, sc[u], RopeRow{nullptr, nullptr, nullptr});
+            for (int u = 0; u < 2; ++u) rc[u].template store<false>(tile, r0 + 64 * u, sc[u], none, 0);
             fence_proxy_async_smem();
           }
         }
@@ -568,7 +601,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           const int col = h * 64 + 2 * e;
           float d0, d1;
           f2_split(f2_add(f2_make(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), neg_m), d0, d1);
-          const float p0 = fast_exp2(d0), p1 = fast_exp2(d1);
+          float p0, p1;
+          if (kExp2PolyPeriod > 0 && e % (kExp2PolyPeriod > 0 ? kExp2PolyPeriod : 1) == kExp2PolyPeriod - 1) {
+            exp2_poly_pair(d0, d1, p0, p1);  // on the FMA pipe
+          } else {
+            p0 = fast_exp2(d0);
+            p1 = fast_exp2(d1);
+          }
           sv[h * 64 + e] = pack_bf16x2(p0, p1);
           lsum[e & 3] = f2_add(lsum[e & 3], f2_make(p0, p1));
         }
@@ -655,10 +694,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
         const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
         RowCodes<D, QF> rc;
-        if (ok) rc.load(tile + CC::OFF, r, valid, (mem ? p.mem_bs[0] : p.ring_bs[0]) + (grow * p.H + head) * (D / 16));
-        if constexpr (VOTE) ok = bar_all(1, 128, ok);
-        if (!ok) break;
-        rc.template store<true>(tile, r, sc, rr);
+        if constexpr (CC::SELF) {
+          // each row's codes sit under its own output: convert half by half, no barrier
+          if (!ok) break;
+#pragma unroll 1
+          for (int part = 0; part < RowCodes<D, QF>::PARTS; ++part) {
+            rc.load_codes(tile + CC::OFF, r, valid, part);
+            rc.template store<true>(tile, r, sc, rr, part);
+          }
+        } else {
+          if (ok) {
+            rc.load_codes(tile + CC::OFF, r, valid, 0);
+            rc.load_scales((mem ? p.mem_bs[0] : p.ring_bs[0]) + (grow * p.H + head) * (D / 16), valid);
+          }
+          ok = bar_all(1, 128, ok);
+          if (!ok) break;
+          rc.template store<true>(tile, r, sc, rr, 0);
+        }
       } else {
         if constexpr (VOTE) ok = bar_all(1, 128, ok);
         if (!ok) break;

@@ -437,11 +437,9 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
         }
         uint8_t* rowp = a + r * 128;
         const int sw = r & 7;
-        // codes widened by moving bits, the scale carrying the inverse power of two
-        // (exact; a scale too large for that takes the conversion instructions)
-        const bool fold = FMT == 2 ? (sc < kFp4FoldLimit) : (sc < kE4m3FoldLimit);
-        const float scf = sc * kTwo120;
-        const uint64_t sc2 = f2_make(scf, scf);
+        // codes widened by moving bits to values times a power of two; the scale
+        // carries the inverse power (exact), or for a scale too large for that the
+        // power is multiplied out first (exact) and then the scale
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
           uint32_t o[4];
@@ -450,26 +448,14 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
             const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
             const int b = c >> 1;
             const float e_b = __fmul_rn(fp4::e4m3_to_f32(bsw[b >> 2] >> (8 * (b & 3))), sc);
-            if (fold && e_b < kFp4FoldLimit) {
-              const float ebf = e_b * kTwo112;
-              e2m1x8_to_bf16(word, f2_make(ebf, ebf), o);
-            } else {
-              fp4::decode8(word, e_b, o);
-            }
+            const bool fold = e_b < kFp4FoldLimit;
+            const float m1 = fold ? e_b * kTwo112 : kTwo112;
+            e2m1x8_to_bf16(word, f2_make(m1, m1), fold, f2_make(e_b, e_b), o);
           } else {
+            const bool fold = sc < kE4m3FoldLimit;
+            const float m1 = fold ? sc * kTwo120 : kTwo120;
             const uint4 r4 = raw[c >> 1];
-            const uint32_t w0 = (c & 1) ? r4.z : r4.x, w1 = (c & 1) ? r4.w : r4.y;
-            if (fold) {
-              e4m3x8_to_bf16(w0, w1, sc2, o);
-            } else {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint32_t word = q < 2 ? w0 : w1;
-                float x0, x1;
-                e4m3x2_to_f32_c((q & 1) ? (word >> 16) : (word & 0xFFFFu), x0, x1);
-                o[q] = pack_bf16x2(x0 * sc, x1 * sc);
-              }
-            }
+            e4m3x8_to_bf16((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, f2_make(m1, m1), fold, f2_make(sc, sc), o);
           }
           *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
               make_uint4(o[0], o[1], o[2], o[3]);
