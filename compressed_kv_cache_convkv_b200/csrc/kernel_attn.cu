@@ -145,7 +145,6 @@ struct RowCodes {
   using CC = CodeCfg<D, QF>;
   static constexpr int NR = CC::SELF ? CC::NCH / 2 : CC::NCH;   // 16-byte code chunks held at once
   static constexpr int CPR = QF == 2 ? 4 : 2;                    // 8-channel chunks per 16 code bytes
-  static constexpr int PARTS = CC::NCH / NR;                     // 2 (SELF) or 1 (used by the SELF paths)
   static constexpr int CHUNKS = NR * CPR;                        // 8-channel chunks per part
   uint4 raw[NR];
   uint32_t bs[CC::SCALE_WORDS > 0 ? CC::SCALE_WORDS : 1];
@@ -172,34 +171,45 @@ struct RowCodes {
 
   // Dequantise the held chunks to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale =
   // fp32(s_b * g)), rotate them (ROTATE) and store them as row `row` of the 128-byte-
-  // swizzled bf16 tile; the first held chunk is chunk part * CHUNKS.  The codes are
+  // swizzled bf16 tile; the first held chunk is chunk PART * CHUNKS.  The codes are
   // widened by moving bits to values times a power of two; the scale carries the
   // inverse power (one product, exactly code * scale), or -- for a scale too large to
-  // carry it -- the power is multiplied out first (exact) and then the scale.
-  template <bool ROTATE>
-  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr, int part) const {
+  // carry it, a uniform branch per row -- the power is multiplied out first (exact)
+  // and then the scale.
+  template <bool ROTATE, int PART>
+  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr) const {
+    if constexpr (QF == 2) {
+      store_chunks<ROTATE, PART>(tile, row, sc, rr);
+    } else if (sc < kE4m3FoldLimit) {
+      store_chunks<ROTATE, PART, true>(tile, row, sc * kTwo120, rr);
+    } else {
+      store_chunks<ROTATE, PART, false>(tile, row, sc, rr);
+    }
+  }
+
+  template <bool ROTATE, int PART, bool FOLD = true>
+  __device__ __forceinline__ void store_chunks(uint8_t* tile, int row, float m, const RopeRow& rr) const {
     using C = AttnCfg<D>;
     uint8_t* rowp = tile + row * 128;
     const int sw = row & 7;
-    constexpr float kPow = QF == 2 ? kTwo112 : kTwo120;
-    constexpr float kLim = QF == 2 ? kFp4FoldLimit : kE4m3FoldLimit;
 #pragma unroll
     for (int cc = 0; cc < CHUNKS; ++cc) {
-      const int c = part * CHUNKS + cc;
+      constexpr int c0 = PART * CHUNKS;
+      const int c = c0 + cc;
       uint32_t o[4];
       if constexpr (QF == 2) {
         const uint4 r4 = raw[cc >> 2];
         const uint32_t word = (cc & 3) == 0 ? r4.x : ((cc & 3) == 1 ? r4.y : ((cc & 3) == 2 ? r4.z : r4.w));
         const int b = c >> 1;  // block of 16 channels
-        const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), sc);
-        const bool fold = e_b < kLim;
-        const float m1 = fold ? e_b * kPow : kPow;
-        e2m1x8_to_bf16(word, f2_make(m1, m1), fold, f2_make(e_b, e_b), o);
+        const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), m);
+        if (e_b < kFp4FoldLimit) {
+          e2m1x8_to_bf16<true>(word, e_b * kTwo112, o);
+        } else {
+          e2m1x8_to_bf16<false>(word, e_b, o);
+        }
       } else {
-        const bool fold = sc < kLim;
-        const float m1 = fold ? sc * kPow : kPow;
         const uint4 r4 = raw[cc >> 1];
-        e4m3x8_to_bf16((cc & 1) ? r4.z : r4.x, (cc & 1) ? r4.w : r4.y, f2_make(m1, m1), fold, f2_make(sc, sc), o);
+        e4m3x8_to_bf16<FOLD>((cc & 1) ? r4.z : r4.x, (cc & 1) ? r4.w : r4.y, m, o);
       }
       if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
       *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -489,11 +499,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               int64_t grow;
               const int r = row_of(u, valid, sc, grow);
               RowCodes<D, QF> rc;
-#pragma unroll 1
-              for (int part = 0; part < RowCodes<D, QF>::PARTS; ++part) {
-                rc.load_codes(codes, r, valid, part);
-                rc.template store<false>(tile, r, sc, none, part);
-              }
+              rc.load_codes(codes, r, valid, 0);
+              rc.template store<false, 0>(tile, r, sc, none);
+              rc.load_codes(codes, r, valid, 1);
+              rc.template store<false, 1>(tile, r, sc, none);
             }
             fence_proxy_async_smem();
           }
@@ -515,7 +524,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           if (!bar_all(2, 64, ok)) break;
           if (sg.fp8) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) rc[u].template store<false>(tile, r0 + 64 * u, sc[u], none, 0);
+            for (int u = 0; u < 2; ++u) rc[u].template store<false, 0>(tile, r0 + 64 * u, sc[u], none);
             fence_proxy_async_smem();
           }
         }
@@ -697,11 +706,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         if constexpr (CC::SELF) {
           // each row's codes sit under its own output: convert half by half, no barrier
           if (!ok) break;
-#pragma unroll 1
-          for (int part = 0; part < RowCodes<D, QF>::PARTS; ++part) {
-            rc.load_codes(tile + CC::OFF, r, valid, part);
-            rc.template store<true>(tile, r, sc, rr, part);
-          }
+          rc.load_codes(tile + CC::OFF, r, valid, 0);
+          rc.template store<true, 0>(tile, r, sc, rr);
+          rc.load_codes(tile + CC::OFF, r, valid, 1);
+          rc.template store<true, 1>(tile, r, sc, rr);
         } else {
           if (ok) {
             rc.load_codes(tile + CC::OFF, r, valid, 0);
@@ -709,7 +717,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
           ok = bar_all(1, 128, ok);
           if (!ok) break;
-          rc.template store<true>(tile, r, sc, rr, 0);
+          rc.template store<true, 0>(tile, r, sc, rr);
         }
       } else {
         if constexpr (VOTE) ok = bar_all(1, 128, ok);

@@ -448,14 +448,18 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
             const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
             const int b = c >> 1;
             const float e_b = __fmul_rn(fp4::e4m3_to_f32(bsw[b >> 2] >> (8 * (b & 3))), sc);
-            const bool fold = e_b < kFp4FoldLimit;
-            const float m1 = fold ? e_b * kTwo112 : kTwo112;
-            e2m1x8_to_bf16(word, f2_make(m1, m1), fold, f2_make(e_b, e_b), o);
+            if (e_b < kFp4FoldLimit) {
+              e2m1x8_to_bf16<true>(word, e_b * kTwo112, o);
+            } else {
+              e2m1x8_to_bf16<false>(word, e_b, o);
+            }
           } else {
-            const bool fold = sc < kE4m3FoldLimit;
-            const float m1 = fold ? sc * kTwo120 : kTwo120;
             const uint4 r4 = raw[c >> 1];
-            e4m3x8_to_bf16((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, f2_make(m1, m1), fold, f2_make(sc, sc), o);
+            if (sc < kE4m3FoldLimit) {
+              e4m3x8_to_bf16<true>((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, sc * kTwo120, o);
+            } else {
+              e4m3x8_to_bf16<false>((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, sc, o);
+            }
           }
           *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =
               make_uint4(o[0], o[1], o[2], o[3]);
