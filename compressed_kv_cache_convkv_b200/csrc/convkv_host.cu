@@ -82,14 +82,17 @@ struct convkv {
   // NVFP4: ringK/ringV/memK/memV hold e2m1 pairs; e4m3 block scales per 16 channels
   uint8_t *ringBK = nullptr, *ringBV = nullptr, *memBK = nullptr, *memBV = nullptr;
   void *sinkK = nullptr, *sinkV = nullptr;    // bf16 reference frames, both formats
+  void *scrK = nullptr, *scrV = nullptr;      // e4m3 / NVFP4: bf16 scratch [Sg][(C + W) * T][H][D]
+  int Sg = 0;                                 // states per dequantise-and-attend group
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
   CUtensorMap mapRingK{}, mapRingV{}, mapRingKr{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
       mapSinkV{};
-  // e4m3 / NVFP4: code tiles of the ring and memory, staged by the attention kernel
-  CUtensorMap mapRingCK{}, mapRingCV{}, mapMemCK{}, mapMemCV{};
+  // e4m3 / NVFP4: code tiles of the ring (read by the conv), and the bf16 scratch the
+  // window and memory are dequantised into for each group of Sg states
+  CUtensorMap mapRingCK{}, mapRingCV{}, mapScrK{}, mapScrV{};
   CUtensorMap mapMemKr{}, mapSinkKr{};
   cudaStream_t stream = nullptr;
   int64_t launches = 0;
@@ -195,6 +198,11 @@ int validate(const convkv_cfg* c) {
   // TMA coordinates and row counts are 32-bit
   if (T * (R > c->mem_slots ? R : c->mem_slots) > (int64_t(1) << 30) || T * Bmax > (int64_t(1) << 30) ||
       T * c->sink_frames > (int64_t(1) << 30))
+    return CONVKV_ERR_UNSUPPORTED;
+  // the streaming kernels index a frame's 16-byte vectors with 32-bit integers and put
+  // (state, frame) pairs on the grid's y dimension
+  if (T * c->heads * c->head_dim / 8 > (int64_t(1) << 30) ||
+      int64_t(c->num_states) * (Bmax > c->sink_frames + c->mem_slots ? Bmax : c->sink_frames + c->mem_slots) > 65535)
     return CONVKV_ERR_UNSUPPORTED;
   const int pt = rope_pairs_t(D), ph = rope_pairs_h(D);
   const int64_t tab_units = (int64_t(c->sink_frames) + c->mem_slots + c->window_frames + Bmax) * rope_units(0, pt) +
@@ -322,6 +330,13 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t sink_b = static_cast<size_t>(h->S) * h->Rs * fe * 2;
   const size_t rkr_b = h->prerot ? ring_b : 0;
   const size_t mkr_b = h->prerot ? mem_b : 0;
+  // e4m3 / NVFP4: the dequantisation scratch holds up to 4 GiB of states at a time
+  if (h->fp8) {
+    const size_t per_state = static_cast<size_t>(h->C + h->W) * fe * 2 * 2;
+    const size_t budget = size_t(4) << 30;
+    h->Sg = static_cast<int>(per_state * h->S <= budget ? h->S : (budget / per_state > 0 ? budget / per_state : 1));
+  }
+  const size_t scr_b = h->fp8 ? static_cast<size_t>(h->Sg) * (h->C + h->W) * fe * 2 : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -333,7 +348,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
                o_v = take(io_b), o_o = take(io_b), o_rsc = take(rsc_b), o_msc = take(msc_b), o_sk = take(stg_b),
                o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b),
                o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b),
-               o_rkr = take(rkr_b), o_mkr = take(mkr_b), o_skr = take(sink_b);
+               o_rkr = take(rkr_b), o_mkr = take(mkr_b), o_skr = take(sink_b), o_sck = take(scr_b),
+               o_scv = take(scr_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -356,6 +372,8 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->stageK = a + o_sk;
     h->stageV = a + o_sv;
     h->amax = reinterpret_cast<unsigned int*>(a + o_am);
+    h->scrK = a + o_sck;
+    h->scrV = a + o_scv;
   }
   if (h->fp4) {
     h->ringBK = reinterpret_cast<uint8_t*>(a + o_rbk);
@@ -390,15 +408,16 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   }
   if ((e = cudaStreamSynchronize(h->stream)) != cudaSuccess) goto fail_cuda;
   if (h->fp8) {
-    // the attention stages the ring's and memory's code tiles with TMA and expands
-    // them itself; the bf16 staging of the current block is loaded as is
+    // the conv stages the ring's code tiles with TMA; the attention reads the bf16
+    // staging of the current block and the dequantisation scratch
     const int cb = h->fp4 ? h->D / 2 : h->D;
     rc = encode_4d(&h->mapStageK, h->stageK, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapStageV, h->stageV, h->D, h->H, static_cast<int64_t>(h->Bmax) * h->T, h->S);
     if (!rc) rc = encode_codes(&h->mapRingCK, h->ringK, cb, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_codes(&h->mapRingCV, h->ringV, cb, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
-    if (!rc) rc = encode_codes(&h->mapMemCK, h->memK, cb, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
-    if (!rc) rc = encode_codes(&h->mapMemCV, h->memV, cb, h->H, static_cast<int64_t>(h->C) * h->T, h->S);
+    const int64_t scr_rows = static_cast<int64_t>(h->C + h->W) * h->T;
+    if (!rc) rc = encode_4d(&h->mapScrK, h->scrK, h->D, h->H, scr_rows, h->Sg);
+    if (!rc) rc = encode_4d(&h->mapScrV, h->scrV, h->D, h->H, scr_rows, h->Sg);
   } else {
     rc = encode_4d(&h->mapRingK, h->ringK, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
     if (!rc) rc = encode_4d(&h->mapRingKr, h->ringKr, h->D, h->H, static_cast<int64_t>(h->R) * h->T, h->S);
@@ -460,6 +479,8 @@ static int rotate_moving_keys(convkv_t* h, int64_t B0) {
   rp.tables = h->tables;
   rp.tab_t_rows = h->tab_t_rows;
   rp.tab_h_rows = h->gh;
+  rp.div_heads = FastDiv(static_cast<uint32_t>(h->H));
+  rp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
   const int e = launch_rotate_keys(h->D, rp, h->stream);
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
   if (rp.r + rp.m > 0) h->launches++;
@@ -558,6 +579,8 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
   ap.frame_elems = h->frame_elems();
   ap.H = h->H;
   ap.D = h->D;
+  ap.div_heads = FastDiv(static_cast<uint32_t>(h->H));
+  ap.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
   if (h->prerot || h->fp8) {
     // bf16: K is also written rotated into ringKr; e4m3 / NVFP4: the current block's
     // bf16 staging copy of K is written rotated
@@ -677,49 +700,48 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   ap.Nq = b * T;
   ap.tq0 = r + m + w;
   int tiles = 0;
-  auto add = [&](int buf, int frame0, int nframes, int t0) {
+  // every key segment is bf16 and stored rotated: the ring's rotated K (window and
+  // current, bf16 format), the rotated memory and reference frames, the dequantised
+  // scratch and the rotated staging of the current block (e4m3 / NVFP4 formats)
+  auto add = [&](int buf, int frame0, int nframes, int t0, int local) {
     KeySeg& s = ap.seg[ap.nseg++];
     s.buf = buf;
     s.row0 = frame0 * T;
     s.nrows = nframes * T;
     s.t0 = t0;
     s.tile0 = tiles;
-    s.fp8 = (h->fp8 && buf < 2) ? 1 : 0;
-    // keys stored rotated: the bf16 ring's K (window and current) and the bf16
-    // staging of the current block in the e4m3 / NVFP4 formats
-    s.prerot = ((h->prerot && buf <= 1) || (h->fp8 && buf == 2) || buf == 3) ? 1 : 0;
-    s.slot0 = frame0;
+    s.prerot = 1;
+    s.local = local;
     tiles += (s.nrows + 127) / 128;
   };
-  if (r > 0) add(3, 0, r, 0);
-  if (m > 0) {
-    const int pos0 = static_cast<int>((h->Sn - m) % h->C);
-    const int n1 = m < h->C - pos0 ? m : h->C - pos0;
-    add(1, pos0, n1, r);
-    if (m > n1) add(1, 0, m - n1, r + n1);
-  }
-  {
-    // bf16: window and current block are consecutive ring frames; fp8: the window
-    // is e4m3 in the ring and the current block bf16 in staging
-    const int n = h->fp8 ? w : w + b;
+  if (r > 0) add(3, 0, r, 0, 0);
+  if (h->fp8) {
+    // [memory | window] dequantised into the scratch in attend order, then the
+    // current block's bf16 staging
+    if (m + w > 0) add(0, 0, m + w, r, 1);
+    add(2, 0, b, r + m + w, 0);
+  } else {
+    if (m > 0) {
+      const int pos0 = static_cast<int>((h->Sn - m) % h->C);
+      const int n1 = m < h->C - pos0 ? m : h->C - pos0;
+      add(1, pos0, n1, r, 0);
+      if (m > n1) add(1, 0, m - n1, r + n1, 0);
+    }
+    // window and current block are consecutive ring frames
+    const int n = w + b;
     const int start = static_cast<int>(h->E % h->R);
     const int n1 = n < h->R - start ? n : h->R - start;
-    if (n1 > 0) add(0, start, n1, r + m);
-    if (n > n1) add(0, 0, n - n1, r + m + n1);
-    if (h->fp8) add(2, 0, b, r + m + w);
+    if (n1 > 0) add(0, start, n1, r + m, 0);
+    if (n > n1) add(0, 0, n - n1, r + m + n1, 0);
   }
   ap.ntiles = tiles;
   ap.all_prerot = 1;
-  for (int i = 0; i < ap.nseg; ++i)
-    if (!ap.seg[i].prerot || ap.seg[i].fp8) ap.all_prerot = 0;
   ap.tab_t_rows = h->tab_t_rows;
   ap.tab_h_rows = h->gh;
   ap.tab_w_rows = h->gw;
   ap.tables = h->tables;
   ap.out = static_cast<__nv_bfloat16*>(out);
   ap.q_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->D)));
-  ap.R = h->R;
-  ap.C = h->C;
   ap.status = h->status;
   CUtensorMap mq{};
   if (q_sh) {
@@ -735,28 +757,66 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   }
   CUtensorMap km[4], vm[4];
   if (h->fp8) {
-    ap.ring_scale = h->ring_scale;
-    ap.mem_scale = h->mem_scale;
-    ap.ring8[0] = static_cast<const uint8_t*>(h->ringK);
-    ap.ring8[1] = static_cast<const uint8_t*>(h->ringV);
-    ap.mem8[0] = static_cast<const uint8_t*>(h->memK);
-    ap.mem8[1] = static_cast<const uint8_t*>(h->memV);
-    ap.ring_bs[0] = h->ringBK;
-    ap.ring_bs[1] = h->ringBV;
-    ap.mem_bs[0] = h->memBK;
-    ap.mem_bs[1] = h->memBV;
-    // ring and memory: code tiles (expanded by the kernel); staging: bf16 tiles
-    km[0] = h->mapRingCK; km[1] = h->mapMemCK; km[2] = h->mapStageK;
-    vm[0] = h->mapRingCV; vm[1] = h->mapMemCV; vm[2] = h->mapStageV;
+    km[0] = h->mapScrK; km[1] = h->mapScrK; km[2] = h->mapStageK;
+    vm[0] = h->mapScrV; vm[1] = h->mapScrV; vm[2] = h->mapStageV;
   } else {
     km[0] = h->mapRingKr; km[1] = h->mapMemKr; km[2] = h->mapRingK;
     vm[0] = h->mapRingV; vm[1] = h->mapMemV; vm[2] = h->mapRingV;
   }
   km[3] = r ? h->mapSinkKr : km[2];
   vm[3] = r ? h->mapSinkV : vm[2];
-  int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->fp4 ? 2 : (h->fp8 ? 1 : 0), h->stream);
-  h->launches++;
-  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  if (!h->fp8) {
+    ap.state0 = 0;
+    int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->stream);
+    h->launches++;
+    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    return CONVKV_OK;
+  }
+  // e4m3 / NVFP4: per group of states, dequantise [memory | window] into the scratch
+  // (K rotated), then attend over [reference | scratch | staging]
+  DequantParams dp{};
+  dp.m = m;
+  dp.w = w;
+  dp.r = r;
+  dp.C = h->C;
+  dp.R = h->R;
+  dp.H = h->H;
+  dp.grid_w = h->gw;
+  dp.pos0 = static_cast<int>((h->Sn - m) % h->C);
+  dp.ring0 = static_cast<int>(h->E % h->R);
+  dp.out_frames = h->C + h->W;
+  dp.fp4 = h->fp4 ? 1 : 0;
+  dp.frame_elems = h->frame_elems();
+  dp.ring8[0] = static_cast<const uint8_t*>(h->ringK);
+  dp.ring8[1] = static_cast<const uint8_t*>(h->ringV);
+  dp.mem8[0] = static_cast<const uint8_t*>(h->memK);
+  dp.mem8[1] = static_cast<const uint8_t*>(h->memV);
+  dp.ring_scale = h->ring_scale;
+  dp.mem_scale = h->mem_scale;
+  dp.ring_bs[0] = h->ringBK;
+  dp.ring_bs[1] = h->ringBV;
+  dp.mem_bs[0] = h->memBK;
+  dp.mem_bs[1] = h->memBV;
+  dp.out[0] = h->scrK;
+  dp.out[1] = h->scrV;
+  dp.tables = h->tables;
+  dp.tab_t_rows = h->tab_t_rows;
+  dp.tab_h_rows = h->gh;
+  dp.div_heads = FastDiv(static_cast<uint32_t>(h->H));
+  dp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
+  __nv_bfloat16* const out0 = ap.out;
+  for (int g0 = 0; g0 < h->S; g0 += h->Sg) {
+    const int n = h->S - g0 < h->Sg ? h->S - g0 : h->Sg;
+    dp.state0 = g0;
+    int e = launch_dequant(h->D, dp, n, h->stream);
+    if (m + w > 0) h->launches++;
+    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    ap.state0 = g0;
+    ap.out = out0;
+    e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
+    h->launches++;
+    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  }
   return CONVKV_OK;
 }
 

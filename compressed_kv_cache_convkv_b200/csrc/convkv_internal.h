@@ -18,20 +18,37 @@ __host__ __device__ constexpr int rope_pairs_t(int D) { return (D - 4 * (D / 6))
 // 16-byte table units of an axis whose pairs are global pairs [g, g + n)
 __host__ __device__ constexpr int rope_units(int g, int n) { return (g + n + 1) / 2 - g / 2; }
 
+// Division of a non-negative int (< 2^31) by a fixed divisor d (1 <= d < 2^31) with a
+// multiply-high, shift and add (Granlund and Montgomery, "Division by invariant
+// integers using multiplication", PLDI 1994): l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(m, n) + n) >> l.
+struct FastDiv {
+  uint32_t d = 1, m = 1, l = 0;
+  FastDiv() = default;
+  __host__ explicit FastDiv(uint32_t div) : d(div) {
+    while ((1u << l) < d) ++l;
+    m = static_cast<uint32_t>((((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d) + 1);
+  }
+  __device__ __forceinline__ int div(int n) const {
+    const uint32_t t = __umulhi(m, static_cast<uint32_t>(n));
+    return static_cast<int>((t + static_cast<uint32_t>(n)) >> l);
+  }
+};
+
 // Device status word values (written by kernels, read by convkv_status()).
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
 
-// One contiguous run of key rows in one buffer.
+// One contiguous run of key rows in one buffer (all bf16).
 struct KeySeg {
-  int buf;     // 0 ring, 1 memory, 2 current-block staging (fp8 format only), 3 reference frames
+  int buf;     // tensor map pair: 0 ring (bf16 format) or dequantised scratch (e4m3 / NVFP4),
+               // 1 memory, 2 current-block staging (e4m3 / NVFP4), 3 reference frames
   int row0;    // first row (token) in that buffer, a frame boundary
   int nrows;   // rows = frames * T
   int t0;      // RoPE time index of the segment's first frame
   int tile0;   // index of the segment's first 128-row key tile in the attend's tile list
-  int fp8;     // 1 if the rows are e4m3 with per-(frame, head) fp32 scales
-  int slot0;   // ring slot or memory position of the segment's first frame (row0 / T)
-  int prerot;  // 1 if the K rows are stored already rotated (window and current block, bf16)
+  int prerot;  // 1 if the K rows are stored already rotated
+  int local;   // 1 if the buffer holds only the launch's group of states (the scratch)
 };
 
 // A block's rows (frames * T tokens) split into G contiguous sequence shards, one
@@ -69,15 +86,7 @@ struct AttnParams {
   const float4* tables;
   __nv_bfloat16* out;     // [S][Nq][H][D]
   float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
-  const float* ring_scale;  // fp8: [S][2][R][H]
-  const float* mem_scale;   // fp8: [S][2][C][H]
-  const uint8_t* ring8[2];  // fp8: e4m3 K, V rings [S][R*T][H][D]
-  const uint8_t* mem8[2];   // fp8: e4m3 K, V memory [S][C*T][H][D]
-  // NVFP4: ring8 / mem8 hold e2m1 code pairs [..][D/2], these the e4m3 block scales
-  // [..][D/16]; ring_scale / mem_scale the fp32 scales per (frame or slot, head)
-  const uint8_t* ring_bs[2];
-  const uint8_t* mem_bs[2];
-  int R, C;
+  int state0;             // first state of the launch's group (grid z walks the group)
   int all_prerot;         // every key segment is stored rotated: no RoPE work on K tiles
   int* status;
   // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
@@ -131,6 +140,7 @@ struct AppendParams {
   void* ringKr;
   const float4* tables;
   int tab_t_rows, tab_h_rows, t_row0, grid_w;
+  FastDiv div_heads, div_grid_w;   // by H and by grid_w (token -> head, row, column)
 };
 
 // Rotation of the cached keys that are not stored rotated at append: the r reference
@@ -147,9 +157,31 @@ struct RotateParams {
   void* mem_dst;
   const float4* tables;
   int tab_t_rows, tab_h_rows;
+  FastDiv div_heads, div_grid_w;
+};
+
+// Dequantisation of the e4m3 / NVFP4 window and memory into a bf16 scratch, once per
+// attend and group of states: frame i < m is the memory position (pos0 + i) mod C,
+// frame i >= m the ring slot (ring0 + i - m) mod R; every value is bf16(fp32(code *
+// scale)) (NVFP4 scale fp32(s_b * g)), K rotated with time-table row r + i.  Output
+// [S_group][out_frames * T][H][D] bf16 for K and V, frames in attend order.
+struct DequantParams {
+  int state0, m, w, r, C, R, H, grid_w, pos0, ring0, out_frames, fp4;
+  int64_t frame_elems;            // T * H * D
+  const uint8_t* ring8[2];        // codes: e4m3 [S][R*T][H][D], or NVFP4 pairs [..][D/2]
+  const uint8_t* mem8[2];
+  const float* ring_scale;        // [S][2][R][H]
+  const float* mem_scale;         // [S][2][C][H]
+  const uint8_t* ring_bs[2];      // NVFP4 e4m3 block scales [..][D/16]
+  const uint8_t* mem_bs[2];
+  void* out[2];
+  const float4* tables;
+  int tab_t_rows, tab_h_rows;
+  FastDiv div_heads, div_grid_w;
 };
 
 // Kernel launchers (return cudaError_t of the launch).
+int launch_dequant(int D, const DequantParams& p, int states, cudaStream_t s);
 int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s);
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
                        cudaStream_t s);
@@ -163,10 +195,10 @@ int launch_conv_fp8(int D, const ConvParams& p, const CUtensorMap& codesK, const
 int launch_conv_fp4(int D, const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV,
                     const CUtensorMap& wmap, cudaStream_t s);
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s);
-// k, v: tensor maps of buffers 0..3 (ring, memory, staging, reference frames)
-// fmt: 0 bf16, 1 e4m3, 2 NVFP4 (ring and memory segments)
+// k, v: tensor maps of buffers 0..3 (ring or scratch, memory, staging, reference frames);
+// S: states in the launch (from p.state0)
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k,
-                  const CUtensorMap* v, int S, int fmt, cudaStream_t s);
+                  const CUtensorMap* v, int S, cudaStream_t s);
 size_t attend_smem_bytes(int D, const AttnParams& p);
 size_t conv_smem_bytes(int D);
 

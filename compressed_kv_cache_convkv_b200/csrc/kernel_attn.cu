@@ -22,20 +22,18 @@
 //               the max grows by more than 2^8); P written back over S as bf16
 //   warps 12-15 RoPE of each landed K tile that is not stored rotated, in place
 //               in shared memory (cos/sin tables read through the read-only data
-//               cache); with every key stored rotated (bf16 cache) they are idle and
-//               the MMA issuer takes K tiles straight from TMA
-//   warps 2-3   (e4m3 / NVFP4 cache only) dequantisation of V tiles
-// In the e4m3 / NVFP4 formats the producer stages each ring or memory tile's codes
-// with TMA in the upper half of its stage buffer; the RoPE warpgroup (K) and warps
-// 2-3 (V) turn them into bf16 rows in place.
+//               cache); when every key arrives rotated (the usual case) they are
+//               idle and the MMA issuer takes K tiles straight from TMA
+// Every operand is bf16.  The e4m3 / NVFP4 caches are dequantised (and their keys
+// rotated) once per attend into a bf16 scratch by kernels_dequant.cu, instead of by
+// each of the query-block CTAs that read a tile.  One launch covers a group of
+// states (grid z); p.state0 is the group's first state.
 // TMEM: S_0 | S_1 | O_0 | O_1 = 128 | 128 | D | D columns of 512.
 // Every barrier wait is bounded; on expiry the CTA raises an abort flag, skips
 // the remaining work, drains its outstanding copies and MMAs, frees TMEM and
 // records CONVKV_ERR_DEVICE_TIMEOUT in the status word.
 #include "convkv_internal.h"
 #include "sm100.cuh"
-#include "nvfp4.cuh"
-#include "lowp_codes.cuh"
 #include "rope.cuh"
 
 namespace ckv {
@@ -59,7 +57,7 @@ struct AttnCfg {
   static constexpr int REG_LAUNCH = 128, REG_CTRL = 96, REG_ROPE = 80, REG_SOFTMAX = 168;
   static_assert(128 * REG_CTRL + 128 * REG_ROPE + 256 * REG_SOFTMAX == THREADS * REG_LAUNCH,
                 "register split must add up to the launch allocation");
-  static constexpr int NBARS = 1 + 1 + 3 * KST + 3 * VST + 3 * 2 + 1;
+  static constexpr int NBARS = 1 + 1 + 3 * KST + 2 * VST + 3 * 2 + 1;
   static constexpr size_t FIXED =
       1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16 + kMaxSegs * sizeof(KeySeg);
 };
@@ -108,160 +106,7 @@ __device__ __forceinline__ void load_row(uint8_t* tile, int row, const __nv_bflo
   }
 }
 
-// Code tiles of the e4m3 / NVFP4 cache, staged by TMA: 128 rows of CB bytes (the
-// codes of one head's row), written with the CB-byte swizzle into the upper half of
-// a stage buffer, and turned into the bf16 tile in place.
-template <int D, int QF>
-struct CodeCfg {
-  static constexpr int CB = QF == 2 ? D / 2 : D;   // code bytes per row
-  static constexpr int BYTES = 128 * CB;
-  static constexpr int OFF = AttnCfg<D>::TILE / 2;  // 1024-aligned
-  static constexpr int NCH = CB / 16;               // 16-byte chunks per row
-  static constexpr uint32_t MASK = CB == 128 ? 7u : (CB == 64 ? 3u : 1u);
-  // e4m3 at D = 128: a row's codes lie inside the bytes of its own bf16 output (the
-  // second 64-channel box), so each thread converts its rows with no barrier.
-  // Otherwise the codes of one row sit under other rows' output: the converting
-  // threads read all their codes, meet at a barrier, then write.
-  static constexpr bool SELF = QF == 1 && D == 128;
-  static constexpr int SCALE_WORDS = QF == 2 ? (D / 16 + 3) / 4 : 0;  // NVFP4 block-scale words per row
-};
-
-// 16-byte chunk c of row r of a staged code tile (the TMA swizzle XORs address bits
-// [4, 7) with bits [7, 10), masked to the swizzle span).
-template <int CB, uint32_t MASK>
-__device__ __forceinline__ uint4 code_chunk(const uint8_t* codes, int r, int c) {
-  const uint32_t logical = static_cast<uint32_t>(r * CB + c * 16);
-  const uint32_t phys = logical ^ (((logical >> 7) & MASK) << 4);
-  return *reinterpret_cast<const uint4*>(codes + phys);
-}
-
-// The codes of (part of) one row, zeros for rows past the segment, and for NVFP4 the
-// row's block scales from global memory.  For e4m3 at D = 128 a row is handled in two
-// halves of 64 channels (the second half's codes are read after the first half's
-// output, which does not cover them, is written), so at most 16 code registers are
-// live; otherwise the whole row's codes (at most 64 bytes) are held.
-template <int D, int QF>
-struct RowCodes {
-  using CC = CodeCfg<D, QF>;
-  static constexpr int NR = CC::SELF ? CC::NCH / 2 : CC::NCH;   // 16-byte code chunks held at once
-  static constexpr int CPR = QF == 2 ? 4 : 2;                    // 8-channel chunks per 16 code bytes
-  static constexpr int CHUNKS = NR * CPR;                        // 8-channel chunks per part
-  uint4 raw[NR];
-  uint32_t bs[CC::SCALE_WORDS > 0 ? CC::SCALE_WORDS : 1];
-
-  __device__ __forceinline__ void load_codes(const uint8_t* codes, int r, bool valid, int part) {
-#pragma unroll
-    for (int k = 0; k < NR; ++k)
-      raw[k] = valid ? code_chunk<CC::CB, CC::MASK>(codes, r, part * NR + k) : make_uint4(0, 0, 0, 0);
-  }
-  __device__ __forceinline__ void load_scales(const uint8_t* bs_row, bool valid) {
-    if constexpr (QF == 2) {
-      if constexpr (D / 16 >= 4) {
-#pragma unroll
-        for (int k = 0; k < CC::SCALE_WORDS; ++k) bs[k] = valid ? __ldg(reinterpret_cast<const uint32_t*>(bs_row) + k) : 0u;
-      } else {
-        // D / 16 block scales per row, fewer than four: byte loads
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) w |= valid ? static_cast<uint32_t>(__ldg(bs_row + k)) << (8 * k) : 0u;
-        bs[0] = w;
-      }
-    }
-  }
-
-  // Dequantise the held chunks to bf16 on use (bf16(fp32(code * scale)); NVFP4 scale =
-  // fp32(s_b * g)), rotate them (ROTATE) and store them as row `row` of the 128-byte-
-  // swizzled bf16 tile; the first held chunk is chunk PART * CHUNKS.  The codes are
-  // widened by moving bits to values times a power of two; the scale carries the
-  // inverse power (one product, exactly code * scale), or -- for a scale too large to
-  // carry it, a uniform branch per row -- the power is multiplied out first (exact)
-  // and then the scale.
-  template <bool ROTATE, int PART>
-  __device__ __forceinline__ void store(uint8_t* tile, int row, float sc, const RopeRow& rr) const {
-    if constexpr (QF == 2) {
-      store_chunks<ROTATE, PART>(tile, row, sc, rr);
-    } else if (sc < kE4m3FoldLimit) {
-      store_chunks<ROTATE, PART, true>(tile, row, sc * kTwo120, rr);
-    } else {
-      store_chunks<ROTATE, PART, false>(tile, row, sc, rr);
-    }
-  }
-
-  template <bool ROTATE, int PART, bool FOLD = true>
-  __device__ __forceinline__ void store_chunks(uint8_t* tile, int row, float m, const RopeRow& rr) const {
-    using C = AttnCfg<D>;
-    uint8_t* rowp = tile + row * 128;
-    const int sw = row & 7;
-#pragma unroll
-    for (int cc = 0; cc < CHUNKS; ++cc) {
-      constexpr int c0 = PART * CHUNKS;
-      const int c = c0 + cc;
-      uint32_t o[4];
-      if constexpr (QF == 2) {
-        const uint4 r4 = raw[cc >> 2];
-        const uint32_t word = (cc & 3) == 0 ? r4.x : ((cc & 3) == 1 ? r4.y : ((cc & 3) == 2 ? r4.z : r4.w));
-        const int b = c >> 1;  // block of 16 channels
-        const float e_b = __fmul_rn(fp4::e4m3_to_f32(bs[b >> 2] >> (8 * (b & 3))), m);
-        if (e_b < kFp4FoldLimit) {
-          e2m1x8_to_bf16<true>(word, e_b * kTwo112, o);
-        } else {
-          e2m1x8_to_bf16<false>(word, e_b, o);
-        }
-      } else {
-        const uint4 r4 = raw[cc >> 1];
-        e4m3x8_to_bf16<FOLD>((cc & 1) ? r4.z : r4.x, (cc & 1) ? r4.w : r4.y, m, o);
-      }
-      if (ROTATE) rope_chunk<D, false>(o, c, rr, 1.0f);
-      *reinterpret_cast<uint4*>(rowp + (c >> 3) * C::BOX + (((c & 7) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-};
-
-// AND of `v` over the `nthreads` threads (whole warps) that meet at named barrier `id`.
-__device__ __forceinline__ bool bar_all(int id, int nthreads, bool v) {
-  uint32_t r;
-  __syncwarp();  // the barrier is warp-aligned: reconverge first
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
-// One pair of 2^x (x <= 8) per kExp2PolyPeriod pairs of the softmax is computed on the
-// FMA pipe instead of the exponential unit: x = n + f with n = round(x) (the 1.5 * 2^23
-// rounding constant) and |f| <= 1/2, 2^f by a cubic fitted here for the smallest
-// relative error on [-1/2, 1/2] (Lawson iteration on Chebyshev points), then n added
-// to the exponent field.  Relative error <= 1.5e-4, far below the bf16 rounding of P.
-// x is clamped at -126 (2^-126 in place of smaller weights; masked columns, at -inf,
-// get 2^-126 against V rows that are zero).  0 keeps every exponential on the unit.
-#ifndef CKV_EXP2_POLY_PERIOD
-#define CKV_EXP2_POLY_PERIOD 0
-#endif
-constexpr int kExp2PolyPeriod = CKV_EXP2_POLY_PERIOD;
-
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  const uint64_t magic = f2_make(12582912.0f, 12582912.0f);
-  const uint64_t x = f2_make(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = f2_add(x, magic);
-  const uint64_t f = f2_sub(x, f2_sub(t, magic));
-  uint64_t p = f2_fma(f, f2_make(0.055171669626346814f, 0.055171669626346814f),
-                      f2_make(0.24261112621210384f, 0.24261112621210384f));
-  p = f2_fma(p, f, f2_make(0.6932609857037668f, 0.6932609857037668f));
-  p = f2_fma(p, f, f2_make(0.9999280733003428f, 0.9999280733003428f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
-// QF: storage of the ring and memory segments, 0 bf16, 1 e4m3, 2 NVFP4
-template <int D, int QF>
+template <int D>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                 const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmK1,
@@ -269,7 +114,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                 const __grid_constant__ CUtensorMap tmV2, const __grid_constant__ CUtensorMap tmK3,
                 const __grid_constant__ CUtensorMap tmV3, const AttnParams p) {
   using C = AttnCfg<D>;
-  constexpr bool FP8 = QF != 0;  // low-precision ring and memory, dequantised in the kernel
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -286,8 +130,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint64_t* s_full = v_empty + C::VST;   // [2]
   uint64_t* p_full = s_full + 2;         // [2]
   uint64_t* o_full = p_full + 2;         // [2]
-  uint64_t* v_ready = o_full + 2;        // [VST] fp8: V tile dequantised by warps 2-3
-  uint64_t* drain = v_ready + C::VST;
+  uint64_t* drain = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   KeySeg* seg = reinterpret_cast<KeySeg*>(tmem_slot + 4);
@@ -297,7 +140,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   const float4* tab_w = tab_h + p.tab_h_rows * C::UH;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.y, state = blockIdx.z;
+  // sl: the state within this launch's group (coordinate of the group-local scratch);
+  // state: its index in the handle (queries, outputs, staging, reference frames)
+  const int head = blockIdx.y, sl = blockIdx.z, state = sl + p.state0;
   const int q_row0 = blockIdx.x * (C::QT * C::BM);
 
   if (threadIdx.x == 0) {
@@ -311,7 +156,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     for (int i = 0; i < C::VST; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
-      mbar_init(&v_ready[i], 64);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -354,31 +198,20 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
         const KeySeg& sg = seg[cur.s];
         const int row = sg.row0 + cur.jt * C::BN;
+        const int st = sg.local ? sl : state;   // the scratch holds only this launch's group
         const int ks = j % C::KST;
         if (j >= C::KST && !mbar_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
-        if (FP8 && sg.fp8) {
-          // the tile's codes into the upper half of the stage; the RoPE warpgroup expands them
-          mbar_expect_tx(&k_full[ks], CodeCfg<D, QF>::BYTES);
-          tma_load_4d(sK + ks * C::TILE + CodeCfg<D, QF>::OFF, kmap(sg.buf), &k_full[ks], 0, head, row, state);
-        } else {
-          mbar_expect_tx(&k_full[ks], C::TILE);
+        mbar_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
-          for (int bx = 0; bx < C::NBOX; ++bx)
-            tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap(sg.buf), &k_full[ks], bx * 64, head, row, state);
-        }
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sK + ks * C::TILE + bx * C::BOX, kmap(sg.buf), &k_full[ks], bx * 64, head, row, st);
         ++kiss[ks];
         const int vs = j % C::VST;
         if (j >= C::VST && !mbar_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, abort_flag)) break;
-        if (FP8 && sg.fp8) {
-          // the tile's codes into the upper half of the stage; warps 2-3 expand them
-          mbar_expect_tx(&v_full[vs], CodeCfg<D, QF>::BYTES);
-          tma_load_4d(sV + vs * C::TILE + CodeCfg<D, QF>::OFF, vmap(sg.buf), &v_full[vs], 0, head, row, state);
-        } else {
-          mbar_expect_tx(&v_full[vs], C::TILE);
+        mbar_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll
-          for (int bx = 0; bx < C::NBOX; ++bx)
-            tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap(sg.buf), &v_full[vs], bx * 64, head, row, state);
-        }
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(sV + vs * C::TILE + bx * C::BOX, vmap(sg.buf), &v_full[vs], bx * 64, head, row, st);
         ++viss[vs];
       }
       // drain: every issued copy must land before the CTA exits
@@ -433,7 +266,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         bool ok = true;
         for (int j = 0; j < p.ntiles && ok; ++j) {
           const int vs = j % C::VST;
-          if (!mbar_wait(FP8 ? &v_ready[vs] : &v_full[vs], (j / C::VST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag)) { ok = false; break; }
           const bool has_next = j + 1 < p.ntiles;
           const int ksn = (j + 1) % C::KST;
           for (int i = 0; i < 2; ++i) {
@@ -462,74 +295,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         mbar_wait(drain, 0, &no_abort);
       }
     }
-  } else if (FP8 && (warp == 2 || warp == 3)) {
-      // ---------------------------------------------------------- V dequantisation
-      using CC = CodeCfg<D, QF>;
-      const int r0 = (warp - 2) * 32 + lane;  // rows r0 and r0 + 64 of each V tile
-      TileCursor cur;
-      for (int j = 0; j < p.ntiles; ++j, cur.next(seg)) {
-        const int vs = j % C::VST;
-        bool ok = mbar_wait(&v_full[vs], (j / C::VST) & 1, abort_flag);
-        const KeySeg& sg = seg[cur.s];
-        uint8_t* tile = sV + vs * C::TILE;
-        const uint8_t* codes = tile + CC::OFF;
-        const bool mem = sg.buf == 1;
-        const int nsl = mem ? p.C : p.R;
-        const float* scl = mem ? p.mem_scale : p.ring_scale;
-        const uint8_t* bsb = mem ? p.mem_bs[1] : p.ring_bs[1];
-        const RopeRow none{nullptr, nullptr, nullptr};
-        // (row, valid, scale) of this thread's rows r0 and r0 + 64
-        auto row_of = [&](int u, bool& valid, float& sc, int64_t& grow) {
-          const int r = r0 + 64 * u;
-          const int lr = cur.jt * C::BN + r;
-          valid = lr < sg.nrows;
-          const int f = valid ? lr / p.T : 0;
-          grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
-          sc = valid ? __ldg(&scl[((static_cast<int64_t>(state) * 2 + 1) * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-          return r;
-        };
-        if constexpr (CC::SELF) {
-          if (!ok) break;
-          if (sg.fp8) {
-            // each row's codes sit under its own output: convert row by row, half by half
-#pragma unroll 1
-            for (int u = 0; u < 2; ++u) {
-              bool valid;
-              float sc;
-              int64_t grow;
-              const int r = row_of(u, valid, sc, grow);
-              RowCodes<D, QF> rc;
-              rc.load_codes(codes, r, valid, 0);
-              rc.template store<false, 0>(tile, r, sc, none);
-              rc.load_codes(codes, r, valid, 1);
-              rc.template store<false, 1>(tile, r, sc, none);
-            }
-            fence_proxy_async_smem();
-          }
-        } else {
-          RowCodes<D, QF> rc[2];
-          float sc[2];
-          if (ok && sg.fp8) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              bool valid;
-              int64_t grow;
-              const int r = row_of(u, valid, sc[u], grow);
-              rc[u].load_codes(codes, r, valid, 0);
-              rc[u].load_scales(bsb + (grow * p.H + head) * (D / 16), valid);
-            }
-          }
-          // every code of the tile is in registers before any row is written (and a
-          // timeout anywhere in the group stops all of it together)
-          if (!bar_all(2, 64, ok)) break;
-          if (sg.fp8) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) rc[u].template store<false, 0>(tile, r0 + 64 * u, sc[u], none);
-            fence_proxy_async_smem();
-          }
-        }
-        mbar_arrive(&v_ready[vs]);
-      }
   }
   } else if (warp < 12) {
     regs_inc<C::REG_SOFTMAX>();
@@ -610,13 +375,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           const int col = h * 64 + 2 * e;
           float d0, d1;
           f2_split(f2_add(f2_make(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1])), neg_m), d0, d1);
-          float p0, p1;
-          if (kExp2PolyPeriod > 0 && e % (kExp2PolyPeriod > 0 ? kExp2PolyPeriod : 1) == kExp2PolyPeriod - 1) {
-            exp2_poly_pair(d0, d1, p0, p1);  // on the FMA pipe
-          } else {
-            p0 = fast_exp2(d0);
-            p1 = fast_exp2(d1);
-          }
+          const float p0 = fast_exp2(d0), p1 = fast_exp2(d1);
           sv[h * 64 + e] = pack_bf16x2(p0, p1);
           lsum[e & 3] = f2_add(lsum[e & 3], f2_make(p0, p1));
         }
@@ -676,53 +435,21 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   } else {
     regs_dec<C::REG_ROPE>();
     // ------------------------------------------------------------ K RoPE
-    using CC = CodeCfg<D, QF>;
-    // staged codes that lie under other rows' output: the warpgroup meets at a barrier
-    // on every tile (uniformly, so a timeout anywhere stops all of it together)
-    constexpr bool VOTE = FP8 && !CC::SELF;
     const int r = threadIdx.x - 384;
     TileCursor cur;
     for (int j = 0; j < (p.all_prerot ? 0 : p.ntiles); ++j, cur.next(seg)) {
       const int ks = j % C::KST;
-      bool ok = mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag);
+      if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
       const KeySeg& sg = seg[cur.s];
       const int lr = cur.jt * C::BN + r;
-      const bool valid = lr < sg.nrows;
-      const int f = valid ? lr / p.T : 0;
-      const int s = valid ? lr - f * p.T : 0;
-      const int t = sg.t0 + f;
-      const int y = s / p.grid_w;
-      const int x = s - y * p.grid_w;
-      const RopeRow rr{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW};
-      uint8_t* tile = sK + ks * C::TILE;
-      if (FP8 && sg.fp8) {
-        // e4m3 / NVFP4 codes staged by TMA: dequantise, rotate, write the bf16 row
-        const bool mem = sg.buf == 1;
-        const int nsl = mem ? p.C : p.R;
-        const float* scl = mem ? p.mem_scale : p.ring_scale;
-        const int64_t grow = static_cast<int64_t>(state) * nsl * p.T + sg.row0 + lr;
-        const float sc = valid ? __ldg(&scl[(static_cast<int64_t>(state) * 2 * nsl + sg.slot0 + f) * p.H + head]) : 0.0f;
-        RowCodes<D, QF> rc;
-        if constexpr (CC::SELF) {
-          // each row's codes sit under its own output: convert half by half, no barrier
-          if (!ok) break;
-          rc.load_codes(tile + CC::OFF, r, valid, 0);
-          rc.template store<true, 0>(tile, r, sc, rr);
-          rc.load_codes(tile + CC::OFF, r, valid, 1);
-          rc.template store<true, 1>(tile, r, sc, rr);
-        } else {
-          if (ok) {
-            rc.load_codes(tile + CC::OFF, r, valid, 0);
-            rc.load_scales((mem ? p.mem_bs[0] : p.ring_bs[0]) + (grow * p.H + head) * (D / 16), valid);
-          }
-          ok = bar_all(1, 128, ok);
-          if (!ok) break;
-          rc.template store<true, 0>(tile, r, sc, rr);
-        }
-      } else {
-        if constexpr (VOTE) ok = bar_all(1, 128, ok);
-        if (!ok) break;
-        if (valid && !sg.prerot) rope_row<D, false>(tile, r, rr, 1.0f);
+      if (lr < sg.nrows && !sg.prerot) {
+        const int f = lr / p.T;
+        const int s = lr - f * p.T;
+        const int t = sg.t0 + f;
+        const int y = s / p.grid_w;
+        const int x = s - y * p.grid_w;
+        rope_row<D, false>(sK + ks * C::TILE, r, RopeRow{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW},
+                           1.0f);
       }
       fence_proxy_async_smem();
       mbar_arrive(&k_ready[ks]);
@@ -746,11 +473,11 @@ size_t smem_for(const AttnParams&) {
   return C::FIXED > 120 * 1024 ? C::FIXED : 120 * 1024;
 }
 
-template <int D, int QF>
+template <int D>
 int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v, int S,
              cudaStream_t s) {
   const size_t smem = smem_for<D>(p);
-  auto kern = attn_kernel<D, QF>;
+  auto kern = attn_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid((p.Nq + 255) / 256, p.H, S);
@@ -763,15 +490,9 @@ int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, co
 size_t attend_smem_bytes(int D, const AttnParams& p) { return D == 128 ? smem_for<128>(p) : smem_for<64>(p); }
 
 int launch_attend(int D, const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, const CUtensorMap* v,
-                  int S, int fmt, cudaStream_t s) {
-  if (D == 128) {
-    if (fmt == 2) return launch_t<128, 2>(p, q, k, v, S, s);
-    return fmt ? launch_t<128, 1>(p, q, k, v, S, s) : launch_t<128, 0>(p, q, k, v, S, s);
-  }
-  if (D == 64) {
-    if (fmt == 2) return launch_t<64, 2>(p, q, k, v, S, s);
-    return fmt ? launch_t<64, 1>(p, q, k, v, S, s) : launch_t<64, 0>(p, q, k, v, S, s);
-  }
+                  int S, cudaStream_t s) {
+  if (D == 128) return launch_t<128>(p, q, k, v, S, s);
+  if (D == 64) return launch_t<64>(p, q, k, v, S, s);
   return static_cast<int>(cudaErrorInvalidValue);
 }
 

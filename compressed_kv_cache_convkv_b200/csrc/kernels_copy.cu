@@ -9,6 +9,18 @@
 namespace ckv {
 namespace {
 
+// Blocks along x for a launch whose y (and z) dimensions cover `frames` frames of
+// `per_frame` work items: about 8 blocks per SM in total, at least one per frame.
+int frame_grid_x(int64_t per_frame, int frames, int threads) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t need = (per_frame + threads - 1) / threads;
+  int64_t want = (static_cast<int64_t>(sms) * 8 + frames - 1) / frames;
+  if (want < 1) want = 1;
+  return static_cast<int>(need < want ? need : want);
+}
+
 int grid_for(int64_t work_items, int threads) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -42,37 +54,42 @@ __device__ __forceinline__ const uint4* block_vec(const void* plain, const void*
 // written rotated into ringKr at the same place: a window or current-block key
 // keeps its RoPE position relative to every later query (both are stream
 // positions), so it is rotated once here instead of at every attend.
+// Table row pointers of token `tok` of a frame whose time index is table row t_row.
+template <int D>
+__device__ __forceinline__ dev::RopeRow rope_row_of(const float4* tables, int tab_t_rows, int tab_h_rows,
+                                                    const FastDiv& div_gw, int grid_w, int t_row, int tok) {
+  using RC = RopeCfg<D>;
+  const float4* tab_h = tables + static_cast<int64_t>(tab_t_rows) * RC::UT;
+  const float4* tab_w = tab_h + static_cast<int64_t>(tab_h_rows) * RC::UH;
+  const int y = div_gw.div(tok);
+  const int x = tok - y * grid_w;
+  return dev::RopeRow{tables + static_cast<int64_t>(t_row) * RC::UT, tab_h + y * RC::UH, tab_w + x * RC::UW};
+}
+
+// grid = (x, states * b): y is the frame, x walks its 16-byte vectors.
 template <int D>
 __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                    uint4* __restrict__ ringK, uint4* __restrict__ ringV, AppendParams p) {
-  using RC = RopeCfg<D>;
-  const int64_t fv = p.frame_elems / 8;  // 16-byte vectors per frame
-  const int vpr = p.H * D / 8;           // vectors per token
-  const int64_t total = static_cast<int64_t>(p.S) * p.b * fv;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
-  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int64_t sf = i / fv;               // state * b + f
-    const int64_t e = i - sf * fv;
-    const int s = static_cast<int>(sf / p.b);
-    const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
-    int slot = p.slot0 + f;
-    if (slot >= p.R) slot -= p.R;
-    const int64_t dst = (static_cast<int64_t>(s) * p.R + slot) * fv + e;
+  constexpr int DV = D / 8;               // 16-byte vectors per head
+  const int fv = static_cast<int>(p.frame_elems / 8);  // 16-byte vectors per frame
+  const int sf = blockIdx.y;              // state * b + frame
+  const int s = sf / p.b;
+  const int f = sf - s * p.b;
+  int slot = p.slot0 + f;
+  if (slot >= p.R) slot -= p.R;
+  const int64_t dst0 = (static_cast<int64_t>(s) * p.R + slot) * fv;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
     const uint4 kv = __ldcs(block_vec(k, p.k_sh, p, s, f, e));
     const uint4 vv = __ldcs(block_vec(v, p.v_sh, p, s, f, e));
-    ringK[dst] = kv;
-    ringV[dst] = vv;
+    ringK[dst0 + e] = kv;
+    ringV[dst0 + e] = vv;
     if (p.ringKr) {
-      const int tok = static_cast<int>(e / vpr);
-      const int c = static_cast<int>(e % (D / 8));  // chunk of 8 channels within the head
-      const int y = tok / p.grid_w, x = tok - (tok / p.grid_w) * p.grid_w;
-      const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.t_row0 + f) * RC::UT, tab_h + y * RC::UH,
-                            tab_w + x * RC::UW};
+      const int tok = p.div_heads.div(e / DV);
+      const dev::RopeRow rr =
+          rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, p.t_row0 + f, tok);
       uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-      dev::rope_chunk<D, false>(w, c, rr, 1.0f);
-      static_cast<uint4*>(p.ringKr)[dst] = make_uint4(w[0], w[1], w[2], w[3]);
+      dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
+      static_cast<uint4*>(p.ringKr)[dst0 + e] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
@@ -80,41 +97,34 @@ __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __r
 // Rotated copies of the reference frames and memory slots for the current time table
 // (bit-identical to rotating them tile by tile in the attention: same table, same
 // rounding).
+// grid = (x, states * (r + m)): y is the frame, x walks its 16-byte vectors.
 template <int D>
 __global__ void rotate_keys_kernel(RotateParams p) {
-  using RC = RopeCfg<D>;
+  constexpr int DV = D / 8;
   const int nf = p.r + p.m;
-  const int64_t total = static_cast<int64_t>(p.S) * nf * p.frame_vecs;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int vpr = p.H * D / 8;
-  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
-  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int64_t sf = i / p.frame_vecs;   // state * nf + frame
-    const int64_t e = i - sf * p.frame_vecs;
-    const int s = static_cast<int>(sf / nf);
-    const int fi = static_cast<int>(sf - static_cast<int64_t>(s) * nf);
-    const uint4* src;
-    uint4* dst;
-    if (fi < p.r) {
-      const int64_t off = (static_cast<int64_t>(s) * p.r + fi) * p.frame_vecs + e;
-      src = static_cast<const uint4*>(p.sink_src) + off;
-      dst = static_cast<uint4*>(p.sink_dst) + off;
-    } else {
-      int pos = p.pos0 + fi - p.r;
-      if (pos >= p.C) pos -= p.C;
-      const int64_t off = (static_cast<int64_t>(s) * p.C + pos) * p.frame_vecs + e;
-      src = static_cast<const uint4*>(p.mem_src) + off;
-      dst = static_cast<uint4*>(p.mem_dst) + off;
-    }
-    const uint4 x = __ldg(src);
-    const int tok = static_cast<int>(e / vpr);
-    const int c = static_cast<int>(e % (D / 8));
-    const int y = tok / p.grid_w, xx = tok - (tok / p.grid_w) * p.grid_w;
-    const dev::RopeRow rr{p.tables + static_cast<int64_t>(fi) * RC::UT, tab_h + y * RC::UH, tab_w + xx * RC::UW};
+  const int fv = static_cast<int>(p.frame_vecs);
+  const int s = blockIdx.y / nf;
+  const int fi = blockIdx.y - s * nf;
+  const uint4* src;
+  uint4* dst;
+  if (fi < p.r) {
+    const int64_t off = (static_cast<int64_t>(s) * p.r + fi) * fv;
+    src = static_cast<const uint4*>(p.sink_src) + off;
+    dst = static_cast<uint4*>(p.sink_dst) + off;
+  } else {
+    int pos = p.pos0 + fi - p.r;
+    if (pos >= p.C) pos -= p.C;
+    const int64_t off = (static_cast<int64_t>(s) * p.C + pos) * fv;
+    src = static_cast<const uint4*>(p.mem_src) + off;
+    dst = static_cast<uint4*>(p.mem_dst) + off;
+  }
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
+    const uint4 x = __ldg(src + e);
+    const int tok = p.div_heads.div(e / DV);
+    const dev::RopeRow rr = rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, fi, tok);
     uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    dev::rope_chunk<D, false>(w, c, rr, 1.0f);
-    *dst = make_uint4(w[0], w[1], w[2], w[3]);
+    dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
+    dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -137,24 +147,20 @@ __global__ void permute_weights_kernel(const __nv_bfloat16* __restrict__ src, __
 
 // Mean of the 5 evicted frames (the model card's --mean_memory option):
 // out = bf16(sum_j x_j / 5) with the sum and divide in fp32.
+// grid = (x, states, groups * 2 (K|V)).
 __global__ void mean_bf16_kernel(const uint4* __restrict__ ringK, const uint4* __restrict__ ringV,
                                  uint4* __restrict__ memK, uint4* __restrict__ memV, ConvParams p,
                                  int64_t frame_vecs) {
-  const int64_t per_group = static_cast<int64_t>(p.S) * frame_vecs * 2;
-  const int64_t total = per_group * p.ngroups;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int g = static_cast<int>(i / per_group);
-    int64_t r = i - g * per_group;
-    const int kv = static_cast<int>(r / (static_cast<int64_t>(p.S) * frame_vecs));
-    r -= static_cast<int64_t>(kv) * p.S * frame_vecs;
-    const int s = static_cast<int>(r / frame_vecs);
-    const int64_t e = r - static_cast<int64_t>(s) * frame_vecs;
-    const uint4* src = kv ? ringV : ringK;
+  const int fv = static_cast<int>(frame_vecs);
+  const int s = blockIdx.y;
+  const int g = blockIdx.z >> 1, kv = blockIdx.z & 1;
+  const uint4* src = kv ? ringV : ringK;
+  uint4* dst = (kv ? memV : memK) + (static_cast<int64_t>(s) * p.C + p.grp[g].mem_pos) * fv;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int j = 0; j < kEvict; ++j) {
-      const uint4 x = src[(static_cast<int64_t>(s) * p.R + p.grp[g].ring_slot[j]) * frame_vecs + e];
+      const uint4 x = src[(static_cast<int64_t>(s) * p.R + p.grp[g].ring_slot[j]) * fv + e];
       const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -168,8 +174,7 @@ __global__ void mean_bf16_kernel(const uint4* __restrict__ ringK, const uint4* _
       __nv_bfloat162 h2 = __floats2bfloat162_rn(__fdiv_rn(acc[2 * q], 5.0f), __fdiv_rn(acc[2 * q + 1], 5.0f));
       o[q] = *reinterpret_cast<uint32_t*>(&h2);
     }
-    uint4* dst = kv ? reinterpret_cast<uint4*>(p.memV) : reinterpret_cast<uint4*>(p.memK);
-    dst[(static_cast<int64_t>(s) * p.C + p.grp[g].mem_pos) * frame_vecs + e] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[e] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -267,44 +272,41 @@ __global__ void append_amax_kernel(const uint4* __restrict__ k, const uint4* __r
 // The block's K row chunk as written to staging: rotated at its stream position
 // (frame f of the block at time-table row t_row0 + f) when the tables are given --
 // the current block keeps its RoPE position relative to every later query, like
-// the pre-rotated ring of the bf16 format -- else as is.
+// the pre-rotated ring of the bf16 format -- else as is.  e: the vector's index in
+// its frame.
 template <int D>
-__device__ __forceinline__ uint4 staged_k(uint4 x, const AppendParams& p, int f, int64_t e) {
+__device__ __forceinline__ uint4 staged_k(uint4 x, const AppendParams& p, int f, int e) {
   if (!p.tables) return x;
-  using RC = RopeCfg<D>;
-  const int vpr = p.H * D / 8;
-  const int tok = static_cast<int>(e / vpr);
-  const int c = static_cast<int>(e % (D / 8));
-  const int y = tok / p.grid_w, xx = tok - (tok / p.grid_w) * p.grid_w;
-  const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
-  const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
-  const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.t_row0 + f) * RC::UT, tab_h + y * RC::UH,
-                        tab_w + xx * RC::UW};
+  constexpr int DV = D / 8;
+  const int tok = p.div_heads.div(e / DV);
+  const dev::RopeRow rr =
+      rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, p.t_row0 + f, tok);
   uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  dev::rope_chunk<D, false>(w, c, rr, 1.0f);
+  dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // pass 2: quantise into the ring, copy to staging (K rotated), record the scales.
+// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-byte vectors.
 template <int D>
 __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
-  const int64_t fv = p.frame_elems / 8;
-  const int64_t per_kv = static_cast<int64_t>(p.S) * p.b * fv;
-  const int64_t total = 2 * per_kv;
-  const int vec_per_row = p.H * p.D / 8;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int kv = static_cast<int>(i / per_kv);
-    const int64_t iv = i - kv * per_kv;       // vector index within [S][b*T][H][D]
-    const int64_t sf = iv / fv;               // s * b + f
-    const int64_t e = iv - sf * fv;
-    const int s = static_cast<int>(sf / p.b);
-    const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
-    const int h = static_cast<int>((e % vec_per_row) * 8 / p.D);
+  constexpr int DV = D / 8;
+  const int fv = static_cast<int>(p.frame_elems / 8);
+  const int sf = blockIdx.y;
+  const int s = sf / p.b;
+  const int f = sf - s * p.b;
+  const int kv = blockIdx.z;
+  int slot = p.slot0 + f;
+  if (slot >= p.R) slot -= p.R;
+  const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
+  uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
+  uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + (static_cast<int64_t>(s) * p.R + slot) * fv;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
+    const int hv = e / DV;                          // token * H + head
+    const int h = hv - p.div_heads.div(hv) * p.H;
     const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
-    reinterpret_cast<uint4*>(p.stage[kv])[(static_cast<int64_t>(s) * p.stage_frames + f) * fv + e] =
-        kv == 0 ? staged_k<D>(x, p, f, e) : x;
-    const float amax = __uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]);
+    stage[e] = kv == 0 ? staged_k<D>(x, p, f, e) : x;
+    const float amax = __uint_as_float(amax_f[h]);
     const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
     uint32_t o[2];
@@ -321,10 +323,8 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
             "f"(__fdiv_rn(__uint_as_float(w[2 * q + 1] << 16), scale)));
       o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
     }
-    int slot = p.slot0 + f;
-    if (slot >= p.R) slot -= p.R;
-    reinterpret_cast<uint2*>(p.ring8[kv])[(static_cast<int64_t>(s) * p.R + slot) * fv + e] = make_uint2(o[0], o[1]);
-    if (e < vec_per_row && (e * 8) % p.D == 0)  // first vector of head h in token 0 of the frame
+    codes[e] = make_uint2(o[0], o[1]);
+    if (hv < p.H && e % DV == 0)  // first vector of head h in token 0 of the frame
       p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
   }
 }
@@ -332,30 +332,31 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
 // NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
 // e2m1 codes into the ring, the bf16 values into staging (K rotated), the tensor
 // scale once.
+// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-channel blocks.
 template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
-  const int nb = p.D / fp4::kBlock;                           // blocks per token-head
-  const int64_t T = p.frame_elems / (static_cast<int64_t>(p.H) * p.D);
-  const int64_t per_frame = T * p.H * nb;
-  const int64_t per_kv = static_cast<int64_t>(p.S) * p.b * per_frame;
-  const int64_t fv = p.frame_elems / 8;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * per_kv; i += stride) {
-    const int kv = static_cast<int>(i / per_kv);
-    const int64_t ib = i - kv * per_kv;
-    const int64_t sf = ib / per_frame;                         // s * b + f
-    const int64_t rb = ib - sf * per_frame;                    // (token * H + h) * nb + blk
-    const int s = static_cast<int>(sf / p.b);
-    const int f = static_cast<int>(sf - static_cast<int64_t>(s) * p.b);
-    const int64_t th = rb / nb;                                // token * H + h
-    const int blk = static_cast<int>(rb - th * nb);
-    const int h = static_cast<int>(th % p.H);
-    const int64_t e0 = th * (p.D / 8) + blk * 2;               // first 16-byte vector of the block
+  constexpr int NB = D / fp4::kBlock;                      // blocks per token-head
+  const int fv = static_cast<int>(p.frame_elems / 8);
+  const int per_frame = static_cast<int>(p.frame_elems / fp4::kBlock);
+  const int sf = blockIdx.y;
+  const int s = sf / p.b;
+  const int f = sf - s * p.b;
+  const int kv = blockIdx.z;
+  int slot = p.slot0 + f;
+  if (slot >= p.R) slot -= p.R;
+  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * D));
+  const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
+  uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
+  const int64_t row0 = (static_cast<int64_t>(s) * p.R + slot) * T * p.H;   // first token-head row of the slot
+  for (int ib = blockIdx.x * blockDim.x + threadIdx.x; ib < per_frame; ib += gridDim.x * blockDim.x) {
+    const int th = ib / NB;                                    // token * H + h
+    const int blk = ib - th * NB;
+    const int h = th - p.div_heads.div(th) * p.H;
+    const int e0 = th * (D / 8) + blk * 2;                     // first 16-byte vector of the block
     const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
     const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
-    uint4* st = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv + e0;
-    st[0] = kv == 0 ? staged_k<D>(x0, p, f, e0) : x0;
-    st[1] = kv == 0 ? staged_k<D>(x1, p, f, e0 + 1) : x1;
+    stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, e0) : x0;
+    stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, e0 + 1) : x1;
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
     float xs[fp4::kBlock];
     float a_b = 0.0f;
@@ -365,14 +366,12 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
       xs[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
       a_b = fmaxf(a_b, fmaxf(fabsf(xs[2 * q]), fabsf(xs[2 * q + 1])));
     }
-    const float g = fp4::tensor_scale(__uint_as_float(p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h]));
+    const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
     float e_b;
     const uint32_t sc = fp4::block_scale(a_b, g, e_b);
-    int slot = p.slot0 + f;
-    if (slot >= p.R) slot -= p.R;
-    const int64_t row = (static_cast<int64_t>(s) * p.R + slot) * T * p.H + th;   // token-head row in the ring
-    reinterpret_cast<uint2*>(p.ring8[kv])[row * nb + blk] = fp4::encode_block(xs, e_b);
-    p.ring_bs[kv][row * nb + blk] = static_cast<uint8_t>(sc);
+    const int64_t row = row0 + th;                              // token-head row in the ring
+    reinterpret_cast<uint2*>(p.ring8[kv])[row * NB + blk] = fp4::encode_block(xs, e_b);
+    p.ring_bs[kv][row * NB + blk] = static_cast<uint8_t>(sc);
     if (th < p.H && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
   }
 }
@@ -381,18 +380,19 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
 
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
                        cudaStream_t s) {
-  const int64_t total = static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
   auto kern = p.D == 128 ? append_bf16_kernel<128> : append_bf16_kernel<64>;
-  kern<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
-                                            static_cast<uint4*>(ringK), static_cast<uint4*>(ringV), p);
+  dim3 grid(frame_grid_x(p.frame_elems / 8, p.S * p.b, 256), p.S * p.b);
+  kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(ringK),
+                            static_cast<uint4*>(ringV), p);
   return static_cast<int>(cudaGetLastError());
 }
 
 int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s) {
-  const int64_t total = static_cast<int64_t>(p.S) * (p.r + p.m) * p.frame_vecs;
-  if (total == 0) return 0;
+  const int frames = p.S * (p.r + p.m);
+  if (frames == 0) return 0;
   auto kern = D == 128 ? rotate_keys_kernel<128> : rotate_keys_kernel<64>;
-  kern<<<grid_for(total, 256), 256, 0, s>>>(p);
+  dim3 grid(frame_grid_x(p.frame_vecs, frames, 256), frames);
+  kern<<<grid, 256, 0, s>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -405,10 +405,10 @@ int launch_permute_weights(const void* src, void* dst, int S, int H, int D, cuda
 
 int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* ringV, cudaStream_t s) {
   const int64_t frame_vecs = static_cast<int64_t>(p.T) * p.H * D / 8;
-  const int64_t total = frame_vecs * p.S * 2 * p.ngroups;
-  mean_bf16_kernel<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(ringK),
-                                                        static_cast<const uint4*>(ringV), static_cast<uint4*>(p.memK),
-                                                        static_cast<uint4*>(p.memV), p, frame_vecs);
+  if (p.ngroups <= 0) return 0;
+  dim3 grid(frame_grid_x(frame_vecs, p.S * 2 * p.ngroups, 256), p.S, 2 * p.ngroups);
+  mean_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(ringK), static_cast<const uint4*>(ringV),
+                                        static_cast<uint4*>(p.memK), static_cast<uint4*>(p.memV), p, frame_vecs);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -431,14 +431,14 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   if (p.fp4) {
-    const int64_t blocks = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / fp4::kBlock);
     auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
-    kern<<<grid_for(blocks, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+    dim3 grid(frame_grid_x(p.frame_elems / fp4::kBlock, 2 * p.S * p.b, 256), p.S * p.b, 2);
+    kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
-  const int64_t total = 2 * static_cast<int64_t>(p.S) * p.b * (p.frame_elems / 8);
   auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
-  kern<<<grid_for(total, 256), 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+  dim3 grid(frame_grid_x(p.frame_elems / 8, 2 * p.S * p.b, 256), p.S * p.b, 2);
+  kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }
 
