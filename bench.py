@@ -406,7 +406,10 @@ def run_ours(args, w):
     value = total_flops / (total_ms * 1e-3) / 1e12
     att_avg_ms = statistics.mean(att_ms)
     att_achieved = statistics.mean(flops) / (att_avg_ms * 1e-3) / 1e12
-    peak = pk["bf16_tflops"]
+    # a kernel timed alone against the burst peak; one timed inside a seconds-long loop
+    # (the 40-state workloads) against the sustained one, reached under the power cap
+    sustained = total_ms > 1000.0
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
     kvb = kv_bytes_per_value(w)
     att_bytes = attention_bytes(b * T, statistics.mean(nk_list), D, H, S, kv_bytes=kvb,
                                 Nk_bf16=(b + r) * T if kvb < 2 else None)
@@ -419,7 +422,9 @@ def run_ours(args, w):
         ac_line = {"bytes_per_step": acb, "gbs": acb / (ac_ms * 1e-3) / 1e9,
                    "frac_of_hbm": acb / (ac_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                    "note": "event time between attends: append, conv groups, the time-table copy and launch gaps"}
-    kernel = {"bf16": "attn_kernel<128, 0>", "e4m3": "attn_kernel<128, 1>", "nvfp4": "attn_kernel<128, 2>"}[fmt]
+    kernel = ("attn_kernel<128>" if fmt == "bf16" else
+              "attn_kernel<128> with dequant_kernel<128> before it (the attend call: the e4m3 / NVFP4 "
+              "window and memory dequantised once per attend into a bf16 scratch)")
     dtype = {"bf16": "bf16", "e4m3": "bf16 compute, e4m3 K/V cache", "nvfp4": "bf16 compute, NVFP4 K/V cache"}[fmt]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -445,8 +450,11 @@ def run_ours(args, w):
         "roofline": {"bound": "tensor", "achieved": att_achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": att_achieved / peak, "traffic": traffic,
                      "algorithmic_bytes": att_bytes, "kernel": kernel,
-                     "peak_source": f"{kind} bf16 burst (MEASURED_PEAKS.json)" if kind == "measured"
-                                    else "fallback bf16 burst (1590 TF/s, earlier measurement on this pool)",
+                     "peak_source": (f"measured bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)"
+                                     if kind == "measured" else
+                                     f"fallback bf16 {'sustained (1400 TF/s' if sustained else 'burst (1590 TF/s'}, "
+                                     "earlier measurement on this pool; no MEASURED_PEAKS.json on the box)"),
+                     "frac_of_burst": att_achieved / pk["bf16_tflops"],
                      "traffic_source": traffic_src},
         "e2e": e2e_line,
         "gpu_launches": launches,
