@@ -703,39 +703,35 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   // every key segment is bf16 and stored rotated: the ring's rotated K (window and
   // current, bf16 format), the rotated memory and reference frames, the dequantised
   // scratch and the rotated staging of the current block (e4m3 / NVFP4 formats)
-  auto add = [&](int buf, int frame0, int nframes, int t0, int local) {
+  auto add = [&](int buf, int frame0, int nframes, int local) {
     KeySeg& s = ap.seg[ap.nseg++];
     s.buf = buf;
     s.row0 = frame0 * T;
     s.nrows = nframes * T;
-    s.t0 = t0;
-    s.tile0 = tiles;
-    s.prerot = 1;
     s.local = local;
     tiles += (s.nrows + 127) / 128;
   };
-  if (r > 0) add(3, 0, r, 0, 0);
+  if (r > 0) add(3, 0, r, 0);
   if (h->fp8) {
     // [memory | window] dequantised into the scratch in attend order, then the
     // current block's bf16 staging
-    if (m + w > 0) add(0, 0, m + w, r, 1);
-    add(2, 0, b, r + m + w, 0);
+    if (m + w > 0) add(0, 0, m + w, 1);
+    add(2, 0, b, 0);
   } else {
     if (m > 0) {
       const int pos0 = static_cast<int>((h->Sn - m) % h->C);
       const int n1 = m < h->C - pos0 ? m : h->C - pos0;
-      add(1, pos0, n1, r, 0);
-      if (m > n1) add(1, 0, m - n1, r + n1, 0);
+      add(1, pos0, n1, 0);
+      if (m > n1) add(1, 0, m - n1, 0);
     }
     // window and current block are consecutive ring frames
     const int n = w + b;
     const int start = static_cast<int>(h->E % h->R);
     const int n1 = n < h->R - start ? n : h->R - start;
-    if (n1 > 0) add(0, start, n1, r + m, 0);
-    if (n > n1) add(0, 0, n - n1, r + m + n1, 0);
+    if (n1 > 0) add(0, start, n1, 0);
+    if (n > n1) add(0, 0, n - n1, 0);
   }
   ap.ntiles = tiles;
-  ap.all_prerot = 1;
   ap.tab_t_rows = h->tab_t_rows;
   ap.tab_h_rows = h->gh;
   ap.tab_w_rows = h->gw;

@@ -39,15 +39,12 @@ struct FastDiv {
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
 
-// One contiguous run of key rows in one buffer (all bf16).
+// One contiguous run of key rows in one buffer (all bf16, K stored rotated).
 struct KeySeg {
   int buf;     // tensor map pair: 0 ring (bf16 format) or dequantised scratch (e4m3 / NVFP4),
                // 1 memory, 2 current-block staging (e4m3 / NVFP4), 3 reference frames
   int row0;    // first row (token) in that buffer, a frame boundary
   int nrows;   // rows = frames * T
-  int t0;      // RoPE time index of the segment's first frame
-  int tile0;   // index of the segment's first 128-row key tile in the attend's tile list
-  int prerot;  // 1 if the K rows are stored already rotated
   int local;   // 1 if the buffer holds only the launch's group of states (the scratch)
 };
 
@@ -87,7 +84,6 @@ struct AttnParams {
   __nv_bfloat16* out;     // [S][Nq][H][D]
   float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
   int state0;             // first state of the launch's group (grid z walks the group)
-  int all_prerot;         // every key segment is stored rotated: no RoPE work on K tiles
   int* status;
   // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
   // and written to the G ranks' shards (peer memory on a multi-GPU node)

@@ -7,10 +7,11 @@
 // with no mask inside that set (blog walk-through, "Neighbor Forcing":
 // block-wise causal mask; "ConvKV Memory": the four-partition context), the
 // RoPE time index reset to run 0.. over memory, window, current (press
-// article and aiboss88.com summary: RoPE Reset), and the cached K kept
-// un-rotated, so the rotation is applied here, on the fly, tile by tile.
+// article and aiboss88.com summary: RoPE Reset).  RoPE is relative, so keys are
+// rotated once at their stream positions (moving ones again when their reset
+// position moves) and only the queries are rotated here.
 //
-// CTA = one (state, head, 256 query rows) work unit, 16 warps:
+// CTA = one (state, head, 256 query rows) work unit, 12 warps:
 //   warp 0      TMA producer: Q (2 tiles of 128 rows), then K/V tiles of 128
 //               keys through 3 (K) and 2 (V) stage rings, per key segment
 //   warp 1      tcgen05.mma issuer and TMEM owner: S_i = Q_i K^T (SS form),
@@ -20,10 +21,10 @@
 //               thread per query row; online softmax in fp32 registers with a
 //               lazily rescaled running max (the O rescale is only done when
 //               the max grows by more than 2^8); P written back over S as bf16
-//   warps 12-15 RoPE of each landed K tile that is not stored rotated, in place
-//               in shared memory (cos/sin tables read through the read-only data
-//               cache); when every key arrives rotated (the usual case) they are
-//               idle and the MMA issuer takes K tiles straight from TMA
+// Every key arrives stored rotated (window and current keys by the append, memory
+// slots and reference frames by the rotation kernel whenever their positions move,
+// the low-precision window and memory by the dequantisation), so K tiles go from
+// TMA straight to the tensor cores; only the queries are rotated here.
 // Every operand is bf16.  The e4m3 / NVFP4 caches are dequantised (and their keys
 // rotated) once per attend into a bf16 scratch by kernels_dequant.cu, instead of by
 // each of the query-block CTAs that read a tile.  One launch covers a group of
@@ -51,13 +52,15 @@ struct AttnCfg {
   static constexpr int UT = RopeCfg<D>::UT, UH = RopeCfg<D>::UH, UW = RopeCfg<D>::UW;
   static constexpr int O_COL = 256;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 512;
-  // registers per thread after re-balancing: the block launches with 128 x 512;
-  // producer/MMA warpgroup + RoPE warpgroup + two softmax warpgroups must sum to it
-  static constexpr int REG_LAUNCH = 128, REG_CTRL = 96, REG_ROPE = 80, REG_SOFTMAX = 168;
-  static_assert(128 * REG_CTRL + 128 * REG_ROPE + 256 * REG_SOFTMAX == THREADS * REG_LAUNCH,
-                "register split must add up to the launch allocation");
-  static constexpr int NBARS = 1 + 1 + 3 * KST + 2 * VST + 3 * 2 + 1;
+  static constexpr int THREADS = 384;
+  // registers per thread after re-balancing: the block launches with 168 x 384 (the
+  // most 384 threads can have, 65536 / 384 rounded down to a multiple of 8); the
+  // producer/MMA warpgroup gives registers to the two softmax warpgroups, and the
+  // split must stay within the launch allocation or an increase waits forever
+  static constexpr int REG_LAUNCH = 168, REG_CTRL = 96, REG_SOFTMAX = 200;
+  static_assert(128 * REG_CTRL + 256 * REG_SOFTMAX <= THREADS * REG_LAUNCH,
+                "register split must fit the launch allocation");
+  static constexpr int NBARS = 1 + 1 + 2 * KST + 2 * VST + 3 * 2 + 1;
   static constexpr size_t FIXED =
       1024 + static_cast<size_t>(QT + KST + VST) * TILE + NBARS * 8 + 16 + kMaxSegs * sizeof(KeySeg);
 };
@@ -123,8 +126,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* q_ready = q_full + 1;
   uint64_t* k_full = q_ready + 1;        // [KST]
-  uint64_t* k_ready = k_full + C::KST;   // [KST]
-  uint64_t* k_empty = k_ready + C::KST;  // [KST]
+  uint64_t* k_empty = k_full + C::KST;   // [KST]
   uint64_t* v_full = k_empty + C::KST;   // [VST]
   uint64_t* v_empty = v_full + C::VST;   // [VST]
   uint64_t* s_full = v_empty + C::VST;   // [2]
@@ -150,7 +152,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     mbar_init(q_ready, 2 * C::BM);
     for (int i = 0; i < C::KST; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_ready[i], C::BN);
       mbar_init(&k_empty[i], 1);
     }
     for (int i = 0; i < C::VST; ++i) {
@@ -252,8 +253,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // K tiles that are all stored rotated go from TMA straight to the tensor cores
-      uint64_t* kr = p.all_prerot ? k_full : k_ready;
+      uint64_t* kr = k_full;  // K tiles arrive rotated: straight from TMA to the tensor cores
       do {
         if (!mbar_wait(q_ready, 0, abort_flag)) break;
         if (!mbar_wait(&kr[0], 0, abort_flag)) break;
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       }
     }
   }
-  } else if (warp < 12) {
+  } else {
     regs_inc<C::REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int i = (warp - 4) >> 2;
@@ -431,28 +431,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           for (int q = 0; q < 4; ++q) dst[c * 4 + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
-    }
-  } else {
-    regs_dec<C::REG_ROPE>();
-    // ------------------------------------------------------------ K RoPE
-    const int r = threadIdx.x - 384;
-    TileCursor cur;
-    for (int j = 0; j < (p.all_prerot ? 0 : p.ntiles); ++j, cur.next(seg)) {
-      const int ks = j % C::KST;
-      if (!mbar_wait(&k_full[ks], (j / C::KST) & 1, abort_flag)) break;
-      const KeySeg& sg = seg[cur.s];
-      const int lr = cur.jt * C::BN + r;
-      if (lr < sg.nrows && !sg.prerot) {
-        const int f = lr / p.T;
-        const int s = lr - f * p.T;
-        const int t = sg.t0 + f;
-        const int y = s / p.grid_w;
-        const int x = s - y * p.grid_w;
-        rope_row<D, false>(sK + ks * C::TILE, r, RopeRow{tab_t + t * C::UT, tab_h + y * C::UH, tab_w + x * C::UW},
-                           1.0f);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&k_ready[ks]);
     }
   }
 
