@@ -372,10 +372,17 @@ def run_ours(args, w):
     # end to end through the host-buffer entry points: pinned host q/k/v in, host out back, every step
     e2e_line = None
     if not args.no_e2e:
-        qh = pool[0][0].cpu().pin_memory()
-        kh = pool[0][1].cpu().pin_memory()
-        vh = pool[0][2].cpu().pin_memory()
-        oh = torch.empty_like(qh).pin_memory()
+        # pinned host buffers, filled straight from the device; with several ranks on one
+        # node, K and V share one buffer (the same bytes cross PCIe every step) so that
+        # eight 40-state replicas stay well inside the host's memory
+        def pinned_copy(x):
+            hbuf = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+            hbuf.copy_(x)
+            return hbuf
+        qh = pinned_copy(pool[0][0])
+        kh = pinned_copy(pool[0][1])
+        vh = kh if world > 1 else pinned_copy(pool[0][2])
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
         Ke = max(3, min(K, 10))
         for _ in range(2):
             h.append_host(kh, vh)

@@ -18,7 +18,6 @@
 #include "convkv_internal.h"
 #include "sm100.cuh"
 #include "nvfp4.cuh"
-#include "lowp_codes.cuh"
 
 namespace ckv {
 namespace {
@@ -223,7 +222,7 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 // ---------------------------------------------------------------------------
 // fp8 (e4m3) format.  The evicted frames are e4m3 with one fp32 scale per
 // (frame, head); the A operand's codes arrive by TMA and are dequantised to bf16
-// (x * scale) in shared memory by warps 6-9.  The slot is stored e4m3 with one scale
+// (x * scale) in shared memory by warps 6-13.  The slot is stored e4m3 with one scale
 // per (slot, head) = amax / 448 over the slot's [T, D] values, so the launch
 // runs twice: pass 1 only reduces amax (atomicMax on the fp32 bit pattern,
 // values are non-negative), pass 2 recomputes the same tiles and quantises
@@ -245,9 +244,9 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3(float lo, float hi) {
 
 // Low-precision A operand: the evicted frame's code tile (128 token rows of CB code
 // bytes of one head) is staged by TMA into the upper half of the A stage, with the
-// CB-byte swizzle, and expanded in place into the bf16 tile by warps 6-9 (one row
-// each).  For e4m3 at D = 128 a row's codes lie under its own output only; otherwise
-// the converting threads read their codes, meet at a barrier, then write.
+// CB-byte swizzle, and expanded in place into the bf16 tile by warps 6-13 (two
+// threads per row, half a row each; a row's output covers other rows' codes, so the
+// threads read all their codes and meet at a barrier before writing).
 template <int D, int FMT>
 struct LowpA {
   static constexpr int CB = FMT == 2 ? D / 2 : D;
@@ -255,7 +254,6 @@ struct LowpA {
   static constexpr int OFF = ConvCfg<D>::A_BYTES / 2;
   static constexpr int NCH = CB / 16;
   static constexpr uint32_t MASK = CB == 128 ? 7u : (CB == 64 ? 3u : 1u);
-  static constexpr bool SELF = FMT == 1 && D == 128;
 };
 
 __device__ __forceinline__ bool conv_bar_all(int id, int nthreads, bool v) {
@@ -274,7 +272,7 @@ __device__ __forceinline__ bool conv_bar_all(int id, int nthreads, bool v) {
 
 template <int D>
 struct LowpCfg {
-  static constexpr int THREADS = 320;  // producer, MMA, 4 epilogue warps, 4 converter warps
+  static constexpr int THREADS = 448;  // producer, MMA, 4 epilogue warps, 8 converter warps
 };
 
 // Persistent like the bf16 kernel: CTAs walk the units, the accumulator is double-
@@ -304,7 +302,7 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&a_ready[i], 128);
+      mbar_init(&a_ready[i], 256);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -399,8 +397,14 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
       }
     }
   } else if (warp >= 6) {
-    // warps 6..9: expand each staged code tile to bf16 rows (bf16(fp32(code * scale)))
-    const int r = threadIdx.x - 192;
+    // warps 6..13: expand each staged code tile to bf16 rows (bf16(fp32(code * scale))).
+    // Two threads per token row, one half of its channels each; all codes of the tile
+    // are read before any row is written (a row's output covers other threads' codes),
+    // and the barrier also carries a timeout anywhere in the group to all of it.
+    constexpr int HALF_CH = LA::NCH / 2;              // 16-byte code chunks per half row
+    constexpr int HALF_C = D / 16;                    // 8-channel output chunks per half row
+    const int t = threadIdx.x - 192;
+    const int r = t & 127, hf = t >> 7;
     int it = 0;
     bool live = true;
     for (int u = blockIdx.x; u < units && live; u += gridDim.x) {
@@ -415,50 +419,46 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
         const float sc = __ldg(&p.ring_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.R + slot) * p.H + cu.head]);
         const int64_t grow =
             (static_cast<int64_t>(cu.state) * p.R * p.T + static_cast<int64_t>(slot) * p.T + token) * p.H + cu.head;
-        uint4 raw[LA::NCH];
-        uint32_t bsw[D / 64 > 0 ? D / 64 : 1];
+        uint4 raw[HALF_CH];
+        uint32_t bsw = 0;
         if (ok) {
 #pragma unroll
-          for (int k = 0; k < LA::NCH; ++k) {
-            const uint32_t logical = static_cast<uint32_t>(r * LA::CB + k * 16);
+          for (int k = 0; k < HALF_CH; ++k) {
+            const uint32_t logical = static_cast<uint32_t>(r * LA::CB + (hf * HALF_CH + k) * 16);
             const uint32_t phys = logical ^ (((logical >> 7) & LA::MASK) << 4);
             raw[k] = valid ? *reinterpret_cast<const uint4*>(a + LA::OFF + phys) : make_uint4(0, 0, 0, 0);
           }
           if constexpr (FMT == 2) {
-            const uint32_t* bs = reinterpret_cast<const uint32_t*>(p.ring_bs[cu.kv] + grow * (D / 16));
+            // this half's D/32 block scales (4 bytes at D = 128, 2 at D = 64)
+            const uint8_t* bs = p.ring_bs[cu.kv] + grow * (D / 16) + hf * (D / 32);
 #pragma unroll
-            for (int k = 0; k < D / 64; ++k) bsw[k] = valid ? __ldg(bs + k) : 0u;
+            for (int k = 0; k < D / 32; ++k) bsw |= valid ? static_cast<uint32_t>(__ldg(bs + k)) << (8 * k) : 0u;
           }
         }
-        if constexpr (!LA::SELF) ok = conv_bar_all(1, 128, ok);
+        ok = conv_bar_all(1, 256, ok);
         if (!ok) {
           live = false;
           break;
         }
         uint8_t* rowp = a + r * 128;
         const int sw = r & 7;
-        // codes widened by moving bits to values times a power of two; the scale
-        // carries the inverse power (exact), or for a scale too large for that the
-        // power is multiplied out first (exact) and then the scale
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
+        for (int cc = 0; cc < HALF_C; ++cc) {
+          const int c = hf * HALF_C + cc;  // 8-channel chunk of the row
           uint32_t o[4];
           if constexpr (FMT == 2) {
-            const uint4 r4 = raw[c >> 2];
-            const uint32_t word = (c & 3) == 0 ? r4.x : ((c & 3) == 1 ? r4.y : ((c & 3) == 2 ? r4.z : r4.w));
-            const int b = c >> 1;
-            const float e_b = __fmul_rn(fp4::e4m3_to_f32(bsw[b >> 2] >> (8 * (b & 3))), sc);
-            if (e_b < kFp4FoldLimit) {
-              e2m1x8_to_bf16<true>(word, e_b * kTwo112, o);
-            } else {
-              e2m1x8_to_bf16<false>(word, e_b, o);
-            }
+            const uint4 r4 = raw[cc >> 2];
+            const uint32_t word = (cc & 3) == 0 ? r4.x : ((cc & 3) == 1 ? r4.y : ((cc & 3) == 2 ? r4.z : r4.w));
+            const float e_b = __fmul_rn(fp4::e4m3_to_f32(bsw >> (8 * (cc >> 1))), sc);
+            fp4::decode8(word, e_b, o);
           } else {
-            const uint4 r4 = raw[c >> 1];
-            if (sc < kE4m3FoldLimit) {
-              e4m3x8_to_bf16<true>((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, sc * kTwo120, o);
-            } else {
-              e4m3x8_to_bf16<false>((c & 1) ? r4.z : r4.x, (c & 1) ? r4.w : r4.y, sc, o);
+            const uint4 r4 = raw[cc >> 1];
+            const uint32_t w0 = (cc & 1) ? r4.z : r4.x, w1 = (cc & 1) ? r4.w : r4.y;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float x0, x1;
+              e4m3x2_to_f32_c(((q < 2 ? w0 : w1) >> (16 * (q & 1))) & 0xFFFFu, x0, x1);
+              o[q] = pack_bf16x2(x0 * sc, x1 * sc);
             }
           }
           *reinterpret_cast<uint4*>(rowp + (c >> 3) * (C::BM * 128) + (((c & 7) ^ sw) << 4)) =

@@ -186,87 +186,49 @@ __global__ void mean_bf16_kernel(const uint4* __restrict__ ringK, const uint4* _
 // The block's bf16 values are also copied to staging: the current block is
 // attended in bf16 and joins the window, e4m3, at the next append.
 
-// pass 1: amax.  grid = (row splits, frames, states * 2); each warp walks whole
-// rows (tokens) of its block's slice: lane l reads the row's 16-byte vectors l, l+32,
-// ..., so the warp's loads of one step are 512 contiguous bytes, and vector v belongs
-// to head v / (D/8) -- the same head for every row.  Each lane keeps one running max
-// per step in registers; at the end the lanes that share a head reduce by shuffles and
-// one of them does the atomicMax.  Rows wider than kAmaxSteps * 32 vectors take the
-// shared-memory kernel below.
-constexpr int kAmaxSteps = 32;
-
+// pass 1: amax.  grid = (x, states * b, 2 (K|V)): y is the frame, x walks its 16-byte
+// vectors a warp at a time (32 consecutive vectors, so each load step of a warp reads
+// 512 contiguous bytes).  The D/8 lanes that hold one head's vectors reduce by
+// shuffles and one of them updates the block's per-head maximum in shared memory;
+// the block then updates the frame's maxima in global memory once per head.
 template <int D>
-__global__ void append_amax_rows_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p,
-                                        int rows_per_block) {
-  constexpr int G = D / 8;  // lanes (vectors) per head within one step
-  const int f = blockIdx.y;
-  const int kv = blockIdx.z & 1, s = blockIdx.z >> 1;
-  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * D));
-  const int vpr = p.H * D / 8;
-  const int steps = (vpr + 31) / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  uint32_t m[kAmaxSteps];
+__global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
+  extern __shared__ unsigned int sh_max[];
+  constexpr int DV = D / 8;                       // lanes (vectors) per head
+  const int fv = static_cast<int>(p.frame_elems / 8);
+  const int sf = blockIdx.y;
+  const int s = sf / p.b;
+  const int f = sf - s * p.b;
+  const int kv = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  for (int h = threadIdx.x; h < p.H; h += blockDim.x) sh_max[h] = 0;
+  __syncthreads();
+  const int stride = gridDim.x * blockDim.x;
+  // warp-uniform loop: a frame's vector count is a multiple of DV, so a head's lanes
+  // are all inside the frame or all past its end
+  for (int base = blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < fv; base += stride) {
+    const int e = base + lane;
+    uint32_t m = 0;
+    if (e < fv) {
+      const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-  for (int j = 0; j < kAmaxSteps; ++j) m[j] = 0;
-  const int r0 = blockIdx.x * rows_per_block;
-  const int r1 = min(T, r0 + rows_per_block);
-  for (int r = r0 + warp; r < r1; r += nwarps) {
-    const int64_t e0 = static_cast<int64_t>(r) * vpr;
-#pragma unroll
-    for (int j = 0; j < kAmaxSteps; ++j) {
-      const int vi = lane + 32 * j;
-      if (j < steps && vi < vpr) {
-        const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + vi));
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          m[j] = max(m[j], (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
-          m[j] = max(m[j], w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
-        }
+      for (int q = 0; q < 4; ++q) {
+        m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
+        m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
       }
     }
-  }
 #pragma unroll
-  for (int j = 0; j < kAmaxSteps; ++j) {
-    if (j >= steps) break;
-    uint32_t x = m[j];
-#pragma unroll
-    for (int o = G / 2; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, o));
-    const int vi = lane + 32 * j;
-    if ((lane % G) == 0 && vi < vpr && x)
-      atomicMax(&p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + vi / G], x);
-  }
-}
-
-// pass 1 for rows of more than kAmaxSteps * 32 vectors: one block reduces a slice of
-// rows per head in shared memory, then one atomicMax per head.
-__global__ void append_amax_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p,
-                                   int rows_per_block) {
-  extern __shared__ unsigned int sh_amax[];
-  const int f = blockIdx.y;
-  const int kv = blockIdx.z & 1, s = blockIdx.z >> 1;
-  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-  for (int h = threadIdx.x; h < p.H; h += blockDim.x) sh_amax[h] = 0;
-  __syncthreads();
-  const int vec_per_row = p.H * p.D / 8;
-  const int r0 = blockIdx.x * rows_per_block;
-  const int r1 = min(T, r0 + rows_per_block);
-  for (int64_t i = static_cast<int64_t>(r0) * vec_per_row + threadIdx.x; i < static_cast<int64_t>(r1) * vec_per_row;
-       i += blockDim.x) {
-    const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, i));
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t m = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
-      m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
+    for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (e < fv && (lane % DV) == 0 && m) {
+      const int hv = e / DV;
+      atomicMax(&sh_max[hv - p.div_heads.div(hv) * p.H], m);
     }
-    const int h = static_cast<int>((i % vec_per_row) * 8 / p.D);
-    atomicMax(&sh_amax[h], m);
   }
   __syncthreads();
+  unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
   for (int h = threadIdx.x; h < p.H; h += blockDim.x)
-    if (sh_amax[h]) atomicMax(&p.amax[((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H + h], sh_amax[h]);
+    if (sh_max[h]) atomicMax(&amax_f[h], sh_max[h]);
 }
 
 // The block's K row chunk as written to staging: rotated at its stream position
@@ -415,18 +377,10 @@ int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* 
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(unsigned int) * p.S * 2 * p.b * p.H, s);
   if (e != cudaSuccess) return static_cast<int>(e);
-  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-  const int vpr = p.H * p.D / 8;
-  if (vpr <= kAmaxSteps * 32) {
-    const int rows_per_block = 128;
-    dim3 g1((T + rows_per_block - 1) / rows_per_block, p.b, p.S * 2);
-    auto kern = p.D == 128 ? append_amax_rows_kernel<128> : append_amax_rows_kernel<64>;
-    kern<<<g1, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p, rows_per_block);
-  } else {
-    const int rows_per_block = 64;
-    dim3 g1((T + rows_per_block - 1) / rows_per_block, p.b, p.S * 2);
-    append_amax_kernel<<<g1, 256, p.H * sizeof(unsigned int), s>>>(static_cast<const uint4*>(k),
-                                                                   static_cast<const uint4*>(v), p, rows_per_block);
+  {
+    auto kern = p.D == 128 ? append_amax_frames_kernel<128> : append_amax_frames_kernel<64>;
+    dim3 g1(frame_grid_x(p.frame_elems / 8, 2 * p.S * p.b, 256), p.S * p.b, 2);
+    kern<<<g1, 256, p.H * sizeof(unsigned int), s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
