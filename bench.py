@@ -36,7 +36,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0   # B200 dense bf16, for context beside the measured peak
 DEFAULT_WORKLOAD = "fp8_480x832"
 CSRC = os.path.join(ROOT, "compressed_kv_cache_convkv_b200", "csrc")
-ATTN_SOURCES = ("kernel_attn.cu", "sm100.cuh", "convkv_internal.h", "rope.cuh", "nvfp4.cuh")
+# sources of the attend call, per cache format: the attention kernel, and in the
+# e4m3 / NVFP4 formats the dequantisation that runs before it
+ATTN_SOURCES = ("kernel_attn.cu", "sm100.cuh", "convkv_internal.h", "rope.cuh")
+DEQUANT_SOURCES = ("kernels_dequant.cu", "lowp_codes.cuh", "nvfp4.cuh", "quant_div.cuh")
+
+
+def attend_sources(fmt: str):
+    return ATTN_SOURCES if fmt == "bf16" else ATTN_SOURCES + DEQUANT_SOURCES
 
 
 def peaks():
@@ -101,7 +108,7 @@ def measured_traffic(fmt: str, workload: str, algorithmic_bytes: float):
     if not os.path.exists(path):
         return None, None
     d = json.load(open(path))
-    if d.get("source_sha256") != source_sha(ATTN_SOURCES):
+    if d.get("source_sha256") != source_sha(attend_sources(fmt)):
         return None, os.path.relpath(path, ROOT) + " (stale: kernel changed since the capture)"
     return (float(d["dram_bytes_per_launch"]) / float(d["algorithmic_bytes_per_launch"]) * algorithmic_bytes,
             os.path.relpath(path, ROOT))

@@ -57,6 +57,7 @@ _SIGNATURES = {
     "convkv_quantize_e4m3_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_int, _P]),
     "convkv_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
+    "convkv_selftest_div_rn": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P]),
 }
 
 

@@ -18,6 +18,7 @@
 #include "convkv_internal.h"
 #include "sm100.cuh"
 #include "nvfp4.cuh"
+#include "quant_div.cuh"
 
 namespace ckv {
 namespace {
@@ -498,6 +499,7 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
         if (lane == 0 && mx > 0.0f) atomicMax(&p.amax[aidx], __float_as_uint(mx));
       } else if (FMT == 2) {
         const float gs = fp4::tensor_scale(__uint_as_float(p.amax[aidx]));
+        const SharedDivisor g6 = fp4::block_divisor(gs);
         const int64_t row = ((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head;
         uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) + row * (D / 2));
         uint8_t* bs = p.mem_bs[cu.kv] + row * (D / 16);
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
               a_b = fmaxf(a_b, fabsf(xs[e]));
             }
             float e_b;
-            const uint32_t sc = fp4::block_scale(a_b, gs, e_b);
+            const uint32_t sc = fp4::block_scale(a_b, gs, g6, e_b);
             const uint2 cw = fp4::encode_block(xs, e_b);
             if (valid) {
               dst[2 * c + hb] = cw;
@@ -529,6 +531,7 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
       } else {
         const float amax = __uint_as_float(p.amax[aidx]);
         const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        const SharedDivisor dv = make_divisor(scale);
         uint8_t* dst = static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) +
                        (((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head) * D;
 #pragma unroll
@@ -539,10 +542,10 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
           uint32_t w[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const uint32_t lo = f32x2_to_e4m3(__fdiv_rn(__uint_as_float(v[4 * e]), scale),
-                                              __fdiv_rn(__uint_as_float(v[4 * e + 1]), scale));
-            const uint32_t hi = f32x2_to_e4m3(__fdiv_rn(__uint_as_float(v[4 * e + 2]), scale),
-                                              __fdiv_rn(__uint_as_float(v[4 * e + 3]), scale));
+            const uint32_t lo = f32x2_to_e4m3(div_rn(__uint_as_float(v[4 * e]), dv),
+                                              div_rn(__uint_as_float(v[4 * e + 1]), dv));
+            const uint32_t hi = f32x2_to_e4m3(div_rn(__uint_as_float(v[4 * e + 2]), dv),
+                                              div_rn(__uint_as_float(v[4 * e + 3]), dv));
             w[e] = lo | (hi << 16);
           }
           if (valid) {

@@ -4,6 +4,7 @@
 // a multiple of the SM count.
 #include "convkv_internal.h"
 #include "nvfp4.cuh"
+#include "quant_div.cuh"
 #include "rope.cuh"
 
 namespace ckv {
@@ -118,13 +119,22 @@ __global__ void rotate_keys_kernel(RotateParams p) {
     src = static_cast<const uint4*>(p.mem_src) + off;
     dst = static_cast<uint4*>(p.mem_dst) + off;
   }
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
-    const uint4 x = __ldg(src + e);
-    const int tok = p.div_heads.div(e / DV);
-    const dev::RopeRow rr = rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, fi, tok);
-    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
-    dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+  constexpr int U = 2;                            // loads in flight per thread
+  const int stride = gridDim.x * blockDim.x;
+  for (int e0 = blockIdx.x * blockDim.x + threadIdx.x; e0 < fv; e0 += U * stride) {
+    uint4 xs[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) xs[u] = e0 + u * stride < fv ? __ldg(src + e0 + u * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * stride;
+      if (e >= fv) break;
+      const int tok = p.div_heads.div(e / DV);
+      const dev::RopeRow rr = rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, fi, tok);
+      uint32_t w[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+      dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
+      dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
@@ -204,25 +214,32 @@ __global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uin
   for (int h = threadIdx.x; h < p.H; h += blockDim.x) sh_max[h] = 0;
   __syncthreads();
   const int stride = gridDim.x * blockDim.x;
+  constexpr int U = 4;                            // loads in flight per thread
   // warp-uniform loop: a frame's vector count is a multiple of DV, so a head's lanes
   // are all inside the frame or all past its end
-  for (int base = blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < fv; base += stride) {
-    const int e = base + lane;
-    uint32_t m = 0;
-    if (e < fv) {
-      const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  for (int base = blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < fv; base += U * stride) {
+    uint4 x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = base + u * stride + lane;
+      x[u] = e < fv ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = base + u * stride + lane;
+      const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      uint32_t m = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
         m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
       }
-    }
 #pragma unroll
-    for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (e < fv && (lane % DV) == 0 && m) {
-      const int hv = e / DV;
-      atomicMax(&sh_max[hv - p.div_heads.div(hv) * p.H], m);
+      for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (e < fv && (lane % DV) == 0 && m) {
+        const int hv = e / DV;
+        atomicMax(&sh_max[hv - p.div_heads.div(hv) * p.H], m);
+      }
     }
   }
   __syncthreads();
@@ -263,31 +280,46 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
   const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + (static_cast<int64_t>(s) * p.R + slot) * fv;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
-    const int hv = e / DV;                          // token * H + head
-    const int h = hv - p.div_heads.div(hv) * p.H;
-    const uint4 x = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e));
-    stage[e] = kv == 0 ? staged_k<D>(x, p, f, e) : x;
-    const float amax = __uint_as_float(amax_f[h]);
-    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t o[2];
+  const SharedDivisor d448 = make_divisor(448.0f);
+  constexpr int U = 2;                            // loads in flight per thread
+  const int stride = gridDim.x * blockDim.x;
+  for (int e0 = blockIdx.x * blockDim.x + threadIdx.x; e0 < fv; e0 += U * stride) {
+    uint4 xs[U];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint16_t lo, hi;
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-          : "=h"(lo)
-          : "f"(__fdiv_rn(__uint_as_float(w[2 * q] & 0xFFFF0000u), scale)),
-            "f"(__fdiv_rn(__uint_as_float(w[2 * q] << 16), scale)));
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-          : "=h"(hi)
-          : "f"(__fdiv_rn(__uint_as_float(w[2 * q + 1] & 0xFFFF0000u), scale)),
-            "f"(__fdiv_rn(__uint_as_float(w[2 * q + 1] << 16), scale)));
-      o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * stride;
+      xs[u] = e < fv ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e)) : make_uint4(0, 0, 0, 0);
     }
-    codes[e] = make_uint2(o[0], o[1]);
-    if (hv < p.H && e % DV == 0)  // first vector of head h in token 0 of the frame
-      p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * stride;
+      if (e >= fv) break;
+      const int hv = e / DV;                      // token * H + head
+      const int h = hv - p.div_heads.div(hv) * p.H;
+      const uint4 x = xs[u];
+      stage[e] = kv == 0 ? staged_k<D>(x, p, f, e) : x;
+      const float amax = __uint_as_float(amax_f[h]);
+      const float scale = amax > 0.0f ? div_rn(amax, d448) : 1.0f;
+      const SharedDivisor ds = make_divisor(scale);
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t o[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint16_t lo, hi;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(lo)
+            : "f"(div_rn(__uint_as_float(w[2 * q] & 0xFFFF0000u), ds)),
+              "f"(div_rn(__uint_as_float(w[2 * q] << 16), ds)));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(hi)
+            : "f"(div_rn(__uint_as_float(w[2 * q + 1] & 0xFFFF0000u), ds)),
+              "f"(div_rn(__uint_as_float(w[2 * q + 1] << 16), ds)));
+        o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      }
+      codes[e] = make_uint2(o[0], o[1]);
+      if (hv < p.H && e % DV == 0)  // first vector of head h in token 0 of the frame
+        p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
+    }
   }
 }
 
@@ -330,7 +362,7 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
     }
     const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
     float e_b;
-    const uint32_t sc = fp4::block_scale(a_b, g, e_b);
+    const uint32_t sc = fp4::block_scale(a_b, g, fp4::block_divisor(g), e_b);
     const int64_t row = row0 + th;                              // token-head row in the ring
     reinterpret_cast<uint2*>(p.ring8[kv])[row * NB + blk] = fp4::encode_block(xs, e_b);
     p.ring_bs[kv][row * NB + blk] = static_cast<uint8_t>(sc);

@@ -38,38 +38,58 @@ __global__ void dequant_kernel(DequantParams p) {
   uint4* out = static_cast<uint4*>(p.out[kv]) + (static_cast<int64_t>(sl) * p.out_frames + fi) * fv;
   const float4* tab_h = p.tables + static_cast<int64_t>(p.tab_t_rows) * RC::UT;
   const float4* tab_w = tab_h + static_cast<int64_t>(p.tab_h_rows) * RC::UH;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
-    const int hv = e / DV;                       // token * H + head
-    const int c = e - hv * DV;                   // 8-channel chunk within the head
-    const int tok = p.div_heads.div(hv);
-    const int h = hv - tok * p.H;
-    const float sc = __ldg(scl + h);
-    uint32_t o[4];
-    if (p.fp4) {
-      const uint32_t word = __ldg(reinterpret_cast<const uint32_t*>(codes + frame * (p.frame_elems / 2)) + e);
-      const uint8_t sb = __ldg(bsb + frame * (p.frame_elems / 16) + static_cast<int64_t>(hv) * (D / 16) + (c >> 1));
-      const float e_b = __fmul_rn(fp4::e4m3_to_f32(sb), sc);
-      if (e_b < dev::kFp4FoldLimit) {
-        dev::e2m1x8_to_bf16<true>(word, e_b * dev::kTwo112, o);
+  constexpr int U = 4;                            // code loads in flight per thread
+  const int stride = gridDim.x * blockDim.x;
+  for (int e0 = blockIdx.x * blockDim.x + threadIdx.x; e0 < fv; e0 += U * stride) {
+    uint2 cw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * stride;
+      if (e >= fv) {
+        cw[u] = make_uint2(0, 0);
+      } else if (p.fp4) {
+        cw[u].x = __ldg(reinterpret_cast<const uint32_t*>(codes + frame * (p.frame_elems / 2)) + e);
+        cw[u].y = 0;
       } else {
-        dev::e2m1x8_to_bf16<false>(word, e_b, o);
-      }
-    } else {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes + frame * p.frame_elems) + e);
-      if (sc < dev::kE4m3FoldLimit) {
-        dev::e4m3x8_to_bf16<true>(w.x, w.y, sc * dev::kTwo120, o);
-      } else {
-        dev::e4m3x8_to_bf16<false>(w.x, w.y, sc, o);
+        cw[u] = __ldg(reinterpret_cast<const uint2*>(codes + frame * p.frame_elems) + e);
       }
     }
-    if (kv == 0) {
-      const int y = p.div_grid_w.div(tok);
-      const int x = tok - y * p.grid_w;
-      const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.r + fi) * RC::UT, tab_h + y * RC::UH,
-                            tab_w + x * RC::UW};
-      dev::rope_chunk<D, false>(o, c, rr, 1.0f);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * stride;
+      if (e >= fv) break;
+      const int hv = e / DV;                        // token * H + head
+      const int c = e - hv * DV;                    // 8-channel chunk within the head
+      const int tok = p.div_heads.div(hv);
+      const int h = hv - tok * p.H;
+      const float sc = __ldg(scl + h);
+      uint32_t o[4];
+      if (p.fp4) {
+        const uint32_t word = cw[u].x;
+        const uint8_t sb = __ldg(bsb + frame * (p.frame_elems / 16) + static_cast<int64_t>(hv) * (D / 16) + (c >> 1));
+        const float e_b = __fmul_rn(fp4::e4m3_to_f32(sb), sc);
+        if (e_b < dev::kFp4FoldLimit) {
+          dev::e2m1x8_to_bf16<true>(word, e_b * dev::kTwo112, o);
+        } else {
+          dev::e2m1x8_to_bf16<false>(word, e_b, o);
+        }
+      } else {
+        const uint2 w = cw[u];
+        if (sc < dev::kE4m3FoldLimit) {
+          dev::e4m3x8_to_bf16<true>(w.x, w.y, sc * dev::kTwo120, o);
+        } else {
+          dev::e4m3x8_to_bf16<false>(w.x, w.y, sc, o);
+        }
+      }
+      if (kv == 0) {
+        const int y = p.div_grid_w.div(tok);
+        const int x = tok - y * p.grid_w;
+        const dev::RopeRow rr{p.tables + static_cast<int64_t>(p.r + fi) * RC::UT, tab_h + y * RC::UH,
+                              tab_w + x * RC::UW};
+        dev::rope_chunk<D, false>(o, c, rr, 1.0f);
+      }
+      out[e] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    out[e] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

@@ -15,6 +15,7 @@
 #include <cuda_fp16.h>
 
 #include "convkv_internal.h"
+#include "quant_div.cuh"
 #include "sm100.cuh"
 
 namespace ckv {
@@ -53,19 +54,24 @@ __device__ __forceinline__ float tensor_scale(float amax) { return amax > 0.0f ?
 
 // Block scale code of a block with max |x| = a_b under tensor scale g, and the
 // effective scale e_b = s_b * g it stands for.
-__device__ __forceinline__ uint32_t block_scale(float a_b, float g, float& e_b) {
-  const uint32_t s = f32_to_e4m3(__fdiv_rn(a_b, __fmul_rn(g, 6.0f)));
+// g6 is the shared divisor g * 6 (rounded), built once per tensor scale.
+__device__ __forceinline__ uint32_t block_scale(float a_b, float g, const SharedDivisor& g6, float& e_b) {
+  const uint32_t s = f32_to_e4m3(div_rn(a_b, g6));
   e_b = __fmul_rn(e4m3_to_f32(s), g);
   return s;
 }
+__device__ __forceinline__ SharedDivisor block_divisor(float g) { return make_divisor(__fmul_rn(g, 6.0f)); }
 
 // 16 values of one block -> 8 code bytes (as two 32-bit words each holding 4 bytes)
 __device__ __forceinline__ uint2 encode_block(const float (&x)[kBlock], float e_b) {
   uint32_t w[2] = {0, 0};
+  if (e_b > 0.0f) {
+    const SharedDivisor d = make_divisor(e_b);
 #pragma unroll
-  for (int j = 0; j < kBlock / 2; ++j) {
-    const uint32_t b = e_b > 0.0f ? f32x2_to_e2m1(__fdiv_rn(x[2 * j], e_b), __fdiv_rn(x[2 * j + 1], e_b)) : 0u;
-    w[j >> 2] |= b << (8 * (j & 3));
+    for (int j = 0; j < kBlock / 2; ++j) {
+      const uint32_t b = f32x2_to_e2m1(div_rn(x[2 * j], d), div_rn(x[2 * j + 1], d));
+      w[j >> 2] |= b << (8 * (j & 3));
+    }
   }
   return make_uint2(w[0], w[1]);
 }

@@ -221,6 +221,16 @@ int64_t convkv_launch_count(const convkv_t* h);
  * stays usable.  Errors: INVALID_ARG, CUDA. */
 int convkv_selftest_wait_timeout(int* dev_status, long long budget_clocks, void* stream);
 
+/* Self-test of the quantisers' division (the e4m3 / NVFP4 codes are decided by
+ * fp32 quotients x / scale rounded to nearest, as the FP8 / FP4 cache formats of
+ * the SoulX-LiveAct model card store them): for each of the n pairs
+ * (dev_x[i], dev_s[i]) (DEVICE fp32 arrays, caller-owned) the kernels' shared-
+ * divisor quotient is compared bit for bit with CUDA's IEEE division, and the
+ * number of differing pairs is added to *dev_mismatches (DEVICE unsigned int,
+ * caller-owned).  Synchronises `stream`.  Errors: INVALID_ARG, CUDA. */
+int convkv_selftest_div_rn(const float* dev_x, const float* dev_s, int64_t n, unsigned int* dev_mismatches,
+                           void* stream);
+
 /* Failure injection for tests, on the host: the `step`-th launch step (0-based,
  * counted per call: conv, time-table upload, ring append; in dry-run handles the
  * steps are counted but not run) of the next append reports cudaErrorLaunchFailure

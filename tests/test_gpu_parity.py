@@ -68,6 +68,49 @@ def test_bounded_wait_reports_timeout_and_context_survives(torch):
     _run(torch, PRESETS["tiny"], max_blocks=5)
 
 
+def test_quantiser_division_matches_ieee(torch):
+    """The e4m3 / NVFP4 quantisers' shared-divisor quotient (two Markstein correction
+    steps after RN(x * RN(1/s))) equals CUDA's IEEE fp32 division bit for bit: random
+    pairs over the quantisers' ranges, divisors outside the fast path's range, zeros,
+    and quotients placed next to fp32 rounding midpoints."""
+    ckv = _ckv()
+    g = torch.Generator(device="cuda").manual_seed(11)
+    n = 1 << 23
+    dev = "cuda"
+
+    def rand(*shape, dtype=torch.float32):
+        return torch.rand(*shape, device=dev, generator=g, dtype=dtype)
+
+    def randint(lo, hi):
+        return torch.randint(lo, hi, (n,), device=dev, generator=g)
+
+    sets = []
+    # quotients up to 448 in magnitude over divisors 2^-70 .. 2^60 (below 2^-60: IEEE path)
+    s = ((rand(n) + 1) * torch.exp2(randint(-70, 60).float())).float()
+    x = ((rand(n, dtype=torch.float64) * 896 - 448) * s.double()).float()
+    sets.append((x, s))
+    # quotients within a few 2^-25 units of the last place of an fp32 rounding midpoint
+    m = randint(2 ** 23, 2 ** 24).double()
+    e = randint(-11, 9).double()
+    k = randint(-4, 5).double()
+    mid = (m + 0.5 + k * 2.0 ** -25) * torch.exp2(e - 23)
+    s = ((rand(n) + 1) * torch.exp2(randint(-40, 30).float())).float()
+    sets.append(((mid * s.double()).float(), s))
+    # arbitrary dividends, bf16-grid dividends, zeros of both signs
+    s = ((rand(n) + 1) * torch.exp2(randint(-20, 20).float())).float()
+    x = (torch.randn(n, device=dev, generator=g) * torch.exp2(randint(-30, 30).float())).bfloat16().float()
+    x[: n // 64] = 0.0
+    x[n // 64: n // 32] = -0.0
+    sets.append((x, s))
+    bad = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    for xs, ss in sets:
+        xs, ss = xs.contiguous(), ss.contiguous()
+        assert bool(torch.isfinite(xs).all()) and bool((ss > 0).all())
+        assert ckv.library().convkv_selftest_div_rn(xs.data_ptr(), ss.data_ptr(), n, bad.data_ptr(), stream) == 0
+    assert int(bad.item()) == 0
+
+
 def _run(torch, w: Workload, attend_blocks=None, rows=None, compress=0, t_offset=0, override=None,
          check_slots=True, ring_frames=None, max_blocks=None, collect=None, sharp=False, sink=0, heads=None):
     """Stream w through both sides; returns per-block error records.  sink > 0 gives both
