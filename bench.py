@@ -39,7 +39,7 @@ CSRC = os.path.join(ROOT, "compressed_kv_cache_convkv_b200", "csrc")
 # sources of the attend call, per cache format: the attention kernel, and in the
 # e4m3 / NVFP4 formats the dequantisation that runs before it
 ATTN_SOURCES = ("kernel_attn.cu", "sm100.cuh", "convkv_internal.h", "rope.cuh")
-DEQUANT_SOURCES = ("kernels_dequant.cu", "lowp_codes.cuh", "nvfp4.cuh", "quant_div.cuh")
+DEQUANT_SOURCES = ("kernels_dequant.cu", "lowp_codes.cuh", "nvfp4.cuh", "quant_div.cuh", "token_walk.h")
 
 
 def attend_sources(fmt: str):

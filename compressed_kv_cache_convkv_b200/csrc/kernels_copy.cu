@@ -6,8 +6,25 @@
 #include "nvfp4.cuh"
 #include "quant_div.cuh"
 #include "rope.cuh"
+#include "token_walk.h"
 
 namespace ckv {
+
+int token_slabs(int H, int D) { return (H * (D / 8) + kTokenThreads - 1) / kTokenThreads; }
+
+int token_grid_x(int T, int H, int D, int frames_yz) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int slabs = token_slabs(H, D);
+  // about two waves of 8 resident CTAs per SM
+  const int64_t ctas = static_cast<int64_t>(frames_yz) * slabs;
+  int64_t walkers = (2LL * sms * 8 + ctas - 1) / ctas;
+  if (walkers > T) walkers = T;
+  if (walkers < 1) walkers = 1;
+  return static_cast<int>(walkers * slabs);
+}
+
 namespace {
 
 // Blocks along x for a launch whose y (and z) dimensions cover `frames` frames of
@@ -98,10 +115,14 @@ __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __r
 // Rotated copies of the reference frames and memory slots for the current time table
 // (bit-identical to rotating them tile by tile in the attention: same table, same
 // rounding).
-// grid = (x, states * (r + m)): y is the frame, x walks its 16-byte vectors.
+// grid = (x, states * (r + m)): y is the frame; token walk (each thread owns one
+// (head, 8-channel chunk) column, CTAs stride over the frame's tokens).
 template <int D>
 __global__ void rotate_keys_kernel(RotateParams p) {
   constexpr int DV = D / 8;
+  constexpr int U = 2;                            // loads in flight per thread
+  const int HDV = p.H * DV;
+  const int T = static_cast<int>(p.frame_vecs / HDV);
   const int nf = p.r + p.m;
   const int fv = static_cast<int>(p.frame_vecs);
   const int s = blockIdx.y / nf;
@@ -119,21 +140,28 @@ __global__ void rotate_keys_kernel(RotateParams p) {
     src = static_cast<const uint4*>(p.mem_src) + off;
     dst = static_cast<uint4*>(p.mem_dst) + off;
   }
-  constexpr int U = 2;                            // loads in flight per thread
-  const int stride = gridDim.x * blockDim.x;
-  for (int e0 = blockIdx.x * blockDim.x + threadIdx.x; e0 < fv; e0 += U * stride) {
-    uint4 xs[U];
+  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
+  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  if (hc < HDV) {
+    const int c = hc % DV;
+    for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
+      uint4 xs[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) xs[u] = e0 + u * stride < fv ? __ldg(src + e0 + u * stride) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        xs[u] = tok < T ? __ldg(src + tok * HDV + hc) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = e0 + u * stride;
-      if (e >= fv) break;
-      const int tok = p.div_heads.div(e / DV);
-      const dev::RopeRow rr = rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, fi, tok);
-      uint32_t w[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
-      dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
-      dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        if (tok >= T) break;
+        const dev::RopeRow rr =
+            rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, fi, tok);
+        uint32_t w[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+        dev::rope_chunk<D, false>(w, c, rr, 1.0f);
+        dst[tok * HDV + hc] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
   }
 }
@@ -196,80 +224,77 @@ __global__ void mean_bf16_kernel(const uint4* __restrict__ ringK, const uint4* _
 // The block's bf16 values are also copied to staging: the current block is
 // attended in bf16 and joins the window, e4m3, at the next append.
 
-// pass 1: amax.  grid = (x, states * b, 2 (K|V)): y is the frame, x walks its 16-byte
-// vectors a warp at a time (32 consecutive vectors, so each load step of a warp reads
-// 512 contiguous bytes).  The D/8 lanes that hold one head's vectors reduce by
-// shuffles and one of them updates the block's per-head maximum in shared memory;
-// the block then updates the frame's maxima in global memory once per head.
+// pass 1: amax.  grid = (x, states * b, 2 (K|V)), token walk: each thread owns one
+// (head, 8-channel chunk) column and keeps the running max of |x| over the tokens its
+// CTA visits (a CTA's load step reads kTokenThreads * 16 contiguous bytes of a token);
+// the D/8 lanes of a head then reduce by shuffles and one of them updates the frame's
+// per-head maximum in global memory.
 template <int D>
 __global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
-  extern __shared__ unsigned int sh_max[];
   constexpr int DV = D / 8;                       // lanes (vectors) per head
-  const int fv = static_cast<int>(p.frame_elems / 8);
+  constexpr int U = 4;                            // loads in flight per thread
+  const int HDV = p.H * DV;
+  const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
   const int f = sf - s * p.b;
   const int kv = blockIdx.z;
   const int lane = threadIdx.x & 31;
-  for (int h = threadIdx.x; h < p.H; h += blockDim.x) sh_max[h] = 0;
-  __syncthreads();
-  const int stride = gridDim.x * blockDim.x;
-  constexpr int U = 4;                            // loads in flight per thread
-  // warp-uniform loop: a frame's vector count is a multiple of DV, so a head's lanes
-  // are all inside the frame or all past its end
-  for (int base = blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < fv; base += U * stride) {
-    uint4 x[U];
+  unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
+  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
+  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  uint32_t m = 0;
+  if (hc < HDV) {
+    for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
+      uint4 x[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = base + u * stride + lane;
-      x[u] = e < fv ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e)) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = base + u * stride + lane;
-      const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-      uint32_t m = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
-        m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        x[u] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + hc))
+                       : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (e < fv && (lane % DV) == 0 && m) {
-        const int hv = e / DV;
-        atomicMax(&sh_max[hv - p.div_heads.div(hv) * p.H], m);
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          m = max(m, (w[q] & 0x7FFFu) << 16);   // |lo| as fp32 bits
+          m = max(m, w[q] & 0x7FFF0000u);       // |hi| as fp32 bits
+        }
       }
     }
   }
-  __syncthreads();
-  unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
-  for (int h = threadIdx.x; h < p.H; h += blockDim.x)
-    if (sh_max[h]) atomicMax(&amax_f[h], sh_max[h]);
+  // heads start at multiples of DV columns, slabs at multiples of 32, and DV divides 32
+#pragma unroll
+  for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (hc < HDV && (lane % DV) == 0 && m) atomicMax(&amax_f[hc / DV], m);
 }
 
 // The block's K row chunk as written to staging: rotated at its stream position
 // (frame f of the block at time-table row t_row0 + f) when the tables are given --
 // the current block keeps its RoPE position relative to every later query, like
-// the pre-rotated ring of the bf16 format -- else as is.  e: the vector's index in
-// its frame.
+// the pre-rotated ring of the bf16 format -- else as is.  tok: the token within the
+// frame; c: the 8-channel chunk within the head.
 template <int D>
-__device__ __forceinline__ uint4 staged_k(uint4 x, const AppendParams& p, int f, int e) {
+__device__ __forceinline__ uint4 staged_k(uint4 x, const AppendParams& p, int f, int tok, int c) {
   if (!p.tables) return x;
-  constexpr int DV = D / 8;
-  const int tok = p.div_heads.div(e / DV);
   const dev::RopeRow rr =
       rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, p.t_row0 + f, tok);
   uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  dev::rope_chunk<D, false>(w, e % DV, rr, 1.0f);
+  dev::rope_chunk<D, false>(w, c, rr, 1.0f);
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // pass 2: quantise into the ring, copy to staging (K rotated), record the scales.
-// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-byte vectors.
+// grid = (x, states * b, 2 (K|V)), token walk: each thread owns one (head h, chunk c)
+// column, so the head's scale and its divisor are set up once per thread.
 template <int D>
 __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   constexpr int DV = D / 8;
+  constexpr int U = 2;                            // loads in flight per thread
+  const int HDV = p.H * DV;
+  const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int fv = static_cast<int>(p.frame_elems / 8);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
@@ -281,92 +306,120 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + (static_cast<int64_t>(s) * p.R + slot) * fv;
   const SharedDivisor d448 = make_divisor(448.0f);
-  constexpr int U = 2;                            // loads in flight per thread
-  const int stride = gridDim.x * blockDim.x;
-  for (int e0 = blockIdx.x * blockDim.x + threadIdx.x; e0 < fv; e0 += U * stride) {
-    uint4 xs[U];
+  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
+  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  if (hc < HDV) {
+    const int h = hc / DV;
+    const int c = hc - h * DV;
+    const float amax = __uint_as_float(amax_f[h]);
+    const float scale = amax > 0.0f ? div_rn(amax, d448) : 1.0f;
+    const SharedDivisor ds = make_divisor(scale);
+    if (walker == 0 && c == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
+    for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
+      uint4 xs[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = e0 + u * stride;
-      xs[u] = e < fv ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e)) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int e = e0 + u * stride;
-      if (e >= fv) break;
-      const int hv = e / DV;                      // token * H + head
-      const int h = hv - p.div_heads.div(hv) * p.H;
-      const uint4 x = xs[u];
-      stage[e] = kv == 0 ? staged_k<D>(x, p, f, e) : x;
-      const float amax = __uint_as_float(amax_f[h]);
-      const float scale = amax > 0.0f ? div_rn(amax, d448) : 1.0f;
-      const SharedDivisor ds = make_divisor(scale);
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      uint32_t o[2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint16_t lo, hi;
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-            : "=h"(lo)
-            : "f"(div_rn(__uint_as_float(w[2 * q] & 0xFFFF0000u), ds)),
-              "f"(div_rn(__uint_as_float(w[2 * q] << 16), ds)));
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-            : "=h"(hi)
-            : "f"(div_rn(__uint_as_float(w[2 * q + 1] & 0xFFFF0000u), ds)),
-              "f"(div_rn(__uint_as_float(w[2 * q + 1] << 16), ds)));
-        o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        xs[u] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + hc))
+                        : make_uint4(0, 0, 0, 0);
       }
-      codes[e] = make_uint2(o[0], o[1]);
-      if (hv < p.H && e % DV == 0)  // first vector of head h in token 0 of the frame
-        p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = scale;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        if (tok >= T) break;
+        const int e = tok * HDV + hc;
+        const uint4 x = xs[u];
+        stage[e] = kv == 0 ? staged_k<D>(x, p, f, tok, c) : x;
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint16_t lo, hi;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+              : "=h"(lo)
+              : "f"(div_rn(__uint_as_float(w[2 * q] & 0xFFFF0000u), ds)),
+                "f"(div_rn(__uint_as_float(w[2 * q] << 16), ds)));
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+              : "=h"(hi)
+              : "f"(div_rn(__uint_as_float(w[2 * q + 1] & 0xFFFF0000u), ds)),
+                "f"(div_rn(__uint_as_float(w[2 * q + 1] << 16), ds)));
+          o[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        }
+        codes[e] = make_uint2(o[0], o[1]);
+      }
     }
   }
 }
 
-// NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
-// e2m1 codes into the ring, the bf16 values into staging (K rotated), the tensor
-// scale once.
-// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-channel blocks.
+// NVFP4 pass 2: block scales, e2m1 codes into the ring, the bf16 values into staging
+// (K rotated), the tensor scale once.  grid = (x, states * b, 2 (K|V)), token walk:
+// each thread owns one (head, 8-channel chunk) column; the two threads of a 16-channel
+// block (adjacent lanes: heads and slabs start at even columns) share its maximum by
+// a shuffle.
 template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
+  constexpr int DV = D / 8;
   constexpr int NB = D / fp4::kBlock;                      // blocks per token-head
+  constexpr int U = 2;                                     // loads in flight per thread
+  const int HDV = p.H * DV;
+  const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int fv = static_cast<int>(p.frame_elems / 8);
-  const int per_frame = static_cast<int>(p.frame_elems / fp4::kBlock);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
   const int f = sf - s * p.b;
   const int kv = blockIdx.z;
   int slot = p.slot0 + f;
   if (slot >= p.R) slot -= p.R;
-  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * D));
   const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   const int64_t row0 = (static_cast<int64_t>(s) * p.R + slot) * T * p.H;   // first token-head row of the slot
-  for (int ib = blockIdx.x * blockDim.x + threadIdx.x; ib < per_frame; ib += gridDim.x * blockDim.x) {
-    const int th = ib / NB;                                    // token * H + h
-    const int blk = ib - th * NB;
-    const int h = th - p.div_heads.div(th) * p.H;
-    const int e0 = th * (D / 8) + blk * 2;                     // first 16-byte vector of the block
-    const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
-    const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
-    stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, e0) : x0;
-    stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, e0 + 1) : x1;
-    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    float xs[fp4::kBlock];
-    float a_b = 0.0f;
+  uint32_t* codes = reinterpret_cast<uint32_t*>(p.ring8[kv]) + row0 * DV;  // 4 bytes per 8 channels
+  uint8_t* bsc = p.ring_bs[kv] + row0 * NB;
+  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
+  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  const bool act = hc < HDV;
+  const int h = act ? hc / DV : 0;
+  const int c = hc - h * DV;
+  const float g = fp4::tensor_scale(__uint_as_float(act ? amax_f[h] : 0u));
+  const SharedDivisor g6 = fp4::block_divisor(g);
+  if (act && walker == 0 && c == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
+  // every lane runs every step (the block maximum is shuffled between lane pairs)
+  for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
+    uint4 xs[U];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      xs[2 * q] = __uint_as_float(w[q] << 16);
-      xs[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
-      a_b = fmaxf(a_b, fmaxf(fabsf(xs[2 * q]), fabsf(xs[2 * q + 1])));
+    for (int u = 0; u < U; ++u) {
+      const int tok = tok0 + u * walkers;
+      xs[u] = act && tok < T
+                  ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + hc))
+                  : make_uint4(0, 0, 0, 0);
     }
-    const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
-    float e_b;
-    const uint32_t sc = fp4::block_scale(a_b, g, fp4::block_divisor(g), e_b);
-    const int64_t row = row0 + th;                              // token-head row in the ring
-    reinterpret_cast<uint2*>(p.ring8[kv])[row * NB + blk] = fp4::encode_block(xs, e_b);
-    p.ring_bs[kv][row * NB + blk] = static_cast<uint8_t>(sc);
-    if (th < p.H && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int tok = tok0 + u * walkers;
+      if (tok >= T) break;
+      const int e = tok * HDV + hc;
+      const uint4 x = xs[u];
+      if (act) stage[e] = kv == 0 ? staged_k<D>(x, p, f, tok, c) : x;
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      float x8[fp4::kBlock / 2];
+      float a = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        x8[2 * q] = __uint_as_float(w[q] << 16);
+        x8[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+        a = fmaxf(a, fmaxf(fabsf(x8[2 * q]), fabsf(x8[2 * q + 1])));
+      }
+      const float a_b = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      float e_b;
+      const uint32_t sc = fp4::block_scale(a_b, g, g6, e_b);
+      const uint32_t word = fp4::encode_half(x8, e_b);
+      if (act) {
+        codes[e] = word;
+        if ((c & 1) == 0) bsc[(static_cast<int64_t>(tok) * p.H + h) * NB + (c >> 1)] = static_cast<uint8_t>(sc);
+      }
+    }
   }
 }
 
@@ -385,8 +438,9 @@ int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s) {
   const int frames = p.S * (p.r + p.m);
   if (frames == 0) return 0;
   auto kern = D == 128 ? rotate_keys_kernel<128> : rotate_keys_kernel<64>;
-  dim3 grid(frame_grid_x(p.frame_vecs, frames, 256), frames);
-  kern<<<grid, 256, 0, s>>>(p);
+  const int T = static_cast<int>(p.frame_vecs / (static_cast<int64_t>(p.H) * (D / 8)));
+  dim3 grid(token_grid_x(T, p.H, D, frames), frames);
+  kern<<<grid, kTokenThreads, 0, s>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -411,20 +465,23 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   if (e != cudaSuccess) return static_cast<int>(e);
   {
     auto kern = p.D == 128 ? append_amax_frames_kernel<128> : append_amax_frames_kernel<64>;
-    dim3 g1(frame_grid_x(p.frame_elems / 8, 2 * p.S * p.b, 256), p.S * p.b, 2);
-    kern<<<g1, 256, p.H * sizeof(unsigned int), s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+    const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
+    dim3 g1(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+    kern<<<g1, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   if (p.fp4) {
     auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
-    dim3 grid(frame_grid_x(p.frame_elems / fp4::kBlock, 2 * p.S * p.b, 256), p.S * p.b, 2);
-    kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+    const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
+    dim3 grid(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+    kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
   auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
-  dim3 grid(frame_grid_x(p.frame_elems / 8, 2 * p.S * p.b, 256), p.S * p.b, 2);
-  kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
+  dim3 grid(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+  kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }
 
