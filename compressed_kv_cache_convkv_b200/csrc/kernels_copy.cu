@@ -10,13 +10,11 @@
 
 namespace ckv {
 
-int token_slabs(int H, int D) { return (H * (D / 8) + kTokenThreads - 1) / kTokenThreads; }
-
-int token_grid_x(int T, int H, int D, int frames_yz) {
+int token_grid_x(int T, int cols, int frames_yz) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int slabs = token_slabs(H, D);
+  const int slabs = (cols + kTokenThreads - 1) / kTokenThreads;
   // about two waves of 8 resident CTAs per SM
   const int64_t ctas = static_cast<int64_t>(frames_yz) * slabs;
   int64_t walkers = (2LL * sms * 8 + ctas - 1) / ctas;
@@ -354,15 +352,15 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
 
 // NVFP4 pass 2: block scales, e2m1 codes into the ring, the bf16 values into staging
 // (K rotated), the tensor scale once.  grid = (x, states * b, 2 (K|V)), token walk:
-// each thread owns one (head, 8-channel chunk) column; the two threads of a 16-channel
-// block (adjacent lanes: heads and slabs start at even columns) share its maximum by
-// a shuffle.
+// each thread owns one (head, 16-channel block) column, so the head's tensor scale and
+// its divisor are set up once per thread.
 template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   constexpr int DV = D / 8;
   constexpr int NB = D / fp4::kBlock;                      // blocks per token-head
-  constexpr int U = 2;                                     // loads in flight per thread
+  constexpr int U = 2;                                     // tokens in flight per thread
   const int HDV = p.H * DV;
+  const int HNB = p.H * NB;
   const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int fv = static_cast<int>(p.frame_elems / 8);
   const int sf = blockIdx.y;
@@ -374,50 +372,50 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
   const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   const int64_t row0 = (static_cast<int64_t>(s) * p.R + slot) * T * p.H;   // first token-head row of the slot
-  uint32_t* codes = reinterpret_cast<uint32_t*>(p.ring8[kv]) + row0 * DV;  // 4 bytes per 8 channels
+  uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + row0 * NB;        // 8 bytes per block
   uint8_t* bsc = p.ring_bs[kv] + row0 * NB;
-  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int slabs = (HNB + blockDim.x - 1) / blockDim.x;
   const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
-  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
-  const bool act = hc < HDV;
-  const int h = act ? hc / DV : 0;
-  const int c = hc - h * DV;
-  const float g = fp4::tensor_scale(__uint_as_float(act ? amax_f[h] : 0u));
-  const SharedDivisor g6 = fp4::block_divisor(g);
-  if (act && walker == 0 && c == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
-  // every lane runs every step (the block maximum is shuffled between lane pairs)
-  for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
-    uint4 xs[U];
+  const int hb = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  if (hb < HNB) {
+    const int h = hb / NB;
+    const int blk = hb - h * NB;
+    const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
+    const SharedDivisor g6 = fp4::block_divisor(g);
+    if (walker == 0 && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
+    for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
+      uint4 xs[U][2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int tok = tok0 + u * walkers;
-      xs[u] = act && tok < T
-                  ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + hc))
-                  : make_uint4(0, 0, 0, 0);
-    }
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        const int64_t e0 = static_cast<int64_t>(tok) * HDV + 2 * hb;       // first 16-byte vector of the block
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int tok = tok0 + u * walkers;
-      if (tok >= T) break;
-      const int e = tok * HDV + hc;
-      const uint4 x = xs[u];
-      if (act) stage[e] = kv == 0 ? staged_k<D>(x, p, f, tok, c) : x;
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      float x8[fp4::kBlock / 2];
-      float a = 0.0f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        x8[2 * q] = __uint_as_float(w[q] << 16);
-        x8[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
-        a = fmaxf(a, fmaxf(fabsf(x8[2 * q]), fabsf(x8[2 * q + 1])));
+        for (int j = 0; j < 2; ++j)
+          xs[u][j] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + j))
+                             : make_uint4(0, 0, 0, 0);
       }
-      const float a_b = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-      float e_b;
-      const uint32_t sc = fp4::block_scale(a_b, g, g6, e_b);
-      const uint32_t word = fp4::encode_half(x8, e_b);
-      if (act) {
-        codes[e] = word;
-        if ((c & 1) == 0) bsc[(static_cast<int64_t>(tok) * p.H + h) * NB + (c >> 1)] = static_cast<uint8_t>(sc);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int tok = tok0 + u * walkers;
+        if (tok >= T) break;
+        const int e0 = tok * HDV + 2 * hb;
+        const uint4 x0 = xs[u][0], x1 = xs[u][1];
+        stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, tok, 2 * blk) : x0;
+        stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, tok, 2 * blk + 1) : x1;
+        const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float x16[fp4::kBlock];
+        float a_b = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          x16[2 * q] = __uint_as_float(w[q] << 16);
+          x16[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+          a_b = fmaxf(a_b, fmaxf(fabsf(x16[2 * q]), fabsf(x16[2 * q + 1])));
+        }
+        float e_b;
+        const uint32_t sc = fp4::block_scale(a_b, g, g6, e_b);
+        const int64_t row = static_cast<int64_t>(tok) * p.H + h;          // token-head row within the slot
+        codes[row * NB + blk] = fp4::encode_block(x16, e_b);
+        bsc[row * NB + blk] = static_cast<uint8_t>(sc);
       }
     }
   }
@@ -439,7 +437,7 @@ int launch_rotate_keys(int D, const RotateParams& p, cudaStream_t s) {
   if (frames == 0) return 0;
   auto kern = D == 128 ? rotate_keys_kernel<128> : rotate_keys_kernel<64>;
   const int T = static_cast<int>(p.frame_vecs / (static_cast<int64_t>(p.H) * (D / 8)));
-  dim3 grid(token_grid_x(T, p.H, D, frames), frames);
+  dim3 grid(token_grid_x(T, p.H * (D / 8), frames), frames);
   kern<<<grid, kTokenThreads, 0, s>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
@@ -466,7 +464,7 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   {
     auto kern = p.D == 128 ? append_amax_frames_kernel<128> : append_amax_frames_kernel<64>;
     const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-    dim3 g1(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+    dim3 g1(token_grid_x(T, p.H * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
     kern<<<g1, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   }
   e = cudaGetLastError();
@@ -474,13 +472,13 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   if (p.fp4) {
     auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
     const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-    dim3 grid(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+    dim3 grid(token_grid_x(T, p.H * (p.D / fp4::kBlock), 2 * p.S * p.b), p.S * p.b, 2);
     kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
   auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
   const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-  dim3 grid(token_grid_x(T, p.H, p.D, 2 * p.S * p.b), p.S * p.b, 2);
+  dim3 grid(token_grid_x(T, p.H * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
   kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }

@@ -106,7 +106,7 @@ int launch_dequant(int D, const DequantParams& p, int states, cudaStream_t s) {
   if (frames == 0) return 0;
   if (frames > 65535) return static_cast<int>(cudaErrorInvalidValue);
   const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * D));
-  dim3 grid(token_grid_x(T, p.H, D, 2 * frames), frames, 2);
+  dim3 grid(token_grid_x(T, p.H * (D / 8), 2 * frames), frames, 2);
   if (D == 128) {
     dequant_kernel<128><<<grid, kTokenThreads, 0, s>>>(p);
   } else if (D == 64) {

@@ -76,18 +76,6 @@ __device__ __forceinline__ uint2 encode_block(const float (&x)[kBlock], float e_
   return make_uint2(w[0], w[1]);
 }
 
-// 8 values (half a block) -> 4 code bytes (channel pairs in order, even channel in the
-// low nibble), the layout of one half of encode_block's output
-__device__ __forceinline__ uint32_t encode_half(const float (&x)[kBlock / 2], float e_b) {
-  uint32_t w = 0;
-  if (e_b > 0.0f) {
-    const SharedDivisor d = make_divisor(e_b);
-#pragma unroll
-    for (int j = 0; j < kBlock / 4; ++j) w |= f32x2_to_e2m1(div_rn(x[2 * j], d), div_rn(x[2 * j + 1], d)) << (8 * j);
-  }
-  return w;
-}
-
 // 4 code bytes (8 channels) -> 4 bf16x2 words of code * e_b
 __device__ __forceinline__ void decode8(uint32_t word, float e_b, uint32_t (&o)[4]) {
 #pragma unroll

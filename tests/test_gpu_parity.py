@@ -464,3 +464,21 @@ def test_nvfp4_480x832_outliers(torch):
     w = replace(PRESETS["nvfp4_480x832"], num_states=2)
     _run_fp8(torch, w, states=(0, 1), rows=128, ring_frames=[0, 7], heads={0: (0, 39), 1: (20,)}, outliers=True,
              max_blocks=5)
+
+
+# -- odd head counts: the streaming kernels' (head, chunk) columns split into 128-thread
+# slabs end inside a warp (9 heads x 16 chunks = 144 columns: a second slab of 16) ----
+
+ODD_HEADS = Workload("odd_heads", 9, 128, 3, 7, 2, 2, 4, 3, 24, seed=9)
+
+
+def test_odd_heads_stream(torch):
+    _run(torch, ODD_HEADS)
+
+
+def test_odd_heads_fp8_two_states(torch):
+    _run_fp8(torch, replace(ODD_HEADS, fp8=True, num_states=2, name="odd_heads_fp8"), states=(0, 1))
+
+
+def test_odd_heads_nvfp4_two_states(torch):
+    _run_fp8(torch, replace(ODD_HEADS, fp4=True, num_states=2, name="odd_heads_nvfp4"), states=(0, 1))
