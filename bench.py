@@ -174,7 +174,7 @@ class OracleSample:
 SAMPLE_HEADS = (0, 5, 11, 17, 22, 28, 33, 39)
 
 
-def cpu_baseline(w, rows: int = 2048):
+def cpu_baseline(w, rows: int = 4096):
     sample = OracleSample(w, [h for h in SAMPLE_HEADS if h < w.heads])
     dt, flops = sample.time(rows, 0)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",

@@ -350,74 +350,51 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
   }
 }
 
-// NVFP4 pass 2: block scales, e2m1 codes into the ring, the bf16 values into staging
-// (K rotated), the tensor scale once.  grid = (x, states * b, 2 (K|V)), token walk:
-// each thread owns one (head, 16-channel block) column, so the head's tensor scale and
-// its divisor are set up once per thread.
+// NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
+// e2m1 codes into the ring, the bf16 values into staging (K rotated), the tensor
+// scale once.
+// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-channel blocks.
 template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
-  constexpr int DV = D / 8;
   constexpr int NB = D / fp4::kBlock;                      // blocks per token-head
-  constexpr int U = 2;                                     // tokens in flight per thread
-  const int HDV = p.H * DV;
-  const int HNB = p.H * NB;
-  const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int fv = static_cast<int>(p.frame_elems / 8);
+  const int per_frame = static_cast<int>(p.frame_elems / fp4::kBlock);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
   const int f = sf - s * p.b;
   const int kv = blockIdx.z;
   int slot = p.slot0 + f;
   if (slot >= p.R) slot -= p.R;
+  const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * D));
   const unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   const int64_t row0 = (static_cast<int64_t>(s) * p.R + slot) * T * p.H;   // first token-head row of the slot
-  uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + row0 * NB;        // 8 bytes per block
-  uint8_t* bsc = p.ring_bs[kv] + row0 * NB;
-  const int slabs = (HNB + blockDim.x - 1) / blockDim.x;
-  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
-  const int hb = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
-  if (hb < HNB) {
-    const int h = hb / NB;
-    const int blk = hb - h * NB;
-    const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
-    const SharedDivisor g6 = fp4::block_divisor(g);
-    if (walker == 0 && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
-    for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
-      uint4 xs[U][2];
+  for (int ib = blockIdx.x * blockDim.x + threadIdx.x; ib < per_frame; ib += gridDim.x * blockDim.x) {
+    const int th = ib / NB;                                    // token * H + h
+    const int blk = ib - th * NB;
+    const int h = th - p.div_heads.div(th) * p.H;
+    const int e0 = th * (D / 8) + blk * 2;                     // first 16-byte vector of the block
+    const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
+    const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
+    const int tok = p.div_heads.div(th);
+    stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, tok, 2 * blk) : x0;
+    stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, tok, 2 * blk + 1) : x1;
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float xs[fp4::kBlock];
+    float a_b = 0.0f;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tok = tok0 + u * walkers;
-        const int64_t e0 = static_cast<int64_t>(tok) * HDV + 2 * hb;       // first 16-byte vector of the block
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-          xs[u][j] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + j))
-                             : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tok = tok0 + u * walkers;
-        if (tok >= T) break;
-        const int e0 = tok * HDV + 2 * hb;
-        const uint4 x0 = xs[u][0], x1 = xs[u][1];
-        stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, tok, 2 * blk) : x0;
-        stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, tok, 2 * blk + 1) : x1;
-        const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        float x16[fp4::kBlock];
-        float a_b = 0.0f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          x16[2 * q] = __uint_as_float(w[q] << 16);
-          x16[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
-          a_b = fmaxf(a_b, fmaxf(fabsf(x16[2 * q]), fabsf(x16[2 * q + 1])));
-        }
-        float e_b;
-        const uint32_t sc = fp4::block_scale(a_b, g, g6, e_b);
-        const int64_t row = static_cast<int64_t>(tok) * p.H + h;          // token-head row within the slot
-        codes[row * NB + blk] = fp4::encode_block(x16, e_b);
-        bsc[row * NB + blk] = static_cast<uint8_t>(sc);
-      }
+    for (int q = 0; q < 8; ++q) {
+      xs[2 * q] = __uint_as_float(w[q] << 16);
+      xs[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+      a_b = fmaxf(a_b, fmaxf(fabsf(xs[2 * q]), fabsf(xs[2 * q + 1])));
     }
+    const float g = fp4::tensor_scale(__uint_as_float(amax_f[h]));
+    float e_b;
+    const uint32_t sc = fp4::block_scale(a_b, g, fp4::block_divisor(g), e_b);
+    const int64_t row = row0 + th;                              // token-head row in the ring
+    reinterpret_cast<uint2*>(p.ring8[kv])[row * NB + blk] = fp4::encode_block(xs, e_b);
+    p.ring_bs[kv][row * NB + blk] = static_cast<uint8_t>(sc);
+    if (th < p.H && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
   }
 }
 
@@ -471,9 +448,8 @@ int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaS
   if (e != cudaSuccess) return static_cast<int>(e);
   if (p.fp4) {
     auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
-    const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-    dim3 grid(token_grid_x(T, p.H * (p.D / fp4::kBlock), 2 * p.S * p.b), p.S * p.b, 2);
-    kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
+    dim3 grid(frame_grid_x(p.frame_elems / fp4::kBlock, 2 * p.S * p.b, 256), p.S * p.b, 2);
+    kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
   auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
