@@ -88,6 +88,13 @@ struct convkv {
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
+  // host I/O (CONVKV_FLAG_HOST_IO): the *_host entry points copy by chunks of io_chunk
+  // states on their own streams, and each chunk's kernels wait only for that chunk's
+  // copy, so copies in both directions overlap the kernels of other chunks
+  cudaStream_t io_in = nullptr, io_back = nullptr;
+  std::vector<cudaEvent_t> io_ev;  // [0] start, [1 + c] chunk c copied in, [1 + nchunks + c] chunk c done
+  int io_chunk = 0, io_nchunks = 0;
+  bool io_pending = false;         // the next ring append reads io_k / io_v chunk by chunk
   CUtensorMap mapRingK{}, mapRingV{}, mapRingKr{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
       mapSinkV{};
   // e4m3 / NVFP4: code tiles of the ring (read by the conv), and the bf16 scratch the
@@ -270,6 +277,33 @@ const char* convkv_strerror(int code) {
   }
 }
 
+// Copy streams and events of the host-buffer entry points.  Chunks follow the
+// attention's state groups in the low-precision formats (a group's attention waits
+// for its queries only), and split the states eight ways in the bf16 format.
+static int create_host_io(convkv_t* h) {
+  h->io_chunk = h->fp8 ? h->Sg : (h->S + 7) / 8;
+  if (h->io_chunk < 1) h->io_chunk = 1;
+  h->io_nchunks = (h->S + h->io_chunk - 1) / h->io_chunk;
+  if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)
+    return CONVKV_ERR_CUDA;
+  h->io_ev.assign(1 + 2 * h->io_nchunks, nullptr);
+  for (auto& ev : h->io_ev)
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return CONVKV_ERR_CUDA;
+  return CONVKV_OK;
+}
+
+static void release_host_io(convkv_t* h) {
+  if (h->io_in) cudaStreamSynchronize(h->io_in);
+  if (h->io_back) cudaStreamSynchronize(h->io_back);
+  for (auto& ev : h->io_ev)
+    if (ev) cudaEventDestroy(ev);
+  h->io_ev.clear();
+  if (h->io_in) cudaStreamDestroy(h->io_in);
+  if (h->io_back) cudaStreamDestroy(h->io_back);
+  h->io_in = h->io_back = nullptr;
+}
+
 int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   if (!out) return CONVKV_ERR_INVALID_ARG;
   *out = nullptr;
@@ -430,7 +464,9 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   if (!rc && h->Rs) rc = encode_4d(&h->mapSinkK, h->sinkK, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && h->Rs) rc = encode_4d(&h->mapSinkV, h->sinkV, h->D, h->H, static_cast<int64_t>(h->Rs) * h->T, h->S);
   if (!rc && w_b) rc = encode_weights(&h->mapW, h->weights, h->D, h->H, h->S);
+  if (!rc && h->host_io) rc = create_host_io(h);
   if (rc) {
+    release_host_io(h);
     cudaFree(h->arena);
     delete h;
     return rc;
@@ -448,6 +484,7 @@ void convkv_destroy(convkv_t* h) {
   if (!h) return;
   if (h->arena) {
     cudaStreamSynchronize(h->stream);
+    release_host_io(h);
     cudaFree(h->arena);
   }
   delete h;
@@ -491,6 +528,31 @@ static int rotate_moving_keys(convkv_t* h, int64_t B0) {
 
 // The steps of one append.  Advances the counters first (the launches read the new
 // ones); append_impl restores them when a step fails.
+// The ring append's parameters for states [g0, g0 + n): every per-state buffer moves
+// by g0 states (the kernels index states from 0).
+static AppendParams states_slice(const convkv_t* h, const AppendParams& a, int g0, int n, int frames) {
+  if (g0 == 0 && n == a.S) return a;
+  AppendParams p = a;
+  p.S = n;
+  const int64_t fe = h->frame_elems();
+  const int64_t g = g0;
+  if (p.ringKr) p.ringKr = static_cast<char*>(p.ringKr) + g * h->R * fe * 2;
+  if (h->fp8) {
+    const int64_t code_bytes = h->fp4 ? fe / 2 : fe;  // per frame
+    p.amax += g * 2 * frames * h->H;
+    p.ring8[0] += g * h->R * code_bytes;
+    p.ring8[1] += g * h->R * code_bytes;
+    p.ring_scale += g * 2 * h->R * h->H;
+    if (h->fp4) {
+      p.ring_bs[0] += g * h->R * (fe / 16);
+      p.ring_bs[1] += g * h->R * (fe / 16);
+    }
+    p.stage[0] = static_cast<char*>(p.stage[0]) + g * h->Bmax * fe * 2;
+    p.stage[1] = static_cast<char*>(p.stage[1]) + g * h->Bmax * fe * 2;
+  }
+  return p;
+}
+
 static int append_steps(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
                         const void* const* v_sh, int frames) {
   // 1. the previous current block joins the window
@@ -598,7 +660,6 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
       ap.v_sh[r] = v_sh[r];
     }
   }
-  int e;
   if (h->fp8) {
     ap.amax = h->amax;
     ap.ring8[0] = static_cast<uint8_t*>(h->ringK);
@@ -610,13 +671,32 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
     ap.stage[0] = h->stageK;
     ap.stage[1] = h->stageV;
     ap.stage_frames = h->Bmax;
-    e = launch_append_fp8(ap, k, v, h->stream);
-    h->launches += 2;
-  } else {
-    e = launch_append_bf16(ap, k, v, h->ringK, h->ringV, h->stream);
-    h->launches++;
   }
-  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  // one launch set for all states, or (host buffers arriving chunk by chunk) one per
+  // chunk of states, each after its chunk's copy
+  const int chunk = h->io_pending ? h->io_chunk : h->S;
+  for (int g0 = 0, c = 0; g0 < h->S; g0 += chunk, ++c) {
+    const int n = h->S - g0 < chunk ? h->S - g0 : chunk;
+    if (h->io_pending) {
+      cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0);
+      if (w != cudaSuccess) return h->cuda_fail(w);
+    }
+    const AppendParams a = states_slice(h, ap, g0, n, frames);
+    const int64_t in_off = static_cast<int64_t>(g0) * frames * h->frame_elems() * 2;
+    const void* kc = k ? static_cast<const char*>(k) + in_off : nullptr;
+    const void* vc = v ? static_cast<const char*>(v) + in_off : nullptr;
+    int e;
+    if (h->fp8) {
+      e = launch_append_fp8(a, kc, vc, h->stream);
+      h->launches += 2;
+    } else {
+      const int64_t ring_off = static_cast<int64_t>(g0) * h->R * h->frame_elems() * 2;
+      e = launch_append_bf16(a, kc, vc, static_cast<char*>(h->ringK) + ring_off,
+                             static_cast<char*>(h->ringV) + ring_off, h->stream);
+      h->launches++;
+    }
+    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  }
   return CONVKV_OK;
 }
 
@@ -691,7 +771,11 @@ int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
   return CONVKV_OK;
 }
 
-static int attend_impl(convkv_t* h, const void* q, void* out, const void* const* q_sh, void* const* o_sh) {
+// out_host: the host-buffer form (queries copied in by chunks of states, see
+// convkv_attend_host); each chunk's attention waits for its queries, and its outputs
+// are copied back to out_host as soon as it ends.
+static int attend_impl(convkv_t* h, const void* q, void* out, const void* const* q_sh, void* const* o_sh,
+                       char* out_host = nullptr) {
   const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur, T = h->T;
   AttnParams ap{};
   ap.H = h->H;
@@ -761,11 +845,33 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   }
   km[3] = r ? h->mapSinkKr : km[2];
   vm[3] = r ? h->mapSinkV : vm[2];
+  const size_t bps = static_cast<size_t>(b) * h->frame_elems() * 2;   // query / output bytes per state
+  // before chunk c's attention: wait for its queries; after it: send its outputs back
+  auto io_before = [&](int c) -> cudaError_t {
+    return out_host ? cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0) : cudaSuccess;
+  };
+  auto io_after = [&](int c, int g0, int n) -> cudaError_t {
+    if (!out_host) return cudaSuccess;
+    cudaEvent_t done = h->io_ev[1 + h->io_nchunks + c];
+    cudaError_t e = cudaEventRecord(done, h->stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, done, 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(out_host + g0 * bps, static_cast<char*>(out) + g0 * bps, n * bps, cudaMemcpyDeviceToHost,
+                          h->io_back);
+    return e;
+  };
   if (!h->fp8) {
-    ap.state0 = 0;
-    int e = launch_attend(h->D, ap, mq, km, vm, h->S, h->stream);
-    h->launches++;
-    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    // one launch for all states, or one per chunk of states in the host-buffer form
+    const int chunk = out_host ? h->io_chunk : h->S;
+    for (int g0 = 0, c = 0; g0 < h->S; g0 += chunk, ++c) {
+      const int n = h->S - g0 < chunk ? h->S - g0 : chunk;
+      if (cudaError_t w = io_before(c)) return h->cuda_fail(w);
+      ap.state0 = g0;
+      int e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
+      h->launches++;
+      if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+      if (cudaError_t w = io_after(c, g0, n)) return h->cuda_fail(w);
+    }
     return CONVKV_OK;
   }
   // e4m3 / NVFP4: per group of states, dequantise [memory | window] into the scratch
@@ -801,17 +907,20 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   dp.div_heads = FastDiv(static_cast<uint32_t>(h->H));
   dp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
   __nv_bfloat16* const out0 = ap.out;
-  for (int g0 = 0; g0 < h->S; g0 += h->Sg) {
+  // (host-buffer form: the chunks of states are these groups)
+  for (int g0 = 0, c = 0; g0 < h->S; g0 += h->Sg, ++c) {
     const int n = h->S - g0 < h->Sg ? h->S - g0 : h->Sg;
     dp.state0 = g0;
     int e = launch_dequant(h->D, dp, n, h->stream);
     if (m + w > 0) h->launches++;
     if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    if (cudaError_t wt = io_before(c)) return h->cuda_fail(wt);
     ap.state0 = g0;
     ap.out = out0;
     e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
     h->launches++;
     if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    if (cudaError_t wt = io_after(c, g0, n)) return h->cuda_fail(wt);
   }
   return CONVKV_OK;
 }
@@ -832,27 +941,66 @@ int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_
   return attend_impl(h, nullptr, nullptr, q_shards, out_shards);
 }
 
+// Copies of `bps` bytes per state from host to device staging, chunk by chunk on the
+// copy stream, each chunk's completion recorded in its event; the copies start after
+// the work already queued on the handle's stream (which may still read the staging).
+static cudaError_t copy_in_chunks(convkv_t* h, void* const* dst, const void* const* src, int nbuf, size_t bps) {
+  cudaError_t e = cudaEventRecord(h->io_ev[0], h->stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_in, h->io_ev[0], 0);
+  for (int g0 = 0, c = 0; g0 < h->S && e == cudaSuccess; g0 += h->io_chunk, ++c) {
+    const int n = h->S - g0 < h->io_chunk ? h->S - g0 : h->io_chunk;
+    for (int i = 0; i < nbuf && e == cudaSuccess; ++i)
+      e = cudaMemcpyAsync(static_cast<char*>(dst[i]) + g0 * bps, static_cast<const char*>(src[i]) + g0 * bps,
+                          n * bps, cudaMemcpyHostToDevice, h->io_in);
+    if (e == cudaSuccess) e = cudaEventRecord(h->io_ev[1 + c], h->io_in);
+  }
+  return e;
+}
+
 int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames) {
   if (!h || !k_host || !v_host || frames < 1 || frames > h->Bmax) return CONVKV_ERR_INVALID_ARG;
   if (!h->host_io || h->dry) return CONVKV_ERR_BAD_ORDER;
-  const size_t bytes = static_cast<size_t>(h->S) * frames * h->frame_elems() * 2;
-  cudaError_t e = cudaMemcpyAsync(h->io_k, k_host, bytes, cudaMemcpyHostToDevice, h->stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->io_v, v_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  const size_t bps = static_cast<size_t>(frames) * h->frame_elems() * 2;
+  void* const dst[2] = {h->io_k, h->io_v};
+  const void* const src[2] = {k_host, v_host};
+  cudaError_t e = copy_in_chunks(h, dst, src, 2, bps);
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(h->io_in);
+    return h->cuda_fail(e);
+  }
+  // the conv of the evicted frames runs while the block is copied in; the ring append
+  // of each chunk of states waits for that chunk's copy
+  h->io_pending = true;
+  const int rc = convkv_append_block(h, h->io_k, h->io_v, frames);
+  h->io_pending = false;
+  // the caller may reuse its buffers once this returns
+  e = cudaStreamSynchronize(h->io_in);
+  if (rc != CONVKV_OK) return rc;
   if (e != cudaSuccess) return h->cuda_fail(e);
-  return convkv_append_block(h, h->io_k, h->io_v, frames);
+  return CONVKV_OK;
 }
 
 int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
   if (!h || !q_host || !out_host) return CONVKV_ERR_INVALID_ARG;
   if (!h->host_io || h->dry || h->blocks < 1 || h->need_append) return CONVKV_ERR_BAD_ORDER;
-  const size_t bytes = static_cast<size_t>(h->S) * h->bcur * h->frame_elems() * 2;
-  cudaError_t e = cudaMemcpyAsync(h->io_q, q_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  if (h->Rs > 0 && !h->sink_set) return CONVKV_ERR_BAD_ORDER;
+  const size_t bps = static_cast<size_t>(h->bcur) * h->frame_elems() * 2;
+  void* const dst[1] = {h->io_q};
+  const void* const src[1] = {q_host};
+  // queries in by chunks of states; each chunk's attention waits for its queries and
+  // its outputs go back on the second copy stream while later chunks compute
+  cudaError_t e = copy_in_chunks(h, dst, src, 1, bps);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, h->io_ev[0], 0);
+  int rc = CONVKV_OK;
+  if (e == cudaSuccess) rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host));
+  const cudaError_t e1 = cudaStreamSynchronize(h->io_in);
+  const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
+  const cudaError_t e3 = cudaStreamSynchronize(h->stream);
   if (e != cudaSuccess) return h->cuda_fail(e);
-  int rc = convkv_attend(h, h->io_q, h->io_out);
-  if (rc) return rc;
-  e = cudaMemcpyAsync(out_host, h->io_out, bytes, cudaMemcpyDeviceToHost, h->stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
-  if (e != cudaSuccess) return h->cuda_fail(e);
+  if (rc != CONVKV_OK) return rc;
+  if (e1 != cudaSuccess) return h->cuda_fail(e1);
+  if (e2 != cudaSuccess) return h->cuda_fail(e2);
+  if (e3 != cudaSuccess) return h->cuda_fail(e3);
   return CONVKV_OK;
 }
 

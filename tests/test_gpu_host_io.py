@@ -1,0 +1,72 @@
+"""The host-buffer entry points (convkv_append_block_host / convkv_attend_host) against
+the device-buffer ones, on the GPU.
+
+The host forms copy their inputs in by chunks of states on a copy stream, start each
+chunk's kernels as soon as its copy lands, and copy each chunk's outputs back while
+later chunks compute.  The kernels and their arithmetic are the same as in the device
+forms, so the outputs must be identical bit for bit, for several chunks: a bf16 handle
+of 3 states (three chunks) and an e4m3 handle of 8 states at 480x832 (two groups of
+states, hence two chunks, under the 4 GiB dequantisation scratch).
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+
+import seeded_inputs as si
+from compressed_kv_cache_convkv_b200.configs import PRESETS
+from streams import device_weights
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as t
+    assert t.cuda.is_available(), "GPU tests need a CUDA device"
+    from compressed_kv_cache_convkv_b200 import build
+    build.build()
+    si.build(device=True)
+    return t
+
+
+def _block(torch, w, tid, frame0, frames):
+    x = torch.empty((w.num_states, frames * w.T, w.heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    fe = w.T * w.heads * w.head_dim
+    stream = torch.cuda.current_stream().cuda_stream
+    for s in range(w.num_states):
+        si.frames_device(x[s].data_ptr(), w.seed, tid, s, frame0, frames, fe, 1.0, stream)
+    return x
+
+
+def _pinned(torch, x):
+    h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    h.copy_(x)
+    return h
+
+
+@pytest.mark.parametrize("name,states,blocks", [("tiny", 3, 12), ("fp8_480x832", 8, 5)])
+def test_host_buffers_match_device_buffers(torch, name, states, blocks):
+    import compressed_kv_cache_convkv_b200 as ckv
+    w = replace(PRESETS[name], num_states=states)
+    weights = device_weights(w, torch)
+    dev = ckv.ConvKV(w.config(), weights)
+    hio = ckv.ConvKV(w.config(host_io=True), weights)
+    frame0 = 0
+    for i, frames in enumerate(w.block_sizes()[:blocks]):
+        q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
+        frame0 += frames
+        dev.append(k, v)
+        o_dev = dev.attend(q)
+        qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        hio.append_host(kh, vh)
+        hio.attend_host(qh, oh)
+        torch.cuda.synchronize()
+        a = o_dev.view(torch.int16).cpu().numpy()
+        b = oh.view(torch.int16).numpy()
+        assert np.array_equal(a, b), (name, i)
+        assert dev.counters() == hio.counters()
+    assert dev.status() == 0 and hio.status() == 0
+    dev.close()
+    hio.close()
