@@ -95,6 +95,8 @@ struct convkv {
   std::vector<cudaEvent_t> io_ev;  // [0] start, [1 + c] chunk c copied in, [1 + nchunks + c] chunk c done
   int io_chunk = 0, io_nchunks = 0;
   bool io_pending = false;         // the next ring append reads io_k / io_v chunk by chunk
+  bool io_defer = false;           // the ring append is left to the caller (convkv_step_host)
+  AppendParams io_ap{};            // ... with these parameters
   CUtensorMap mapRingK{}, mapRingV{}, mapRingKr{}, mapMemK{}, mapMemV{}, mapW{}, mapStageK{}, mapStageV{}, mapSinkK{},
       mapSinkV{};
   // e4m3 / NVFP4: code tiles of the ring (read by the conv), and the bf16 scratch the
@@ -553,6 +555,33 @@ static AppendParams states_slice(const convkv_t* h, const AppendParams& a, int g
   return p;
 }
 
+// Step 4 of the append for states [g0, g0 + n): the new block into the ring (and the
+// rotated K / the staging copy).  With host buffers arriving by chunks, it first waits
+// for the chunk's copy (g0 is then a chunk boundary).
+static int ring_append_states(convkv_t* h, const AppendParams& ap, const void* k, const void* v, int g0, int n) {
+  if (h->io_pending) {
+    cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + g0 / h->io_chunk], 0);
+    if (w != cudaSuccess) return h->cuda_fail(w);
+  }
+  const int frames = ap.b;
+  const AppendParams a = states_slice(h, ap, g0, n, frames);
+  const int64_t in_off = static_cast<int64_t>(g0) * frames * h->frame_elems() * 2;
+  const void* kc = k ? static_cast<const char*>(k) + in_off : nullptr;
+  const void* vc = v ? static_cast<const char*>(v) + in_off : nullptr;
+  int e;
+  if (h->fp8) {
+    e = launch_append_fp8(a, kc, vc, h->stream);
+    h->launches += 2;
+  } else {
+    const int64_t ring_off = static_cast<int64_t>(g0) * h->R * h->frame_elems() * 2;
+    e = launch_append_bf16(a, kc, vc, static_cast<char*>(h->ringK) + ring_off, static_cast<char*>(h->ringV) + ring_off,
+                           h->stream);
+    h->launches++;
+  }
+  if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  return CONVKV_OK;
+}
+
 static int append_steps(convkv_t* h, const void* k, const void* v, const void* const* k_sh,
                         const void* const* v_sh, int frames) {
   // 1. the previous current block joins the window
@@ -672,30 +701,16 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
     ap.stage[1] = h->stageV;
     ap.stage_frames = h->Bmax;
   }
+  if (h->io_defer) {
+    h->io_ap = ap;
+    return CONVKV_OK;
+  }
   // one launch set for all states, or (host buffers arriving chunk by chunk) one per
   // chunk of states, each after its chunk's copy
   const int chunk = h->io_pending ? h->io_chunk : h->S;
-  for (int g0 = 0, c = 0; g0 < h->S; g0 += chunk, ++c) {
+  for (int g0 = 0; g0 < h->S; g0 += chunk) {
     const int n = h->S - g0 < chunk ? h->S - g0 : chunk;
-    if (h->io_pending) {
-      cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0);
-      if (w != cudaSuccess) return h->cuda_fail(w);
-    }
-    const AppendParams a = states_slice(h, ap, g0, n, frames);
-    const int64_t in_off = static_cast<int64_t>(g0) * frames * h->frame_elems() * 2;
-    const void* kc = k ? static_cast<const char*>(k) + in_off : nullptr;
-    const void* vc = v ? static_cast<const char*>(v) + in_off : nullptr;
-    int e;
-    if (h->fp8) {
-      e = launch_append_fp8(a, kc, vc, h->stream);
-      h->launches += 2;
-    } else {
-      const int64_t ring_off = static_cast<int64_t>(g0) * h->R * h->frame_elems() * 2;
-      e = launch_append_bf16(a, kc, vc, static_cast<char*>(h->ringK) + ring_off,
-                             static_cast<char*>(h->ringV) + ring_off, h->stream);
-      h->launches++;
-    }
-    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    if (int rc = ring_append_states(h, ap, k, v, g0, n)) return rc;
   }
   return CONVKV_OK;
 }
@@ -775,7 +790,8 @@ int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
 // convkv_attend_host); each chunk's attention waits for its queries, and its outputs
 // are copied back to out_host as soon as it ends.
 static int attend_impl(convkv_t* h, const void* q, void* out, const void* const* q_sh, void* const* o_sh,
-                       char* out_host = nullptr) {
+                       char* out_host = nullptr, int gbeg = 0, int gend = -1) {
+  if (gend < 0) gend = h->S;
   const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur, T = h->T;
   AttnParams ap{};
   ap.H = h->H;
@@ -863,8 +879,8 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   if (!h->fp8) {
     // one launch for all states, or one per chunk of states in the host-buffer form
     const int chunk = out_host ? h->io_chunk : h->S;
-    for (int g0 = 0, c = 0; g0 < h->S; g0 += chunk, ++c) {
-      const int n = h->S - g0 < chunk ? h->S - g0 : chunk;
+    for (int g0 = gbeg, c = gbeg / chunk; g0 < gend; g0 += chunk, ++c) {
+      const int n = gend - g0 < chunk ? gend - g0 : chunk;
       if (cudaError_t w = io_before(c)) return h->cuda_fail(w);
       ap.state0 = g0;
       int e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
@@ -908,8 +924,8 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   dp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
   __nv_bfloat16* const out0 = ap.out;
   // (host-buffer form: the chunks of states are these groups)
-  for (int g0 = 0, c = 0; g0 < h->S; g0 += h->Sg, ++c) {
-    const int n = h->S - g0 < h->Sg ? h->S - g0 : h->Sg;
+  for (int g0 = gbeg, c = gbeg / h->Sg; g0 < gend; g0 += h->Sg, ++c) {
+    const int n = gend - g0 < h->Sg ? gend - g0 : h->Sg;
     dp.state0 = g0;
     int e = launch_dequant(h->D, dp, n, h->stream);
     if (m + w > 0) h->launches++;
@@ -997,6 +1013,58 @@ int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
   const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
   const cudaError_t e3 = cudaStreamSynchronize(h->stream);
   if (e != cudaSuccess) return h->cuda_fail(e);
+  if (rc != CONVKV_OK) return rc;
+  if (e1 != cudaSuccess) return h->cuda_fail(e1);
+  if (e2 != cudaSuccess) return h->cuda_fail(e2);
+  if (e3 != cudaSuccess) return h->cuda_fail(e3);
+  return CONVKV_OK;
+}
+
+int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
+                     int frames) {
+  if (!h || !k_host || !v_host || !q_host || !out_host || frames < 1 || frames > h->Bmax)
+    return CONVKV_ERR_INVALID_ARG;
+  if (!h->host_io || h->dry) return CONVKV_ERR_BAD_ORDER;
+  if (h->Rs > 0 && !h->sink_set) return CONVKV_ERR_BAD_ORDER;
+  const size_t bps = static_cast<size_t>(frames) * h->frame_elems() * 2;
+  void* const dst[3] = {h->io_k, h->io_v, h->io_q};
+  const void* const src[3] = {k_host, v_host, q_host};
+  cudaError_t e = copy_in_chunks(h, dst, src, 3, bps);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, h->io_ev[0], 0);
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(h->io_in);
+    return h->cuda_fail(e);
+  }
+  // bookkeeping, conv, time table and key rotation for all states (while the block is
+  // copied in); then per chunk of states: its ring append, its attention, its outputs
+  // back -- a chunk's kernels wait only for its own inputs
+  const int64_t P = h->P, E = h->E, Sn = h->Sn, blocks = h->blocks;
+  const int bcur = h->bcur, last_groups = h->last_groups;
+  h->io_pending = true;
+  h->io_defer = true;
+  int rc = convkv_append_block(h, h->io_k, h->io_v, frames);
+  h->io_defer = false;
+  for (int g0 = 0; rc == CONVKV_OK && g0 < h->S; g0 += h->io_chunk) {
+    const int n = h->S - g0 < h->io_chunk ? h->S - g0 : h->io_chunk;
+    rc = ring_append_states(h, h->io_ap, h->io_k, h->io_v, g0, n);
+    if (rc == CONVKV_OK)
+      rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host), g0, g0 + n);
+    if (rc != CONVKV_OK) {
+      // as a failed append (later chunks are not appended): counters back, attends
+      // refused until an append succeeds, which rewrites the same ring slots
+      h->P = P;
+      h->E = E;
+      h->Sn = Sn;
+      h->blocks = blocks;
+      h->bcur = bcur;
+      h->last_groups = last_groups;
+      h->need_append = true;
+    }
+  }
+  h->io_pending = false;
+  const cudaError_t e1 = cudaStreamSynchronize(h->io_in);
+  const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
+  const cudaError_t e3 = cudaStreamSynchronize(h->stream);
   if (rc != CONVKV_OK) return rc;
   if (e1 != cudaSuccess) return h->cuda_fail(e1);
   if (e2 != cudaSuccess) return h->cuda_fail(e2);

@@ -126,12 +126,32 @@ int convkv_append_block(convkv_t* h, const void* k, const void* v, int frames);
  * Errors: INVALID_ARG, BAD_ORDER, CUDA. */
 int convkv_attend(convkv_t* h, const void* q, void* out);
 
-/* Same as append_block / attend but with HOST buffers (pinned or pageable):
- * the inputs are copied into handle-owned device staging, the output is copied
- * back, and the call returns after the copy back completed.  Needs
- * CONVKV_FLAG_HOST_IO at create.  Errors: as above, plus BAD_ORDER without the flag. */
+/* Same as append_block / attend but with HOST buffers (pinned or pageable): the
+ * inputs are copied into handle-owned device staging by chunks of states on the
+ * handle's own copy stream, and each chunk's ring append or attention starts as soon
+ * as that chunk has landed; attend_host copies each chunk's outputs back on a second
+ * copy stream while later chunks compute (chunks: the attention's groups of states
+ * in the e4m3 / NVFP4 formats, eighths of the states in bf16).  Both calls return
+ * once the host buffers are no longer accessed: the inputs copied in, the outputs
+ * copied back.  With pinned buffers the copies overlap the kernels.  Needs
+ * CONVKV_FLAG_HOST_IO at create (which also creates the two copy streams and their
+ * events).  Errors: as above, plus BAD_ORDER without the flag. */
 int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames);
 int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host);
+
+/* One step from and to HOST buffers: append_block_host(k_host, v_host, frames)
+ * followed by attend_host(q_host, out_host), with the queries of the new block
+ * (`frames` frames).  The inputs are copied in by chunks of states; each chunk's
+ * ring append and attention start as soon as its k, v and q have landed, and its
+ * outputs go back while later chunks compute (the conv of the evicted frames, the
+ * time table and the key rotation run for all states first, while the block is
+ * copied in).  Same results, bit for bit, as the two calls.  Returns once the host
+ * buffers are no longer accessed.  A failure after the bookkeeping counts as a
+ * failed append (counters restored, attends BAD_ORDER until an append succeeds).
+ * Needs CONVKV_FLAG_HOST_IO.  Errors: as append_block and attend, plus BAD_ORDER
+ * without the flag. */
+int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
+                     int frames);
 
 /* Device bytes owned by the handle; constant from create to destroy. */
 size_t convkv_state_bytes(const convkv_t* h);

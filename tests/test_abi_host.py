@@ -84,6 +84,15 @@ def test_call_order_and_argument_checks():
     assert lib.convkv_attend(h._h, None, None) == ckv.OK
     assert lib.convkv_read_slot(h._h, 0, 0, 0, None, None) == ckv.ERR_INVALID_ARG
     assert lib.convkv_append_block_host(h._h, None, None, 2) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_step_host(h._h, None, None, None, None, 2) == ckv.ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(16)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    c1 = h.counters()
+    # the host-buffer forms need device staging: dry-run handles refuse them untouched
+    assert lib.convkv_step_host(h._h, p, p, p, p, 2) == ckv.ERR_BAD_ORDER
+    assert lib.convkv_step_host(h._h, p, p, p, p, 3) == ckv.ERR_INVALID_ARG   # > max block
+    assert lib.convkv_append_block_host(h._h, p, p, 2) == ckv.ERR_BAD_ORDER
+    assert h.counters() == c1
     assert lib.convkv_state_bytes(h._h) == 0 and h.launch_count() == 0
     lib.convkv_destroy(None)
 

@@ -3,7 +3,8 @@ the device-buffer ones, on the GPU.
 
 The host forms copy their inputs in by chunks of states on a copy stream, start each
 chunk's kernels as soon as its copy lands, and copy each chunk's outputs back while
-later chunks compute.  The kernels and their arithmetic are the same as in the device
+later chunks compute; convkv_step_host does an append and an attend in one such
+pipelined call.  The kernels and their arithmetic are the same as in the device
 forms, so the outputs must be identical bit for bit, for several chunks: a bf16 handle
 of 3 states (three chunks) and an e4m3 handle of 8 states at 480x832 (two groups of
 states, hence two chunks, under the 4 GiB dequantisation scratch).
@@ -52,6 +53,7 @@ def test_host_buffers_match_device_buffers(torch, name, states, blocks):
     weights = device_weights(w, torch)
     dev = ckv.ConvKV(w.config(), weights)
     hio = ckv.ConvKV(w.config(host_io=True), weights)
+    fused = ckv.ConvKV(w.config(host_io=True), weights)
     frame0 = 0
     for i, frames in enumerate(w.block_sizes()[:blocks]):
         q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
@@ -60,13 +62,15 @@ def test_host_buffers_match_device_buffers(torch, name, states, blocks):
         o_dev = dev.attend(q)
         qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
         oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        of = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
         hio.append_host(kh, vh)
         hio.attend_host(qh, oh)
+        fused.step_host(kh, vh, qh, of)
         torch.cuda.synchronize()
         a = o_dev.view(torch.int16).cpu().numpy()
-        b = oh.view(torch.int16).numpy()
-        assert np.array_equal(a, b), (name, i)
-        assert dev.counters() == hio.counters()
-    assert dev.status() == 0 and hio.status() == 0
-    dev.close()
-    hio.close()
+        assert np.array_equal(a, oh.view(torch.int16).numpy()), (name, i, "append_host + attend_host")
+        assert np.array_equal(a, of.view(torch.int16).numpy()), (name, i, "step_host")
+        assert dev.counters() == hio.counters() == fused.counters()
+    assert dev.status() == 0 and hio.status() == 0 and fused.status() == 0
+    for h in (dev, hio, fused):
+        h.close()
