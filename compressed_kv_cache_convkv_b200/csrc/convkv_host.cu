@@ -85,6 +85,8 @@ struct convkv {
   void *scrK = nullptr, *scrV = nullptr;      // e4m3 / NVFP4: bf16 scratch [Sg][(C + W) * T][H][D]
   int Sg = 0;                                 // states per dequantise-and-attend group
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
+  float* convacc = nullptr;                   // e4m3 / NVFP4: fp32 conv outputs of one append
+  int gmax = 0;                               // eviction groups one append can produce
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
@@ -373,6 +375,11 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->Sg = static_cast<int>(per_state * h->S <= budget ? h->S : (budget / per_state > 0 ? budget / per_state : 1));
   }
   const size_t scr_b = h->fp8 ? static_cast<size_t>(h->Sg) * (h->C + h->W) * fe * 2 : 0;
+  // e4m3 / NVFP4: the conv's fp32 outputs for the groups of one append (the window
+  // holds at most W + Bmax frames before an append's evictions, so at most
+  // ceil(Bmax / 5) groups)
+  h->gmax = (h->Bmax + kEvict - 1) / kEvict;
+  const size_t acc_b = h->fp8 ? static_cast<size_t>(h->S) * h->gmax * 2 * fe * sizeof(float) : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -385,7 +392,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
                o_sv = take(stg_b), o_am = take(amax_b), o_rfk = take(sink_b), o_rfv = take(sink_b),
                o_rbk = take(rbs_b), o_rbv = take(rbs_b), o_mbk = take(mbs_b), o_mbv = take(mbs_b),
                o_rkr = take(rkr_b), o_mkr = take(mkr_b), o_skr = take(sink_b), o_sck = take(scr_b),
-               o_scv = take(scr_b);
+               o_scv = take(scr_b), o_acc = take(acc_b);
   h->arena_bytes = off;
   cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
   if (e != cudaSuccess) {
@@ -410,6 +417,7 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     h->amax = reinterpret_cast<unsigned int*>(a + o_am);
     h->scrK = a + o_sck;
     h->scrV = a + o_scv;
+    h->convacc = reinterpret_cast<float*>(a + o_acc);
   }
   if (h->fp4) {
     h->ringBK = reinterpret_cast<uint8_t*>(a + o_rbk);
@@ -623,7 +631,9 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
         cp.ring8[1] = static_cast<const uint8_t*>(h->ringV);
         cp.ring_scale = h->ring_scale;
         cp.amax = h->amax;
+        cp.acc = h->convacc;
         cp.mem_scale = h->mem_scale;
+        if (cp.ngroups > h->gmax) return h->cuda_fail(cudaErrorInvalidValue);
         cp.ring_bs[0] = h->ringBK;
         cp.ring_bs[1] = h->ringBV;
         cp.mem_bs[0] = h->memBK;

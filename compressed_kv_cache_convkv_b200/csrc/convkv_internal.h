@@ -103,8 +103,9 @@ struct ConvParams {
   void* memK;             // bf16 [S][C*T][H][D], or e4m3 in the fp8 format
   void* memV;
   int* status;
-  // fp8 format: e4m3 ring input with per-(frame, head) scales, two passes
-  int pass;                   // 1: amax of the conv output only, 2: quantise with that amax
+  // fp8 format: e4m3 ring input with per-(frame, head) scales; the conv pass keeps its
+  // fp32 outputs and their per-(slot, head) amax, a second kernel quantises them
+  float* acc;                 // fp32 conv outputs [S][ngroups][2][T][H][D] of this launch
   const uint8_t* ring8[2];    // e4m3 K, V rings [S][R*T][H][D]
   const float* ring_scale;    // [S][2][R][H]
   unsigned int* amax;         // [S][2][ngroups][H] fp32 bit patterns (scratch, zeroed before pass 1)

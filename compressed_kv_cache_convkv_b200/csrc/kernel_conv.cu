@@ -13,12 +13,12 @@
 // k-block is its own load, so wrap costs nothing) and the matching D x D
 // weight block.  Warp 0 issues TMA, warp 1 issues tcgen05.mma (M=128, N=D,
 // K=16 steps) and owns the TMEM accumulators, warps 2-5 drain them.  The bf16
-// kernel is persistent (one CTA per SM walking the units); the low-precision one
-// keeps one unit per CTA.
+// and low-precision kernels are persistent (one CTA per SM walking the units).
 #include "convkv_internal.h"
 #include "sm100.cuh"
 #include "nvfp4.cuh"
 #include "quant_div.cuh"
+#include "token_walk.h"
 
 namespace ckv {
 namespace {
@@ -224,12 +224,12 @@ __global__ void __launch_bounds__(ConvCfg<D>::THREADS, 1)
 // fp8 (e4m3) format.  The evicted frames are e4m3 with one fp32 scale per
 // (frame, head); the A operand's codes arrive by TMA and are dequantised to bf16
 // (x * scale) in shared memory by warps 6-13.  The slot is stored e4m3 with one scale
-// per (slot, head) = amax / 448 over the slot's [T, D] values, so the launch
-// runs twice: pass 1 only reduces amax (atomicMax on the fp32 bit pattern,
-// values are non-negative), pass 2 recomputes the same tiles and quantises
-// with that scale (round-to-nearest-even, saturating to +-448).  FMT 2 is the
-// NVFP4 format: e2m1 codes with an e4m3 scale per 16 channels and the fp32
-// scale per (frame or slot, head) of the same two-pass rule (nvfp4.cuh).
+// per (slot, head) = amax / 448 over the slot's [T, D] values, so the conv keeps
+// its fp32 outputs in a scratch and reduces amax (atomicMax on the fp32 bit
+// pattern, values are non-negative); slot_quant_kernel then quantises them with
+// that scale (round-to-nearest-even, saturating to +-448).  FMT 2 is the NVFP4
+// format: e2m1 codes with an e4m3 scale per 16 channels and the fp32 scale per
+// (frame or slot, head) from the same amax (nvfp4.cuh).
 __device__ __forceinline__ void e4m3x2_to_f32_c(uint32_t two, float& lo, float& hi) {
   uint32_t h2;
   asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
@@ -277,9 +277,9 @@ struct LowpCfg {
 };
 
 // Persistent like the bf16 kernel: CTAs walk the units, the accumulator is double-
-// buffered in TMEM.  PASS 1 reduces each slot's amax; PASS 2 recomputes the same
-// tiles and quantises with it.
-template <int D, int PASS, int FMT>
+// buffered in TMEM.  The epilogue keeps the fp32 outputs (p.acc) and reduces each new
+// slot's amax over its tokens; slot_quant_kernel then quantises them with it.
+template <int D, int FMT>
 __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
     conv_lowp_kernel(const __grid_constant__ CUtensorMap tmCodesK, const __grid_constant__ CUtensorMap tmCodesV,
                      const __grid_constant__ CUtensorMap tmW, const ConvParams p, int MT, int units) {
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
       }
     }
   } else {
-    // warps 2..5: drain the accumulator -> amax (pass 1) or codes (pass 2)
+    // warps 2..5: drain the accumulator -> fp32 outputs and the slot's amax
     const int lane_base = (warp & 3) * 32;
     const int r = lane_base + lane;
     int n = 0;
@@ -483,79 +483,27 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
       const bool valid = token < p.T;
       const uint32_t tacc = tmem + ab * C::TMEM_COLS + (static_cast<uint32_t>(lane_base) << 16);
       const int64_t aidx = ((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.ngroups + cu.g) * p.H + cu.head;
-      if (PASS == 1) {
-        float mx = 0.0f;
+      // amax of the slot, and the fp32 outputs for the quantiser (one row per thread)
+      float* orow = p.acc + ((((static_cast<int64_t>(cu.state) * p.ngroups + cu.g) * 2 + cu.kv) * p.T + token) * p.H +
+                             cu.head) * D;
+      float mx = 0.0f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tacc + c * 32, v);
-          tmem_ld_wait();
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tacc + c * 32, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(__uint_as_float(v[e])));
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(__uint_as_float(v[e])));
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<uint4*>(orow + c * 32)[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
-        if (!valid) mx = 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0 && mx > 0.0f) atomicMax(&p.amax[aidx], __float_as_uint(mx));
-      } else if (FMT == 2) {
-        const float gs = fp4::tensor_scale(__uint_as_float(p.amax[aidx]));
-        const SharedDivisor g6 = fp4::block_divisor(gs);
-        const int64_t row = ((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head;
-        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) + row * (D / 2));
-        uint8_t* bs = p.mem_bs[cu.kv] + row * (D / 16);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tacc + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-            float xs[fp4::kBlock];
-            float a_b = 0.0f;
-#pragma unroll
-            for (int e = 0; e < fp4::kBlock; ++e) {
-              xs[e] = __uint_as_float(v[hb * 16 + e]);
-              a_b = fmaxf(a_b, fabsf(xs[e]));
-            }
-            float e_b;
-            const uint32_t sc = fp4::block_scale(a_b, gs, g6, e_b);
-            const uint2 cw = fp4::encode_block(xs, e_b);
-            if (valid) {
-              dst[2 * c + hb] = cw;
-              bs[2 * c + hb] = static_cast<uint8_t>(sc);
-            }
-          }
-        }
-        if (cu.mt == 0 && r == 0)
-          p.mem_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.C + p.grp[cu.g].mem_pos) * p.H + cu.head] = gs;
-      } else {
-        const float amax = __uint_as_float(p.amax[aidx]);
-        const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        const SharedDivisor dv = make_divisor(scale);
-        uint8_t* dst = static_cast<uint8_t*>(cu.kv ? p.memV : p.memK) +
-                       (((static_cast<int64_t>(cu.state) * p.C + p.grp[cu.g].mem_pos) * p.T + token) * p.H + cu.head) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tacc + c * 32, v);
-          tmem_ld_wait();
-          uint32_t w[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t lo = f32x2_to_e4m3(div_rn(__uint_as_float(v[4 * e]), dv),
-                                              div_rn(__uint_as_float(v[4 * e + 1]), dv));
-            const uint32_t hi = f32x2_to_e4m3(div_rn(__uint_as_float(v[4 * e + 2]), dv),
-                                              div_rn(__uint_as_float(v[4 * e + 3]), dv));
-            w[e] = lo | (hi << 16);
-          }
-          if (valid) {
-            reinterpret_cast<uint4*>(dst)[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
-            reinterpret_cast<uint4*>(dst)[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-          }
-        }
-        if (cu.mt == 0 && r == 0)
-          p.mem_scale[((static_cast<int64_t>(cu.state) * 2 + cu.kv) * p.C + p.grp[cu.g].mem_pos) * p.H + cu.head] = scale;
       }
+      if (!valid) mx = 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0 && mx > 0.0f) atomicMax(&p.amax[aidx], __float_as_uint(mx));
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
     }
@@ -574,6 +522,75 @@ __global__ void __launch_bounds__(LowpCfg<D>::THREADS, 1)
 
 namespace {
 
+// Quantisation of the new memory slots from the conv pass's fp32 outputs, with the
+// slot's amax from that pass: the same arithmetic as quantising in the conv's
+// epilogue (scale = amax / 448, code = e4m3(x / scale); NVFP4: tensor scale, block
+// scales, e2m1 codes), so the codes do not depend on which kernel makes them.
+// grid = (walkers * slabs, S * ngroups, 2 (K|V)), token walk: each thread owns one
+// (head, 8-channel chunk) column (e4m3) or one (head, 16-channel block) column
+// (NVFP4) of the slot.
+template <int D, int FMT>
+__global__ void slot_quant_kernel(ConvParams p) {
+  constexpr int CW = FMT == 2 ? fp4::kBlock : 8;          // channels per column
+  constexpr int NCOL = D / CW;
+  const int cols = p.H * NCOL;
+  const int sg = blockIdx.y;
+  const int s = sg / p.ngroups;
+  const int g = sg - s * p.ngroups;
+  const int kv = blockIdx.z;
+  const int slabs = (cols + blockDim.x - 1) / blockDim.x;
+  const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
+  const int col = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  if (col >= cols) return;
+  const int h = col / NCOL;
+  const int c = col - h * NCOL;
+  const int64_t aidx = ((static_cast<int64_t>(s) * 2 + kv) * p.ngroups + g) * p.H + h;
+  const float amax = __uint_as_float(p.amax[aidx]);
+  const int pos = p.grp[g].mem_pos;
+  const float* src = p.acc + (((static_cast<int64_t>(s) * p.ngroups + g) * 2 + kv) * p.T) * p.H * D + h * D + c * CW;
+  const int64_t row0 = (static_cast<int64_t>(s) * p.C + pos) * p.T * p.H + h;   // token 0's token-head row
+  uint8_t* mem = static_cast<uint8_t*>(kv ? p.memV : p.memK);
+  if constexpr (FMT == 2) {
+    const float gs = fp4::tensor_scale(amax);
+    const SharedDivisor g6 = fp4::block_divisor(gs);
+    if (walker == 0 && c == 0) p.mem_scale[((static_cast<int64_t>(s) * 2 + kv) * p.C + pos) * p.H + h] = gs;
+    for (int tok = walker; tok < p.T; tok += walkers) {
+      const float4* x4 = reinterpret_cast<const float4*>(src + static_cast<int64_t>(tok) * p.H * D);
+      float xs[fp4::kBlock];
+      float a_b = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = __ldcs(x4 + q);
+        xs[4 * q] = v.x;
+        xs[4 * q + 1] = v.y;
+        xs[4 * q + 2] = v.z;
+        xs[4 * q + 3] = v.w;
+      }
+#pragma unroll
+      for (int e = 0; e < fp4::kBlock; ++e) a_b = fmaxf(a_b, fabsf(xs[e]));
+      float e_b;
+      const uint32_t sc = fp4::block_scale(a_b, gs, g6, e_b);
+      const int64_t row = row0 + static_cast<int64_t>(tok) * p.H;
+      reinterpret_cast<uint2*>(mem)[row * NCOL + c] = fp4::encode_block(xs, e_b);
+      p.mem_bs[kv][row * NCOL + c] = static_cast<uint8_t>(sc);
+    }
+  } else {
+    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const SharedDivisor dv = make_divisor(scale);
+    if (walker == 0 && c == 0) p.mem_scale[((static_cast<int64_t>(s) * 2 + kv) * p.C + pos) * p.H + h] = scale;
+    for (int tok = walker; tok < p.T; tok += walkers) {
+      const float4* x4 = reinterpret_cast<const float4*>(src + static_cast<int64_t>(tok) * p.H * D);
+      const float4 a = __ldcs(x4), b = __ldcs(x4 + 1);
+      const uint32_t w0 = f32x2_to_e4m3(div_rn(a.x, dv), div_rn(a.y, dv)) |
+                          (f32x2_to_e4m3(div_rn(a.z, dv), div_rn(a.w, dv)) << 16);
+      const uint32_t w1 = f32x2_to_e4m3(div_rn(b.x, dv), div_rn(b.y, dv)) |
+                          (f32x2_to_e4m3(div_rn(b.z, dv), div_rn(b.w, dv)) << 16);
+      const int64_t row = row0 + static_cast<int64_t>(tok) * p.H;
+      reinterpret_cast<uint2*>(mem + row * D)[c] = make_uint2(w0, w1);
+    }
+  }
+}
+
 template <int D, int FMT>
 int launch_lowp(const ConvParams& p, const CUtensorMap& codesK, const CUtensorMap& codesV, const CUtensorMap& wmap,
                 cudaStream_t s) {
@@ -586,12 +603,14 @@ int launch_lowp(const ConvParams& p, const CUtensorMap& codesK, const CUtensorMa
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = units < sms ? units : sms;
-  auto k1 = conv_lowp_kernel<D, 1, FMT>;
-  auto k2 = conv_lowp_kernel<D, 2, FMT>;
+  auto k1 = conv_lowp_kernel<D, FMT>;
   cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   k1<<<grid, LowpCfg<D>::THREADS, C::SMEM, s>>>(codesK, codesV, wmap, p, MT, units);
-  k2<<<grid, LowpCfg<D>::THREADS, C::SMEM, s>>>(codesK, codesV, wmap, p, MT, units);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  constexpr int NCOL = D / (FMT == 2 ? fp4::kBlock : 8);
+  dim3 qgrid(token_grid_x(p.T, p.H * NCOL, 2 * p.S * p.ngroups), p.S * p.ngroups, 2);
+  slot_quant_kernel<D, FMT><<<qgrid, kTokenThreads, 0, s>>>(p);
   return static_cast<int>(cudaGetLastError());
 }
 
