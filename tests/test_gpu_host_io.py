@@ -74,3 +74,40 @@ def test_host_buffers_match_device_buffers(torch, name, states, blocks):
     assert dev.status() == 0 and hio.status() == 0 and fused.status() == 0
     for h in (dev, hio, fused):
         h.close()
+
+
+@pytest.mark.parametrize("step", [0, 1, 2])
+def test_step_host_failure_rolls_back_and_recovers(torch, step):
+    """A launch failure injected on the host at one step of convkv_step_host's append
+    (conv, time-table upload, ring append) leaves the counters as before the call and
+    refuses attends; repeating the same step then gives the device path's outputs bit
+    for bit (the failed call's partial work is rewritten)."""
+    import compressed_kv_cache_convkv_b200 as ckv
+    w = replace(PRESETS["tiny"], fp8=True, num_states=3, name="tiny_fp8")
+    weights = device_weights(w, torch)
+    dev = ckv.ConvKV(w.config(), weights)
+    hio = ckv.ConvKV(w.config(host_io=True), weights)
+    lib = ckv.library()
+    frame0 = 0
+    for i, frames in enumerate(w.block_sizes()[:8]):
+        q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
+        frame0 += frames
+        dev.append(k, v)
+        o_dev = dev.attend(q)
+        qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        if i == 5:
+            # block 5 evicts a group, so all three append steps run
+            before = hio.counters()
+            assert lib.convkv_debug_fail_step(hio._h, step) == ckv.OK
+            rc = lib.convkv_step_host(hio._h, kh.data_ptr(), vh.data_ptr(), qh.data_ptr(), oh.data_ptr(), frames)
+            assert rc == ckv.ERR_CUDA
+            assert hio.counters() == before
+            assert lib.convkv_attend_host(hio._h, qh.data_ptr(), oh.data_ptr()) == ckv.ERR_BAD_ORDER
+        hio.step_host(kh, vh, qh, oh)
+        torch.cuda.synchronize()
+        assert np.array_equal(o_dev.view(torch.int16).cpu().numpy(), oh.view(torch.int16).numpy()), (step, i)
+        assert dev.counters() == hio.counters()
+    assert dev.status() == 0 and hio.status() == 0
+    dev.close()
+    hio.close()
