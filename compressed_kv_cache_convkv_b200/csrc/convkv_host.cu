@@ -90,12 +90,13 @@ struct convkv {
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
-  // host I/O (CONVKV_FLAG_HOST_IO): the *_host entry points copy by chunks of io_chunk
-  // states on their own streams, and each chunk's kernels wait only for that chunk's
-  // copy, so copies in both directions overlap the kernels of other chunks
+  // host I/O (CONVKV_FLAG_HOST_IO): the *_host entry points copy by chunks of states
+  // on their own streams, and each chunk's kernels wait only for that chunk's copy, so
+  // copies in both directions overlap the kernels of other chunks
   cudaStream_t io_in = nullptr, io_back = nullptr;
   std::vector<cudaEvent_t> io_ev;  // [0] start, [1 + c] chunk c copied in, [1 + nchunks + c] chunk c done
-  int io_chunk = 0, io_nchunks = 0;
+  std::vector<int> io_start;       // chunk c = states [io_start[c], io_start[c + 1])
+  int io_nchunks = 0;
   bool io_pending = false;         // the next ring append reads io_k / io_v chunk by chunk
   bool io_defer = false;           // the ring append is left to the caller (convkv_step_host)
   AppendParams io_ap{};            // ... with these parameters
@@ -281,13 +282,22 @@ const char* convkv_strerror(int code) {
   }
 }
 
-// Copy streams and events of the host-buffer entry points.  Chunks follow the
-// attention's state groups in the low-precision formats (a group's attention waits
-// for its queries only), and split the states eight ways in the bf16 format.
+// Copy streams and events of the host-buffer entry points, and the chunks of states.
+// The first chunk is one state and each next one about 1.35 times larger (at most the
+// attention's group of states in the low-precision formats), so the kernels start
+// after one state's copy and a chunk's copy takes about as long as the previous
+// chunk's kernels (one state's copy in takes about 0.75 of its kernels' time at the
+// 480x832 shape); a short last chunk keeps the final copy back short too.
 static int create_host_io(convkv_t* h) {
-  h->io_chunk = h->fp8 ? h->Sg : (h->S + 7) / 8;
-  if (h->io_chunk < 1) h->io_chunk = 1;
-  h->io_nchunks = (h->S + h->io_chunk - 1) / h->io_chunk;
+  const int cap = h->fp8 ? h->Sg : h->S;
+  h->io_start.assign(1, 0);
+  for (int n = 1; h->io_start.back() < h->S;) {
+    const int g0 = h->io_start.back();
+    h->io_start.push_back(g0 + (h->S - g0 < n ? h->S - g0 : n));
+    n = (n * 135 + 99) / 100;
+    if (n > cap) n = cap;
+  }
+  h->io_nchunks = static_cast<int>(h->io_start.size()) - 1;
   if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)
     return CONVKV_ERR_CUDA;
@@ -564,11 +574,12 @@ static AppendParams states_slice(const convkv_t* h, const AppendParams& a, int g
 }
 
 // Step 4 of the append for states [g0, g0 + n): the new block into the ring (and the
-// rotated K / the staging copy).  With host buffers arriving by chunks, it first waits
-// for the chunk's copy (g0 is then a chunk boundary).
-static int ring_append_states(convkv_t* h, const AppendParams& ap, const void* k, const void* v, int g0, int n) {
-  if (h->io_pending) {
-    cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + g0 / h->io_chunk], 0);
+// rotated K / the staging copy).  With host buffers arriving by chunks (c >= 0: the
+// chunk of these states), it first waits for the chunk's copy.
+static int ring_append_states(convkv_t* h, const AppendParams& ap, const void* k, const void* v, int g0, int n,
+                              int c) {
+  if (c >= 0) {
+    cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0);
     if (w != cudaSuccess) return h->cuda_fail(w);
   }
   const int frames = ap.b;
@@ -717,11 +728,9 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
   }
   // one launch set for all states, or (host buffers arriving chunk by chunk) one per
   // chunk of states, each after its chunk's copy
-  const int chunk = h->io_pending ? h->io_chunk : h->S;
-  for (int g0 = 0; g0 < h->S; g0 += chunk) {
-    const int n = h->S - g0 < chunk ? h->S - g0 : chunk;
-    if (int rc = ring_append_states(h, ap, k, v, g0, n)) return rc;
-  }
+  if (!h->io_pending) return ring_append_states(h, ap, k, v, 0, h->S, -1);
+  for (int c = 0; c < h->io_nchunks; ++c)
+    if (int rc = ring_append_states(h, ap, k, v, h->io_start[c], h->io_start[c + 1] - h->io_start[c], c)) return rc;
   return CONVKV_OK;
 }
 
@@ -874,10 +883,10 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   const size_t bps = static_cast<size_t>(b) * h->frame_elems() * 2;   // query / output bytes per state
   // before chunk c's attention: wait for its queries; after it: send its outputs back
   auto io_before = [&](int c) -> cudaError_t {
-    return out_host ? cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0) : cudaSuccess;
+    return c >= 0 ? cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0) : cudaSuccess;
   };
   auto io_after = [&](int c, int g0, int n) -> cudaError_t {
-    if (!out_host) return cudaSuccess;
+    if (c < 0) return cudaSuccess;
     cudaEvent_t done = h->io_ev[1 + h->io_nchunks + c];
     cudaError_t e = cudaEventRecord(done, h->stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, done, 0);
@@ -886,11 +895,23 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
                           h->io_back);
     return e;
   };
+  // the launch groups: the host-buffer chunks in [gbeg, gend) (chunk index c), else
+  // all states at once (bf16) or groups of Sg states (the scratch's capacity)
+  std::vector<int> gb;   // group starts, then gend
+  int c0 = -1;
+  if (out_host) {
+    for (int c = 0; c < h->io_nchunks; ++c) {
+      if (h->io_start[c] < gbeg || h->io_start[c] >= gend) continue;
+      if (c0 < 0) c0 = c;
+      gb.push_back(h->io_start[c]);
+    }
+  } else {
+    for (int g0 = gbeg; g0 < gend; g0 += h->fp8 ? h->Sg : h->S) gb.push_back(g0);
+  }
+  gb.push_back(gend);
   if (!h->fp8) {
-    // one launch for all states, or one per chunk of states in the host-buffer form
-    const int chunk = out_host ? h->io_chunk : h->S;
-    for (int g0 = gbeg, c = gbeg / chunk; g0 < gend; g0 += chunk, ++c) {
-      const int n = gend - g0 < chunk ? gend - g0 : chunk;
+    for (size_t i = 0; i + 1 < gb.size(); ++i) {
+      const int g0 = gb[i], n = gb[i + 1] - gb[i], c = c0 < 0 ? -1 : c0 + static_cast<int>(i);
       if (cudaError_t w = io_before(c)) return h->cuda_fail(w);
       ap.state0 = g0;
       int e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
@@ -933,9 +954,8 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   dp.div_heads = FastDiv(static_cast<uint32_t>(h->H));
   dp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
   __nv_bfloat16* const out0 = ap.out;
-  // (host-buffer form: the chunks of states are these groups)
-  for (int g0 = gbeg, c = gbeg / h->Sg; g0 < gend; g0 += h->Sg, ++c) {
-    const int n = gend - g0 < h->Sg ? gend - g0 : h->Sg;
+  for (size_t i = 0; i + 1 < gb.size(); ++i) {
+    const int g0 = gb[i], n = gb[i + 1] - gb[i], c = c0 < 0 ? -1 : c0 + static_cast<int>(i);
     dp.state0 = g0;
     int e = launch_dequant(h->D, dp, n, h->stream);
     if (m + w > 0) h->launches++;
@@ -973,8 +993,8 @@ int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_
 static cudaError_t copy_in_chunks(convkv_t* h, void* const* dst, const void* const* src, int nbuf, size_t bps) {
   cudaError_t e = cudaEventRecord(h->io_ev[0], h->stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_in, h->io_ev[0], 0);
-  for (int g0 = 0, c = 0; g0 < h->S && e == cudaSuccess; g0 += h->io_chunk, ++c) {
-    const int n = h->S - g0 < h->io_chunk ? h->S - g0 : h->io_chunk;
+  for (int c = 0; c < h->io_nchunks && e == cudaSuccess; ++c) {
+    const int g0 = h->io_start[c], n = h->io_start[c + 1] - g0;
     for (int i = 0; i < nbuf && e == cudaSuccess; ++i)
       e = cudaMemcpyAsync(static_cast<char*>(dst[i]) + g0 * bps, static_cast<const char*>(src[i]) + g0 * bps,
                           n * bps, cudaMemcpyHostToDevice, h->io_in);
@@ -1054,9 +1074,9 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
   h->io_defer = true;
   int rc = convkv_append_block(h, h->io_k, h->io_v, frames);
   h->io_defer = false;
-  for (int g0 = 0; rc == CONVKV_OK && g0 < h->S; g0 += h->io_chunk) {
-    const int n = h->S - g0 < h->io_chunk ? h->S - g0 : h->io_chunk;
-    rc = ring_append_states(h, h->io_ap, h->io_k, h->io_v, g0, n);
+  for (int c = 0; rc == CONVKV_OK && c < h->io_nchunks; ++c) {
+    const int g0 = h->io_start[c], n = h->io_start[c + 1] - g0;
+    rc = ring_append_states(h, h->io_ap, h->io_k, h->io_v, g0, n, c);
     if (rc == CONVKV_OK)
       rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host), g0, g0 + n);
     if (rc != CONVKV_OK) {
