@@ -282,21 +282,55 @@ const char* convkv_strerror(int code) {
   }
 }
 
-// Copy streams and events of the host-buffer entry points, and the chunks of states.
-// The first chunk is one state and each next one about 1.35 times larger (at most the
-// attention's group of states in the low-precision formats), so the kernels start
-// after one state's copy and a chunk's copy takes about as long as the previous
-// chunk's kernels (one state's copy in takes about 0.75 of its kernels' time at the
-// 480x832 shape); a short last chunk keeps the final copy back short too.
-static int create_host_io(convkv_t* h) {
-  const int cap = h->fp8 ? h->Sg : h->S;
-  h->io_start.assign(1, 0);
-  for (int n = 1; h->io_start.back() < h->S;) {
-    const int g0 = h->io_start.back();
-    h->io_start.push_back(g0 + (h->S - g0 < n ? h->S - g0 : n));
-    n = (n * 135 + 99) / 100;
-    if (n > cap) n = cap;
+// Chunks of states of the host-buffer entry points.  The first chunk is one state, so
+// the kernels start after one state's copy; each next chunk is at most 1.3 times the
+// one before, because a chunk's copy in has to land while the chunk before it computes
+// (copying one state's K, V and queries in takes about 0.77 of its kernels' time at the
+// 480x832 shape).  The steady size c (at most cap and 6) is the one whose attention
+// grid, ctas_per_state * c CTAs, leaves the smallest share of its last wave over `sms`
+// SMs idle: a chunk's kernels start only when the chunk before them has ended, so that
+// idle share is lost on every chunk.  The last chunks shrink by thirds down to one
+// state, so that after the last kernels only one state's outputs remain to copy back
+// (a state's copy back takes about a quarter of its kernels' time).
+static void plan_host_chunks(int S, int cap, int64_t ctas_per_state, int sms, std::vector<int>& start) {
+  const int hi = cap < 6 ? (cap > 0 ? cap : 1) : 6;
+  int c = 1;
+  double best = 2.0;
+  for (int n = 1; n <= hi; ++n) {
+    const int64_t w = ctas_per_state * n;
+    const double idle = static_cast<double>((w + sms - 1) / sms * sms - w) / static_cast<double>(w);
+    if (idle < best - 1e-12) {
+      best = idle;
+      c = n;
+    }
   }
+  std::vector<int> tail;
+  for (int t = c; t > 1;) {
+    t = (t + 2) / 3;
+    tail.push_back(t);
+  }
+  int tail_states = 0;
+  for (int t : tail) tail_states += t;
+  if (tail_states >= S) tail.clear(), tail_states = 0;
+  start.assign(1, 0);
+  for (int n100 = 100; start.back() < S - tail_states; n100 = n100 * 130 / 100) {
+    int n = n100 / 100;
+    if (n > c) n = c;
+    const int left = S - tail_states - start.back();
+    start.push_back(start.back() + (n < left ? n : left));
+  }
+  for (int t : tail) start.push_back(start.back() + t);
+}
+
+// Copy streams and events of the host-buffer entry points, and their chunk plan.
+static int create_host_io(convkv_t* h) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return CONVKV_ERR_CUDA;
+  // the attention launches one CTA per 256 query rows and head (steady blocks)
+  const int64_t ctas = (static_cast<int64_t>(h->bn) * h->T + 255) / 256 * h->H;
+  plan_host_chunks(h->S, h->fp8 ? h->Sg : h->S, ctas, sms, h->io_start);
   h->io_nchunks = static_cast<int>(h->io_start.size()) - 1;
   if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)

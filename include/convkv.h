@@ -130,9 +130,11 @@ int convkv_attend(convkv_t* h, const void* q, void* out);
  * inputs are copied into handle-owned device staging by chunks of states on the
  * handle's own copy stream, and each chunk's ring append or attention starts as soon
  * as that chunk has landed; attend_host copies each chunk's outputs back on a second
- * copy stream while later chunks compute (chunks: one state, then each about 1.35
- * times the previous, at most the attention's group of states in the e4m3 / NVFP4
- * formats).  Both calls return
+ * copy stream while later chunks compute (chunks: one state, then each at most 1.3
+ * times the previous up to a steady size of at most 6 states, chosen so that the
+ * attention grid of a chunk fills its last wave of SMs best, at most the attention's
+ * group of states in the e4m3 / NVFP4 formats; the last chunks shrink to one state).
+ * Both calls return
  * once the host buffers are no longer accessed: the inputs copied in, the outputs
  * copied back.  With pinned buffers the copies overlap the kernels.  Needs
  * CONVKV_FLAG_HOST_IO at create (which also creates the two copy streams and their
