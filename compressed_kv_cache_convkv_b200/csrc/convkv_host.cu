@@ -52,6 +52,12 @@ EncodeTiledFn get_encoder() {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// A unit of the host-buffer pipeline: states [g0, g0 + n) with heads [h0, h0 + nh);
+// a head range narrower than H only ever covers one state.
+struct IoChunk {
+  int g0, n, h0, nh;
+};
+
 }  // namespace
 
 struct convkv {
@@ -95,7 +101,7 @@ struct convkv {
   // copies in both directions overlap the kernels of other chunks
   cudaStream_t io_in = nullptr, io_back = nullptr;
   std::vector<cudaEvent_t> io_ev;  // [0] start, [1 + c] chunk c copied in, [1 + nchunks + c] chunk c done
-  std::vector<int> io_start;       // chunk c = states [io_start[c], io_start[c + 1])
+  std::vector<IoChunk> io_chunks;  // in stream order
   int io_nchunks = 0;
   bool io_pending = false;         // the next ring append reads io_k / io_v chunk by chunk
   bool io_defer = false;           // the ring append is left to the caller (convkv_step_host)
@@ -282,23 +288,64 @@ const char* convkv_strerror(int code) {
   }
 }
 
-// Chunks of states of the host-buffer entry points.  The first chunk is one state, so
-// the kernels start after one state's copy; each next chunk is at most 1.3 times the
-// one before, because a chunk's copy in has to land while the chunk before it computes
-// (copying one state's K, V and queries in takes about 0.77 of its kernels' time at the
-// 480x832 shape).  The steady size c (at most cap and 6) is the one whose attention
-// grid, ctas_per_state * c CTAs, leaves the smallest share of its last wave over `sms`
-// SMs idle: a chunk's kernels start only when the chunk before them has ended, so that
-// idle share is lost on every chunk.  The last chunks shrink by thirds down to one
-// state, so that after the last kernels only one state's outputs remain to copy back
-// (a state's copy back takes about a quarter of its kernels' time).
-static void plan_host_chunks(int S, int cap, int64_t ctas_per_state, int sms, std::vector<int>& start) {
+// Share of the last wave of `sms` SMs that a grid of `ctas` CTAs leaves idle.
+static double idle_share(int64_t ctas, int sms) {
+  const int64_t full = (ctas + sms - 1) / sms * sms;
+  return static_cast<double>(full - ctas) / static_cast<double>(full);
+}
+
+// Chunks of the host-buffer entry points.
+//
+// Several states: chunks of whole states.  The first chunk is one state, so the
+// kernels start after one state's copy; the sizes then follow a ramp that grows 1.3
+// times per chunk (1, 1, 1, 2, 2, 3, 4, ...), because a chunk's copy in has to land
+// while the chunks before it compute (copying one state's K, V and queries in takes
+// about 0.77 of its kernels' time at the 480x832 shape).  The steady size c (at most
+// cap and 6) is the one whose attention grid, ctas_per_head * H * c CTAs, leaves the
+// smallest share of its last wave idle: a chunk's kernels start only when the chunk
+// before them has ended, so that idle share is lost on every chunk.  The last chunks
+// shrink by thirds down to one state, so that after the last kernels only one state's
+// outputs remain to copy back (a state's copy back takes about a quarter of its
+// kernels' time).
+//
+// One state: chunks of heads, so that the copies overlap the kernels at all.  A
+// chunk's attention takes whole waves: every CTA attends one query block of one head
+// over all the keys, so a wave lasts as long as the CTAs themselves.  The group size
+// is therefore the smallest one whose grid fills its waves to at least 85 % (one wave
+// at the bench shapes: 4 heads x 32 CTAs at 512x512, 4 x 37 at 720x416, 3 x 49 at
+// 480x832), else the one up to H / 2 with the fullest waves, and at least 512 bytes of
+// a token row per strided copy (nh * D values); the last group takes the remaining
+// heads.  Small groups start the kernels early and leave little to do and to copy
+// back after the last copy in: at 512x512 the copies bound the step, at 720x416 the
+// kernels, and one wave per chunk keeps the kernels dense in both.
+static void plan_host_chunks(int S, int H, int D, int cap, int64_t ctas_per_head, int sms,
+                             std::vector<IoChunk>& out) {
+  out.clear();
+  if (S == 1 && H > 1) {
+    const int hmax = H / 2 > 1 ? H / 2 : 1;
+    int hmin = (512 + 2 * D - 1) / (2 * D);
+    if (hmin > hmax) hmin = hmax;
+    int hg = hmin;
+    double best = -1.0;
+    for (int n = hmin; n <= hmax; ++n) {
+      const double fill = 1.0 - idle_share(ctas_per_head * n, sms);
+      if (fill >= 0.85) {
+        hg = n;
+        break;
+      }
+      if (fill > best + 1e-12) {
+        best = fill;
+        hg = n;
+      }
+    }
+    for (int h0 = 0; h0 < H; h0 += hg) out.push_back({0, 1, h0, H - h0 < hg ? H - h0 : hg});
+    return;
+  }
   const int hi = cap < 6 ? (cap > 0 ? cap : 1) : 6;
   int c = 1;
   double best = 2.0;
   for (int n = 1; n <= hi; ++n) {
-    const int64_t w = ctas_per_state * n;
-    const double idle = static_cast<double>((w + sms - 1) / sms * sms - w) / static_cast<double>(w);
+    const double idle = idle_share(ctas_per_head * H * n, sms);
     if (idle < best - 1e-12) {
       best = idle;
       c = n;
@@ -312,14 +359,18 @@ static void plan_host_chunks(int S, int cap, int64_t ctas_per_state, int sms, st
   int tail_states = 0;
   for (int t : tail) tail_states += t;
   if (tail_states >= S) tail.clear(), tail_states = 0;
-  start.assign(1, 0);
-  for (int n100 = 100; start.back() < S - tail_states; n100 = n100 * 130 / 100) {
+  int g0 = 0;
+  for (int n100 = 100; g0 < S - tail_states; n100 = n100 * 130 / 100) {
     int n = n100 / 100;
     if (n > c) n = c;
-    const int left = S - tail_states - start.back();
-    start.push_back(start.back() + (n < left ? n : left));
+    if (n > S - tail_states - g0) n = S - tail_states - g0;
+    out.push_back({g0, n, 0, H});
+    g0 += n;
   }
-  for (int t : tail) start.push_back(start.back() + t);
+  for (int t : tail) {
+    out.push_back({g0, t, 0, H});
+    g0 += t;
+  }
 }
 
 // Copy streams and events of the host-buffer entry points, and their chunk plan.
@@ -329,9 +380,9 @@ static int create_host_io(convkv_t* h) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
     return CONVKV_ERR_CUDA;
   // the attention launches one CTA per 256 query rows and head (steady blocks)
-  const int64_t ctas = (static_cast<int64_t>(h->bn) * h->T + 255) / 256 * h->H;
-  plan_host_chunks(h->S, h->fp8 ? h->Sg : h->S, ctas, sms, h->io_start);
-  h->io_nchunks = static_cast<int>(h->io_start.size()) - 1;
+  const int64_t ctas = (static_cast<int64_t>(h->bn) * h->T + 255) / 256;
+  plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, ctas, sms, h->io_chunks);
+  h->io_nchunks = static_cast<int>(h->io_chunks.size());
   if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)
     return CONVKV_ERR_CUDA;
@@ -387,7 +438,17 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   h->prerot = !h->fp8;
   h->stream = static_cast<cudaStream_t>(cfg->stream);
   h->cfg.conv_weight = nullptr;
+  // e4m3 / NVFP4: the dequantisation scratch holds up to 4 GiB of states at a time
+  if (h->fp8) {
+    const size_t per_state = static_cast<size_t>(h->C + h->W) * h->frame_elems() * 2 * 2;
+    const size_t budget = size_t(4) << 30;
+    h->Sg = static_cast<int>(per_state * h->S <= budget ? h->S : (budget / per_state > 0 ? budget / per_state : 1));
+  }
   if (h->dry) {
+    // the host-buffer chunk plan only, for a B200's 148 SMs (no device is queried)
+    if (h->host_io)
+      plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, (static_cast<int64_t>(h->bn) * h->T + 255) / 256,
+                       148, h->io_chunks);
     *out = h;
     return CONVKV_OK;
   }
@@ -412,12 +473,6 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
   const size_t sink_b = static_cast<size_t>(h->S) * h->Rs * fe * 2;
   const size_t rkr_b = h->prerot ? ring_b : 0;
   const size_t mkr_b = h->prerot ? mem_b : 0;
-  // e4m3 / NVFP4: the dequantisation scratch holds up to 4 GiB of states at a time
-  if (h->fp8) {
-    const size_t per_state = static_cast<size_t>(h->C + h->W) * fe * 2 * 2;
-    const size_t budget = size_t(4) << 30;
-    h->Sg = static_cast<int>(per_state * h->S <= budget ? h->S : (budget / per_state > 0 ? budget / per_state : 1));
-  }
   const size_t scr_b = h->fp8 ? static_cast<size_t>(h->Sg) * (h->C + h->W) * fe * 2 : 0;
   // e4m3 / NVFP4: the conv's fp32 outputs for the groups of one append (the window
   // holds at most W + Bmax frames before an append's evictions, so at most
@@ -607,17 +662,20 @@ static AppendParams states_slice(const convkv_t* h, const AppendParams& a, int g
   return p;
 }
 
-// Step 4 of the append for states [g0, g0 + n): the new block into the ring (and the
-// rotated K / the staging copy).  With host buffers arriving by chunks (c >= 0: the
-// chunk of these states), it first waits for the chunk's copy.
-static int ring_append_states(convkv_t* h, const AppendParams& ap, const void* k, const void* v, int g0, int n,
-                              int c) {
+// Step 4 of the append for the states and heads of chunk `ck`: the new block into the
+// ring (and the rotated K / the staging copy).  With host buffers arriving by chunks
+// (c >= 0: the chunk's index), it first waits for the chunk's copy.
+static int ring_append_chunk(convkv_t* h, const AppendParams& ap, const void* k, const void* v, const IoChunk& ck,
+                             int c) {
   if (c >= 0) {
     cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0);
     if (w != cudaSuccess) return h->cuda_fail(w);
   }
-  const int frames = ap.b;
-  const AppendParams a = states_slice(h, ap, g0, n, frames);
+  const int frames = ap.b, g0 = ck.g0;
+  AppendParams a = states_slice(h, ap, g0, ck.n, frames);
+  a.h0 = ck.h0;
+  a.nh = ck.nh;
+  a.div_nh = FastDiv(static_cast<uint32_t>(ck.nh));
   const int64_t in_off = static_cast<int64_t>(g0) * frames * h->frame_elems() * 2;
   const void* kc = k ? static_cast<const char*>(k) + in_off : nullptr;
   const void* vc = v ? static_cast<const char*>(v) + in_off : nullptr;
@@ -760,11 +818,11 @@ static int append_steps(convkv_t* h, const void* k, const void* v, const void* c
     h->io_ap = ap;
     return CONVKV_OK;
   }
-  // one launch set for all states, or (host buffers arriving chunk by chunk) one per
-  // chunk of states, each after its chunk's copy
-  if (!h->io_pending) return ring_append_states(h, ap, k, v, 0, h->S, -1);
+  // one launch set for all states and heads, or (host buffers arriving chunk by chunk)
+  // one per chunk, each after its chunk's copy
+  if (!h->io_pending) return ring_append_chunk(h, ap, k, v, IoChunk{0, h->S, 0, h->H}, -1);
   for (int c = 0; c < h->io_nchunks; ++c)
-    if (int rc = ring_append_states(h, ap, k, v, h->io_start[c], h->io_start[c + 1] - h->io_start[c], c)) return rc;
+    if (int rc = ring_append_chunk(h, ap, k, v, h->io_chunks[c], c)) return rc;
   return CONVKV_OK;
 }
 
@@ -839,12 +897,26 @@ int convkv_set_sink(convkv_t* h, const void* k, const void* v) {
   return CONVKV_OK;
 }
 
-// out_host: the host-buffer form (queries copied in by chunks of states, see
+// Copy of chunk ck's rows of a [S][rows][H][D] bf16 tensor (bps bytes per state)
+// between host and device: one contiguous copy for whole states, a strided one (one
+// row of nh * D values per token) for a head range.
+static cudaError_t copy_chunk(const convkv_t* h, const IoChunk& ck, void* dst, const void* src, size_t bps,
+                              cudaMemcpyKind kind, cudaStream_t st) {
+  const size_t off = static_cast<size_t>(ck.g0) * bps;
+  if (ck.nh == h->H)
+    return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, ck.n * bps, kind, st);
+  const size_t row = static_cast<size_t>(h->H) * h->D * 2;
+  const size_t col = static_cast<size_t>(ck.h0) * h->D * 2;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + off + col, row, static_cast<const char*>(src) + off + col, row,
+                           static_cast<size_t>(ck.nh) * h->D * 2, bps / row, kind, st);
+}
+
+// out_host: the host-buffer form (queries copied in by chunks, see
 // convkv_attend_host); each chunk's attention waits for its queries, and its outputs
-// are copied back to out_host as soon as it ends.
+// are copied back to out_host as soon as it ends.  [cbeg, cend): the chunks attended
+// by this call.
 static int attend_impl(convkv_t* h, const void* q, void* out, const void* const* q_sh, void* const* o_sh,
-                       char* out_host = nullptr, int gbeg = 0, int gend = -1) {
-  if (gend < 0) gend = h->S;
+                       char* out_host = nullptr, int cbeg = 0, int cend = -1) {
   const int r = h->Rs, m = h->m(), w = h->w(), b = h->bcur, T = h->T;
   AttnParams ap{};
   ap.H = h->H;
@@ -919,39 +991,38 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   auto io_before = [&](int c) -> cudaError_t {
     return c >= 0 ? cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0) : cudaSuccess;
   };
-  auto io_after = [&](int c, int g0, int n) -> cudaError_t {
+  auto io_after = [&](int c) -> cudaError_t {
     if (c < 0) return cudaSuccess;
     cudaEvent_t done = h->io_ev[1 + h->io_nchunks + c];
     cudaError_t e = cudaEventRecord(done, h->stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, done, 0);
-    if (e == cudaSuccess)
-      e = cudaMemcpyAsync(out_host + g0 * bps, static_cast<char*>(out) + g0 * bps, n * bps, cudaMemcpyDeviceToHost,
-                          h->io_back);
+    if (e == cudaSuccess) e = copy_chunk(h, h->io_chunks[c], out_host, out, bps, cudaMemcpyDeviceToHost, h->io_back);
     return e;
   };
-  // the launch groups: the host-buffer chunks in [gbeg, gend) (chunk index c), else
-  // all states at once (bf16) or groups of Sg states (the scratch's capacity)
-  std::vector<int> gb;   // group starts, then gend
-  int c0 = -1;
+  // the launches: the host-buffer chunks [cbeg, cend) (index c), else all states at
+  // once (bf16) or groups of Sg states (the scratch's capacity), with every head
+  struct Unit {
+    IoChunk ck;
+    int c;
+  };
+  std::vector<Unit> units;
   if (out_host) {
-    for (int c = 0; c < h->io_nchunks; ++c) {
-      if (h->io_start[c] < gbeg || h->io_start[c] >= gend) continue;
-      if (c0 < 0) c0 = c;
-      gb.push_back(h->io_start[c]);
-    }
+    if (cend < 0) cend = h->io_nchunks;
+    for (int c = cbeg; c < cend; ++c) units.push_back({h->io_chunks[c], c});
   } else {
-    for (int g0 = gbeg; g0 < gend; g0 += h->fp8 ? h->Sg : h->S) gb.push_back(g0);
+    const int step = h->fp8 ? h->Sg : h->S;
+    for (int g0 = 0; g0 < h->S; g0 += step) units.push_back({{g0, h->S - g0 < step ? h->S - g0 : step, 0, h->H}, -1});
   }
-  gb.push_back(gend);
   if (!h->fp8) {
-    for (size_t i = 0; i + 1 < gb.size(); ++i) {
-      const int g0 = gb[i], n = gb[i + 1] - gb[i], c = c0 < 0 ? -1 : c0 + static_cast<int>(i);
-      if (cudaError_t w = io_before(c)) return h->cuda_fail(w);
-      ap.state0 = g0;
-      int e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
+    for (const Unit& u : units) {
+      if (cudaError_t w = io_before(u.c)) return h->cuda_fail(w);
+      ap.state0 = u.ck.g0;
+      ap.head0 = u.ck.h0;
+      ap.nheads = u.ck.nh;
+      int e = launch_attend(h->D, ap, mq, km, vm, u.ck.n, h->stream);
       h->launches++;
       if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
-      if (cudaError_t w = io_after(c, g0, n)) return h->cuda_fail(w);
+      if (cudaError_t w = io_after(u.c)) return h->cuda_fail(w);
     }
     return CONVKV_OK;
   }
@@ -987,20 +1058,23 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   dp.tab_h_rows = h->gh;
   dp.div_heads = FastDiv(static_cast<uint32_t>(h->H));
   dp.div_grid_w = FastDiv(static_cast<uint32_t>(h->gw));
-  __nv_bfloat16* const out0 = ap.out;
-  for (size_t i = 0; i + 1 < gb.size(); ++i) {
-    const int g0 = gb[i], n = gb[i + 1] - gb[i], c = c0 < 0 ? -1 : c0 + static_cast<int>(i);
-    dp.state0 = g0;
-    int e = launch_dequant(h->D, dp, n, h->stream);
-    if (m + w > 0) h->launches++;
-    if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
-    if (cudaError_t wt = io_before(c)) return h->cuda_fail(wt);
-    ap.state0 = g0;
-    ap.out = out0;
-    e = launch_attend(h->D, ap, mq, km, vm, n, h->stream);
+  for (const Unit& u : units) {
+    int e = 0;
+    if (u.ck.h0 == 0) {
+      // every head of the unit's states; a state's later head chunks reuse its scratch
+      dp.state0 = u.ck.g0;
+      e = launch_dequant(h->D, dp, u.ck.n, h->stream);
+      if (m + w > 0) h->launches++;
+      if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+    }
+    if (cudaError_t wt = io_before(u.c)) return h->cuda_fail(wt);
+    ap.state0 = u.ck.g0;
+    ap.head0 = u.ck.h0;
+    ap.nheads = u.ck.nh;
+    e = launch_attend(h->D, ap, mq, km, vm, u.ck.n, h->stream);
     h->launches++;
     if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
-    if (cudaError_t wt = io_after(c, g0, n)) return h->cuda_fail(wt);
+    if (cudaError_t wt = io_after(u.c)) return h->cuda_fail(wt);
   }
   return CONVKV_OK;
 }
@@ -1028,10 +1102,8 @@ static cudaError_t copy_in_chunks(convkv_t* h, void* const* dst, const void* con
   cudaError_t e = cudaEventRecord(h->io_ev[0], h->stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_in, h->io_ev[0], 0);
   for (int c = 0; c < h->io_nchunks && e == cudaSuccess; ++c) {
-    const int g0 = h->io_start[c], n = h->io_start[c + 1] - g0;
     for (int i = 0; i < nbuf && e == cudaSuccess; ++i)
-      e = cudaMemcpyAsync(static_cast<char*>(dst[i]) + g0 * bps, static_cast<const char*>(src[i]) + g0 * bps,
-                          n * bps, cudaMemcpyHostToDevice, h->io_in);
+      e = copy_chunk(h, h->io_chunks[c], dst[i], src[i], bps, cudaMemcpyHostToDevice, h->io_in);
     if (e == cudaSuccess) e = cudaEventRecord(h->io_ev[1 + c], h->io_in);
   }
   return e;
@@ -1100,8 +1172,8 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
     return h->cuda_fail(e);
   }
   // bookkeeping, conv, time table and key rotation for all states (while the block is
-  // copied in); then per chunk of states: its ring append, its attention, its outputs
-  // back -- a chunk's kernels wait only for its own inputs
+  // copied in); then per chunk (of states, or of one state's heads): its ring append,
+  // its attention, its outputs back -- a chunk's kernels wait only for its own inputs
   const int64_t P = h->P, E = h->E, Sn = h->Sn, blocks = h->blocks;
   const int bcur = h->bcur, last_groups = h->last_groups;
   h->io_pending = true;
@@ -1109,10 +1181,9 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
   int rc = convkv_append_block(h, h->io_k, h->io_v, frames);
   h->io_defer = false;
   for (int c = 0; rc == CONVKV_OK && c < h->io_nchunks; ++c) {
-    const int g0 = h->io_start[c], n = h->io_start[c + 1] - g0;
-    rc = ring_append_states(h, h->io_ap, h->io_k, h->io_v, g0, n, c);
+    rc = ring_append_chunk(h, h->io_ap, h->io_k, h->io_v, h->io_chunks[c], c);
     if (rc == CONVKV_OK)
-      rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host), g0, g0 + n);
+      rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host), c, c + 1);
     if (rc != CONVKV_OK) {
       // as a failed append (later chunks are not appended): counters back, attends
       // refused until an append succeeds, which rewrites the same ring slots
@@ -1134,6 +1205,19 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
   if (e2 != cudaSuccess) return h->cuda_fail(e2);
   if (e3 != cudaSuccess) return h->cuda_fail(e3);
   return CONVKV_OK;
+}
+
+int convkv_host_chunks(const convkv_t* h, int32_t* rec, int cap) {
+  if (!h || (cap > 0 && !rec) || cap < 0) return CONVKV_ERR_INVALID_ARG;
+  const int n = static_cast<int>(h->io_chunks.size());
+  for (int c = 0; c < n && c < cap; ++c) {
+    const IoChunk& k = h->io_chunks[c];
+    rec[4 * c] = k.g0;
+    rec[4 * c + 1] = k.n;
+    rec[4 * c + 2] = k.h0;
+    rec[4 * c + 3] = k.nh;
+  }
+  return n;
 }
 
 int convkv_layout(const convkv_t* h, int32_t* rec, int cap) {

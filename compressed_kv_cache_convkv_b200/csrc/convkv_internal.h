@@ -84,6 +84,7 @@ struct AttnParams {
   __nv_bfloat16* out;     // [S][Nq][H][D]
   float q_scale;          // log2(e) / sqrt(D), folded into the rotated queries
   int state0;             // first state of the launch's group (grid z walks the group)
+  int head0, nheads;      // heads [head0, head0 + nheads) (grid y); nheads 0: all H
   int* status;
   // sequence-sharded queries and outputs (sv.G > 0): rows of the block are read from
   // and written to the G ranks' shards (peer memory on a multi-GPU node)
@@ -118,6 +119,9 @@ struct ConvParams {
 struct AppendParams {
   int S, b, R, slot0;         // states, frames, ring frames, ring slot of frame 0
   int64_t frame_elems;        // T * H * D
+  // heads [h0, h0 + nh) of each token are appended (nh >= 1); div_nh divides by nh
+  int h0, nh;
+  FastDiv div_nh;
   // fp8 format
   int H, D;
   unsigned int* amax;         // [S][2][b][H] fp32 bit patterns (scratch, zeroed before the amax pass)

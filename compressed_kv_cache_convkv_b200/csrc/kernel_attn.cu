@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // sl: the state within this launch's group (coordinate of the group-local scratch);
   // state: its index in the handle (queries, outputs, staging, reference frames)
-  const int head = blockIdx.y, sl = blockIdx.z, state = sl + p.state0;
+  const int head = p.head0 + blockIdx.y, sl = blockIdx.z, state = sl + p.state0;
   const int q_row0 = blockIdx.x * (C::QT * C::BM);
 
   if (threadIdx.x == 0) {
@@ -458,7 +458,7 @@ int launch_t(const AttnParams& p, const CUtensorMap& q, const CUtensorMap* k, co
   auto kern = attn_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid((p.Nq + 255) / 256, p.H, S);
+  dim3 grid((p.Nq + 255) / 256, p.nheads > 0 ? p.nheads : p.H, S);
   kern<<<grid, AttnCfg<D>::THREADS, smem, s>>>(q, k[0], v[0], k[1], v[1], k[2], v[2], k[3], v[3], p);
   return static_cast<int>(cudaGetLastError());
 }

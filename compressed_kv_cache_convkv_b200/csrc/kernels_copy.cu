@@ -82,25 +82,29 @@ __device__ __forceinline__ dev::RopeRow rope_row_of(const float4* tables, int ta
   return dev::RopeRow{tables + static_cast<int64_t>(t_row) * RC::UT, tab_h + y * RC::UH, tab_w + x * RC::UW};
 }
 
-// grid = (x, states * b): y is the frame, x walks its 16-byte vectors.
+// grid = (x, states * b): y is the frame, x walks the 16-byte vectors of its heads
+// [h0, h0 + nh).
 template <int D>
 __global__ void append_bf16_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                    uint4* __restrict__ ringK, uint4* __restrict__ ringV, AppendParams p) {
   constexpr int DV = D / 8;               // 16-byte vectors per head
   const int fv = static_cast<int>(p.frame_elems / 8);  // 16-byte vectors per frame
+  const int nv = fv / p.H * p.nh;         // vectors of the appended heads per frame
   const int sf = blockIdx.y;              // state * b + frame
   const int s = sf / p.b;
   const int f = sf - s * p.b;
   int slot = p.slot0 + f;
   if (slot >= p.R) slot -= p.R;
   const int64_t dst0 = (static_cast<int64_t>(s) * p.R + slot) * fv;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < fv; e += gridDim.x * blockDim.x) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += gridDim.x * blockDim.x) {
+    const int ht = i / DV;                // token * nh + (head - h0)
+    const int tok = p.div_nh.div(ht);
+    const int e = (tok * p.H + p.h0 + (ht - tok * p.nh)) * DV + (i & (DV - 1));
     const uint4 kv = __ldcs(block_vec(k, p.k_sh, p, s, f, e));
     const uint4 vv = __ldcs(block_vec(v, p.v_sh, p, s, f, e));
     ringK[dst0 + e] = kv;
     ringV[dst0 + e] = vv;
     if (p.ringKr) {
-      const int tok = p.div_heads.div(e / DV);
       const dev::RopeRow rr =
           rope_row_of<D>(p.tables, p.tab_t_rows, p.tab_h_rows, p.div_grid_w, p.grid_w, p.t_row0 + f, tok);
       uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -231,7 +235,8 @@ template <int D>
 __global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   constexpr int DV = D / 8;                       // lanes (vectors) per head
   constexpr int U = 4;                            // loads in flight per thread
-  const int HDV = p.H * DV;
+  const int HDV = p.H * DV;                       // vectors per token
+  const int NDV = p.nh * DV;                      // columns: the heads [h0, h0 + nh)
   const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
@@ -239,17 +244,18 @@ __global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uin
   const int kv = blockIdx.z;
   const int lane = threadIdx.x & 31;
   unsigned int* amax_f = p.amax + ((static_cast<int64_t>(s) * 2 + kv) * p.b + f) * p.H;
-  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int slabs = (NDV + blockDim.x - 1) / blockDim.x;
   const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
   const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  const int col = p.h0 * DV + hc;                 // the column within the token
   uint32_t m = 0;
-  if (hc < HDV) {
+  if (hc < NDV) {
     for (int tok0 = walker; tok0 < T; tok0 += U * walkers) {
       uint4 x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int tok = tok0 + u * walkers;
-        x[u] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + hc))
+        x[u] = tok < T ? __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, static_cast<int64_t>(tok) * HDV + col))
                        : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
@@ -266,7 +272,7 @@ __global__ void append_amax_frames_kernel(const uint4* __restrict__ k, const uin
   // heads start at multiples of DV columns, slabs at multiples of 32, and DV divides 32
 #pragma unroll
   for (int o = DV / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (hc < HDV && (lane % DV) == 0 && m) atomicMax(&amax_f[hc / DV], m);
+  if (hc < NDV && (lane % DV) == 0 && m) atomicMax(&amax_f[col / DV], m);
 }
 
 // The block's K row chunk as written to staging: rotated at its stream position
@@ -291,7 +297,8 @@ template <int D>
 __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   constexpr int DV = D / 8;
   constexpr int U = 2;                            // loads in flight per thread
-  const int HDV = p.H * DV;
+  const int HDV = p.H * DV;                       // vectors per token
+  const int NDV = p.nh * DV;                      // columns: the heads [h0, h0 + nh)
   const int T = static_cast<int>(p.frame_elems / HDV / 8);
   const int fv = static_cast<int>(p.frame_elems / 8);
   const int sf = blockIdx.y;
@@ -304,10 +311,10 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   uint2* codes = reinterpret_cast<uint2*>(p.ring8[kv]) + (static_cast<int64_t>(s) * p.R + slot) * fv;
   const SharedDivisor d448 = make_divisor(448.0f);
-  const int slabs = (HDV + blockDim.x - 1) / blockDim.x;
+  const int slabs = (NDV + blockDim.x - 1) / blockDim.x;
   const int walker = blockIdx.x / slabs, walkers = gridDim.x / slabs;
-  const int hc = (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
-  if (hc < HDV) {
+  const int hc = p.h0 * DV + (blockIdx.x - walker * slabs) * blockDim.x + threadIdx.x;
+  if (hc < (p.h0 + p.nh) * DV) {
     const int h = hc / DV;
     const int c = hc - h * DV;
     const float amax = __uint_as_float(amax_f[h]);
@@ -353,12 +360,13 @@ __global__ void append_quant_kernel(const uint4* __restrict__ k, const uint4* __
 // NVFP4 pass 2: one thread per 16-channel block of a token's head: block scale,
 // e2m1 codes into the ring, the bf16 values into staging (K rotated), the tensor
 // scale once.
-// grid = (x, states * b, 2 (K|V)); x walks the frame's 16-channel blocks.
+// grid = (x, states * b, 2 (K|V)); x walks the 16-channel blocks of the frame's heads
+// [h0, h0 + nh).
 template <int D>
 __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, AppendParams p) {
   constexpr int NB = D / fp4::kBlock;                      // blocks per token-head
   const int fv = static_cast<int>(p.frame_elems / 8);
-  const int per_frame = static_cast<int>(p.frame_elems / fp4::kBlock);
+  const int per_frame = static_cast<int>(p.frame_elems / fp4::kBlock / p.H * p.nh);
   const int sf = blockIdx.y;
   const int s = sf / p.b;
   const int f = sf - s * p.b;
@@ -370,13 +378,14 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
   uint4* stage = reinterpret_cast<uint4*>(p.stage[kv]) + (static_cast<int64_t>(s) * p.stage_frames + f) * fv;
   const int64_t row0 = (static_cast<int64_t>(s) * p.R + slot) * T * p.H;   // first token-head row of the slot
   for (int ib = blockIdx.x * blockDim.x + threadIdx.x; ib < per_frame; ib += gridDim.x * blockDim.x) {
-    const int th = ib / NB;                                    // token * H + h
-    const int blk = ib - th * NB;
-    const int h = th - p.div_heads.div(th) * p.H;
+    const int tl = ib / NB;                                    // token * nh + (h - h0)
+    const int blk = ib - tl * NB;
+    const int tok = p.div_nh.div(tl);
+    const int h = p.h0 + (tl - tok * p.nh);
+    const int th = tok * p.H + h;                              // token * H + h
     const int e0 = th * (D / 8) + blk * 2;                     // first 16-byte vector of the block
     const uint4 x0 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0));
     const uint4 x1 = __ldg(block_vec(kv ? v : k, kv ? p.v_sh : p.k_sh, p, s, f, e0 + 1));
-    const int tok = p.div_heads.div(th);
     stage[e0] = kv == 0 ? staged_k<D>(x0, p, f, tok, 2 * blk) : x0;
     stage[e0 + 1] = kv == 0 ? staged_k<D>(x1, p, f, tok, 2 * blk + 1) : x1;
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -394,7 +403,7 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
     const int64_t row = row0 + th;                              // token-head row in the ring
     reinterpret_cast<uint2*>(p.ring8[kv])[row * NB + blk] = fp4::encode_block(xs, e_b);
     p.ring_bs[kv][row * NB + blk] = static_cast<uint8_t>(sc);
-    if (th < p.H && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
+    if (tok == 0 && blk == 0) p.ring_scale[((static_cast<int64_t>(s) * 2 + kv) * p.R + slot) * p.H + h] = g;
   }
 }
 
@@ -402,8 +411,9 @@ __global__ void append_quant_fp4_kernel(const uint4* __restrict__ k, const uint4
 
 int launch_append_bf16(const AppendParams& p, const void* k, const void* v, void* ringK, void* ringV,
                        cudaStream_t s) {
+  if (p.nh < 1 || p.h0 < 0 || p.h0 + p.nh > p.H) return static_cast<int>(cudaErrorInvalidValue);
   auto kern = p.D == 128 ? append_bf16_kernel<128> : append_bf16_kernel<64>;
-  dim3 grid(frame_grid_x(p.frame_elems / 8, p.S * p.b, 256), p.S * p.b);
+  dim3 grid(frame_grid_x(p.frame_elems / 8 / p.H * p.nh, p.S * p.b, 256), p.S * p.b);
   kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(ringK),
                             static_cast<uint4*>(ringV), p);
   return static_cast<int>(cudaGetLastError());
@@ -436,25 +446,26 @@ int launch_mean_bf16(int D, const ConvParams& p, const void* ringK, const void* 
 }
 
 int launch_append_fp8(const AppendParams& p, const void* k, const void* v, cudaStream_t s) {
+  if (p.nh < 1 || p.h0 < 0 || p.h0 + p.nh > p.H) return static_cast<int>(cudaErrorInvalidValue);
   cudaError_t e = cudaMemsetAsync(p.amax, 0, sizeof(unsigned int) * p.S * 2 * p.b * p.H, s);
   if (e != cudaSuccess) return static_cast<int>(e);
   {
     auto kern = p.D == 128 ? append_amax_frames_kernel<128> : append_amax_frames_kernel<64>;
     const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-    dim3 g1(token_grid_x(T, p.H * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
+    dim3 g1(token_grid_x(T, p.nh * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
     kern<<<g1, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   if (p.fp4) {
     auto kern = p.D == 128 ? append_quant_fp4_kernel<128> : append_quant_fp4_kernel<64>;
-    dim3 grid(frame_grid_x(p.frame_elems / fp4::kBlock, 2 * p.S * p.b, 256), p.S * p.b, 2);
+    dim3 grid(frame_grid_x(p.frame_elems / fp4::kBlock / p.H * p.nh, 2 * p.S * p.b, 256), p.S * p.b, 2);
     kern<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
     return static_cast<int>(cudaGetLastError());
   }
   auto kern = p.D == 128 ? append_quant_kernel<128> : append_quant_kernel<64>;
   const int T = static_cast<int>(p.frame_elems / (static_cast<int64_t>(p.H) * p.D));
-  dim3 grid(token_grid_x(T, p.H * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
+  dim3 grid(token_grid_x(T, p.nh * (p.D / 8), 2 * p.S * p.b), p.S * p.b, 2);
   kern<<<grid, kTokenThreads, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v), p);
   return static_cast<int>(cudaGetLastError());
 }

@@ -130,11 +130,12 @@ int convkv_attend(convkv_t* h, const void* q, void* out);
  * inputs are copied into handle-owned device staging by chunks of states on the
  * handle's own copy stream, and each chunk's ring append or attention starts as soon
  * as that chunk has landed; attend_host copies each chunk's outputs back on a second
- * copy stream while later chunks compute (chunks: one state, then each at most 1.3
- * times the previous up to a steady size of at most 6 states, chosen so that the
+ * copy stream while later chunks compute (chunks: one state, then sizes growing 1.3
+ * times per chunk up to a steady size of at most 6 states, chosen so that the
  * attention grid of a chunk fills its last wave of SMs best, at most the attention's
- * group of states in the e4m3 / NVFP4 formats; the last chunks shrink to one state).
- * Both calls return
+ * group of states in the e4m3 / NVFP4 formats; the last chunks shrink to one state.
+ * A handle of one state is chunked by ranges of heads instead: see
+ * convkv_host_chunks).  Both calls return
  * once the host buffers are no longer accessed: the inputs copied in, the outputs
  * copied back.  With pinned buffers the copies overlap the kernels.  Needs
  * CONVKV_FLAG_HOST_IO at create (which also creates the two copy streams and their
@@ -211,6 +212,14 @@ int convkv_ipc_close(void* dev_ptr);
  * current block, or reference frame), RoPE time index}.  Returns the number of
  * key frames, or a negative error; writes at most `cap` records. */
 int convkv_layout(const convkv_t* h, int32_t* rec, int cap);
+
+/* Chunk plan of the host-buffer entry points, in stream order, 4 int32 per chunk:
+ * {first state, states, first head, heads}.  With several states the chunks are
+ * whole states (all heads); with one state they are ranges of its heads (strided
+ * copies of nh * D values per token).  A handle created with CONVKV_FLAG_HOST_IO has
+ * the plan (a dry-run handle too, planned for 148 SMs); any other handle has none.
+ * Returns the number of chunks, or a negative error; writes at most `cap` records. */
+int convkv_host_chunks(const convkv_t* h, int32_t* rec, int cap);
 
 /* Counters {P promoted frames, E evicted frames, S slots produced, m stored
  * slots, w window frames, b current frames, blocks appended, groups compressed

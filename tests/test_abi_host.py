@@ -7,6 +7,7 @@ with the closed form of the eviction rule, for every block of every workload.
 import ctypes
 import math
 import re
+from dataclasses import replace
 
 import numpy as np
 import pytest
@@ -261,3 +262,58 @@ def test_noalloc_quantiser_rejects_misaligned_pointers_before_any_work():
     good = 1 << 20
     for x, c, s in [(good + 8, good, good), (good, good + 4, good), (good, good, good + 2)]:
         assert lib.convkv_quantize_e4m3_noalloc(x, c, s, 1, 16, 2, 64, None) == ckv.ERR_INVALID_ARG
+
+
+def _plan(w, **kw):
+    return _dry(w, host_io=True, **kw).host_chunks().tolist()
+
+
+def test_host_chunk_plan_covers_every_state_and_head_once():
+    """The host-buffer chunk plan (convkv_host_chunks, computed on the host for 148
+    SMs): every (state, head) pair lies in exactly one chunk, in stream order; whole
+    states with several states, ranges of heads with one state."""
+    cases = [(PRESETS[n], {}) for n in ("tiny", "512x512", "720x416", "fp8_480x832", "nvfp4_480x832")]
+    cases += [(replace(PRESETS["fp8_480x832"], num_states=s), {}) for s in (1, 2, 7, 8, 13)]
+    cases += [(replace(PRESETS["tiny"], num_states=s), {}) for s in (1, 2, 3, 5)]
+    cases += [(replace(PRESETS["512x512"], num_states=s), {}) for s in (2, 40)]
+    for w, kw in cases:
+        plan = _plan(w, **kw)
+        H, S = w.heads, w.num_states
+        seen = np.zeros((S, H), dtype=int)
+        for g0, n, h0, nh in plan:
+            assert n >= 1 and nh >= 1
+            if nh < H:
+                assert n == 1, (w.name, plan)
+            seen[g0:g0 + n, h0:h0 + nh] += 1
+        assert (seen == 1).all(), (w.name, S, plan)
+        flat = [(g0, h0) for g0, _, h0, _ in plan]
+        assert flat == sorted(flat), plan
+        if S > 1:
+            assert all(nh == H for _, _, _, nh in plan)
+            sizes = [n for _, n, _, _ in plan]
+            assert sizes[0] == 1 and sizes[-1] == 1, sizes
+        elif H > 1:
+            assert len(plan) >= 2
+    # a handle without host buffers has no plan
+    assert _dry(PRESETS["tiny"]).host_chunks().shape == (0, 4)
+
+
+def test_host_chunk_plan_fills_waves_at_the_bench_shapes():
+    """At the bench shapes the plan's attention grids fill their waves of 148 SMs:
+    480x832 x 40 states in steady chunks of 4 states (4 x 1,960 CTAs = 53 waves, 0.06 %
+    idle); one state in ranges of heads that make one wave each: 4 heads x 32 CTAs at
+    512x512 (86 % full), 4 x 37 at 720x416 (full), 3 x 49 at 480x832 (99 %).  Head
+    ranges are at least 512 bytes per token row."""
+    fp8 = _plan(PRESETS["fp8_480x832"])
+    assert [n for _, n, _, _ in fp8] == [1, 1, 1, 2, 2, 3, 4, 4, 4, 4, 4, 4, 3, 2, 1]
+    assert max(n for _, n, _, _ in fp8) <= 7        # the e4m3 dequantisation group
+    assert _plan(PRESETS["512x512"]) == [[0, 1, h, 4] for h in range(0, 40, 4)]
+    assert _plan(PRESETS["720x416"]) == [[0, 1, h, 4] for h in range(0, 40, 4)]
+    one = _plan(replace(PRESETS["fp8_480x832"], num_states=1))
+    assert one == [[0, 1, h, 3] for h in range(0, 39, 3)] + [[0, 1, 39, 1]]
+    for w in (PRESETS["512x512"], PRESETS["720x416"], replace(PRESETS["fp8_480x832"], num_states=1)):
+        per_head = -(-w.block_frames * w.T // 256)
+        nh = _plan(w)[0][3]
+        ctas = per_head * nh
+        assert ctas <= 148 and ctas / 148 >= 0.85
+        assert nh * w.head_dim * 2 >= 512

@@ -1,13 +1,15 @@
 """The host-buffer entry points (convkv_append_block_host / convkv_attend_host) against
 the device-buffer ones, on the GPU.
 
-The host forms copy their inputs in by chunks of states on a copy stream, start each
-chunk's kernels as soon as its copy lands, and copy each chunk's outputs back while
-later chunks compute; convkv_step_host does an append and an attend in one such
-pipelined call.  The kernels and their arithmetic are the same as in the device
-forms, so the outputs must be identical bit for bit, for several chunks: a bf16 handle
-of 3 states (three chunks) and an e4m3 handle of 8 states at 480x832 (two groups of
-states, hence two chunks, under the 4 GiB dequantisation scratch).
+The host forms copy their inputs in by chunks on a copy stream, start each chunk's
+kernels as soon as its copy lands, and copy each chunk's outputs back while later
+chunks compute; convkv_step_host does an append and an attend in one such pipelined
+call.  The kernels and their arithmetic are the same as in the device forms, so the
+outputs must be identical bit for bit, for several chunks: a bf16 handle of 3 states
+(three chunks), an e4m3 handle of 8 states at 480x832 (chunks of 1 to 2 states, under
+the 4 GiB dequantisation scratch), and handles of one state, whose chunks are ranges
+of heads copied with strided copies (bf16, e4m3 and NVFP4; ranges of 4 heads at
+512x512, of 3 heads and a last one of 1 at 480x832, of one head in the tiny shape).
 """
 from dataclasses import replace
 
@@ -46,10 +48,20 @@ def _pinned(torch, x):
     return h
 
 
-@pytest.mark.parametrize("name,states,blocks", [("tiny", 3, 12), ("fp8_480x832", 8, 5)])
-def test_host_buffers_match_device_buffers(torch, name, states, blocks):
+@pytest.mark.parametrize("name,states,blocks,kw", [
+    ("tiny", 3, 12, {}),
+    ("fp8_480x832", 8, 5, {}),
+    # one state: chunks of heads (strided copies), in every storage format
+    ("tiny", 1, 12, {}),
+    ("tiny", 1, 8, {"fp8": True}),
+    ("tiny", 1, 8, {"fp4": True}),
+    ("512x512", 1, 5, {}),
+    ("fp8_480x832", 1, 4, {}),
+    ("nvfp4_480x832", 1, 4, {}),
+])
+def test_host_buffers_match_device_buffers(torch, name, states, blocks, kw):
     import compressed_kv_cache_convkv_b200 as ckv
-    w = replace(PRESETS[name], num_states=states)
+    w = replace(PRESETS[name], num_states=states, **kw)
     weights = device_weights(w, torch)
     dev = ckv.ConvKV(w.config(), weights)
     hio = ckv.ConvKV(w.config(host_io=True), weights)
