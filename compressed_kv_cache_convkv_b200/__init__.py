@@ -44,6 +44,8 @@ _SIGNATURES = {
     "convkv_append_block_host": (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     "convkv_attend_host": (ctypes.c_int, [_P, _P, _P]),
     "convkv_step_host": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int]),
+    "convkv_step_host_async": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int]),
+    "convkv_sync": (ctypes.c_int, [_P]),
     "convkv_state_bytes": (ctypes.c_size_t, [_P]),
     "convkv_destroy": (None, [_P]),
     "convkv_layout": (ctypes.c_int, [_P, _P, ctypes.c_int]),
@@ -291,15 +293,30 @@ class ConvKV:
         self._frames_of(q, "q")
         self._check(_lib().convkv_attend_host(self._h, q.data_ptr(), out.data_ptr()), "convkv_attend_host")
 
-    def step_host(self, k, v, q, out) -> None:
-        """append_host(k, v) then attend_host(q, out) as one pipelined call (host buffers,
-        pinned for overlap): per chunk of states, copies in, ring append, attention and
-        the copy back overlap the other chunks'."""
+    def _step_frames(self, k, v, q) -> int:
         fk, fq = self._frames_of(k, "k"), self._frames_of(q, "q")
         if fk != self._frames_of(v, "v") or fk != fq:
             raise ValueError("k, v and q must carry the same number of frames")
+        return fk
+
+    def step_host(self, k, v, q, out) -> None:
+        """append_host(k, v) then attend_host(q, out) as one pipelined call (host buffers,
+        pinned for overlap): per chunk, copies in, ring append, attention and the copy
+        back overlap the other chunks'."""
+        fk = self._step_frames(k, v, q)
         self._check(_lib().convkv_step_host(self._h, k.data_ptr(), v.data_ptr(), q.data_ptr(), out.data_ptr(), fk),
                     "convkv_step_host")
+
+    def step_host_async(self, k, v, q, out) -> None:
+        """step_host, returned once queued: the next step's copies overlap this step's
+        kernels.  Keep the buffers alive and unchanged (out unread) until sync()."""
+        fk = self._step_frames(k, v, q)
+        self._check(_lib().convkv_step_host_async(self._h, k.data_ptr(), v.data_ptr(), q.data_ptr(),
+                                                  out.data_ptr(), fk), "convkv_step_host_async")
+
+    def sync(self) -> None:
+        """Wait for every queued call of the handle (kernels and host copies)."""
+        self._check(_lib().convkv_sync(self._h), "convkv_sync")
 
     def dry_append(self, frames: int) -> None:
         """Advance the bookkeeping only (dry-run handles)."""

@@ -96,13 +96,18 @@ struct convkv {
   float4* tables = nullptr;
   int* status = nullptr;
   void *io_q = nullptr, *io_k = nullptr, *io_v = nullptr, *io_out = nullptr;
-  // host I/O (CONVKV_FLAG_HOST_IO): the *_host entry points copy by chunks of states
-  // on their own streams, and each chunk's kernels wait only for that chunk's copy, so
-  // copies in both directions overlap the kernels of other chunks
+  // host I/O (CONVKV_FLAG_HOST_IO): the *_host entry points copy by chunks (of states,
+  // or of one state's heads) on their own streams, and each chunk's kernels wait only
+  // for that chunk's copy, so copies in both directions overlap the kernels of other
+  // chunks -- and of the previous call's chunks: a chunk's staging is refilled as soon
+  // as the previous call's kernels and copy back of that chunk are done
   cudaStream_t io_in = nullptr, io_back = nullptr;
-  std::vector<cudaEvent_t> io_ev;  // [0] start, [1 + c] chunk c copied in, [1 + nchunks + c] chunk c done
+  // n = io_nchunks events each: [c] chunk c copied in (io_in), [n + c] chunk c's
+  // kernels done (stream), [2n + c] chunk c's outputs copied back (io_back)
+  std::vector<cudaEvent_t> io_ev;
   std::vector<IoChunk> io_chunks;  // in stream order
   int io_nchunks = 0;
+  int io_frames = 0;               // block frames of the previous host-buffer call
   bool io_pending = false;         // the next ring append reads io_k / io_v chunk by chunk
   bool io_defer = false;           // the ring append is left to the caller (convkv_step_host)
   AppendParams io_ap{};            // ... with these parameters
@@ -137,6 +142,13 @@ struct convkv {
     return cudaSuccess;
   }
   int64_t frame_elems() const { return static_cast<int64_t>(T) * H * D; }
+  cudaEvent_t ev_in(int c) const { return io_ev[c]; }
+  cudaEvent_t ev_done(int c) const { return io_ev[io_nchunks + c]; }
+  cudaEvent_t ev_out(int c) const { return io_ev[2 * io_nchunks + c]; }
+  // The previous host-buffer call's chunk whose events cover the staging region of
+  // chunk c for blocks of `frames` frames: the same chunk when the layout is the same,
+  // else the last one (the streams run the chunks in order, so it covers them all).
+  int io_prev(int c, int frames) const { return frames == io_frames ? c : io_nchunks - 1; }
   int m() const { return static_cast<int>(Sn < C ? Sn : C); }
   int w() const { return static_cast<int>(P - E); }
 };
@@ -386,7 +398,7 @@ static int create_host_io(convkv_t* h) {
   if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)
     return CONVKV_ERR_CUDA;
-  h->io_ev.assign(1 + 2 * h->io_nchunks, nullptr);
+  h->io_ev.assign(3 * static_cast<size_t>(h->io_nchunks), nullptr);
   for (auto& ev : h->io_ev)
     if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return CONVKV_ERR_CUDA;
   return CONVKV_OK;
@@ -668,7 +680,7 @@ static AppendParams states_slice(const convkv_t* h, const AppendParams& a, int g
 static int ring_append_chunk(convkv_t* h, const AppendParams& ap, const void* k, const void* v, const IoChunk& ck,
                              int c) {
   if (c >= 0) {
-    cudaError_t w = cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0);
+    cudaError_t w = cudaStreamWaitEvent(h->stream, h->ev_in(c), 0);
     if (w != cudaSuccess) return h->cuda_fail(w);
   }
   const int frames = ap.b, g0 = ck.g0;
@@ -690,6 +702,11 @@ static int ring_append_chunk(convkv_t* h, const AppendParams& ap, const void* k,
     h->launches++;
   }
   if (e) return h->cuda_fail(static_cast<cudaError_t>(e));
+  // the chunk's k / v staging is free for the next call once these kernels are done
+  if (c >= 0) {
+    cudaError_t w = cudaEventRecord(h->ev_done(c), h->stream);
+    if (w != cudaSuccess) return h->cuda_fail(w);
+  }
   return CONVKV_OK;
 }
 
@@ -988,15 +1005,19 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
   vm[3] = r ? h->mapSinkV : vm[2];
   const size_t bps = static_cast<size_t>(b) * h->frame_elems() * 2;   // query / output bytes per state
   // before chunk c's attention: wait for its queries; after it: send its outputs back
+  // (and for the previous call's copy back of the chunk's output staging)
   auto io_before = [&](int c) -> cudaError_t {
-    return c >= 0 ? cudaStreamWaitEvent(h->stream, h->io_ev[1 + c], 0) : cudaSuccess;
+    if (c < 0) return cudaSuccess;
+    cudaError_t e = cudaStreamWaitEvent(h->stream, h->ev_in(c), 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->stream, h->ev_out(h->io_prev(c, b)), 0);
+    return e;
   };
   auto io_after = [&](int c) -> cudaError_t {
     if (c < 0) return cudaSuccess;
-    cudaEvent_t done = h->io_ev[1 + h->io_nchunks + c];
-    cudaError_t e = cudaEventRecord(done, h->stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, done, 0);
+    cudaError_t e = cudaEventRecord(h->ev_done(c), h->stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, h->ev_done(c), 0);
     if (e == cudaSuccess) e = copy_chunk(h, h->io_chunks[c], out_host, out, bps, cudaMemcpyDeviceToHost, h->io_back);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_out(c), h->io_back);
     return e;
   };
   // the launches: the host-buffer chunks [cbeg, cend) (index c), else all states at
@@ -1095,18 +1116,32 @@ int convkv_attend_sp(convkv_t* h, const void* const* q_shards, void* const* out_
   return attend_impl(h, nullptr, nullptr, q_shards, out_shards);
 }
 
-// Copies of `bps` bytes per state from host to device staging, chunk by chunk on the
-// copy stream, each chunk's completion recorded in its event; the copies start after
-// the work already queued on the handle's stream (which may still read the staging).
-static cudaError_t copy_in_chunks(convkv_t* h, void* const* dst, const void* const* src, int nbuf, size_t bps) {
-  cudaError_t e = cudaEventRecord(h->io_ev[0], h->stream);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_in, h->io_ev[0], 0);
+// Copies of `bps` bytes per state (blocks of `frames` frames) from host to device
+// staging, chunk by chunk on the copy stream, each chunk's completion recorded in its
+// event.  A chunk's copy waits only until the previous host-buffer call no longer
+// reads that chunk's staging (its kernels of the chunk are done), so it overlaps the
+// previous call's later chunks.
+static cudaError_t copy_in_chunks(convkv_t* h, void* const* dst, const void* const* src, int nbuf, size_t bps,
+                                  int frames) {
+  cudaError_t e = cudaSuccess;
   for (int c = 0; c < h->io_nchunks && e == cudaSuccess; ++c) {
+    e = cudaStreamWaitEvent(h->io_in, h->ev_done(h->io_prev(c, frames)), 0);
     for (int i = 0; i < nbuf && e == cudaSuccess; ++i)
       e = copy_chunk(h, h->io_chunks[c], dst[i], src[i], bps, cudaMemcpyHostToDevice, h->io_in);
-    if (e == cudaSuccess) e = cudaEventRecord(h->io_ev[1 + c], h->io_in);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_in(c), h->io_in);
   }
   return e;
+}
+
+// Waits for everything the handle's three streams hold; the first error.
+static int sync_all(convkv_t* h) {
+  const cudaError_t e1 = cudaStreamSynchronize(h->io_in);
+  const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
+  const cudaError_t e3 = cudaStreamSynchronize(h->stream);
+  if (e1 != cudaSuccess) return h->cuda_fail(e1);
+  if (e2 != cudaSuccess) return h->cuda_fail(e2);
+  if (e3 != cudaSuccess) return h->cuda_fail(e3);
+  return CONVKV_OK;
 }
 
 int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host, int frames) {
@@ -1115,16 +1150,17 @@ int convkv_append_block_host(convkv_t* h, const void* k_host, const void* v_host
   const size_t bps = static_cast<size_t>(frames) * h->frame_elems() * 2;
   void* const dst[2] = {h->io_k, h->io_v};
   const void* const src[2] = {k_host, v_host};
-  cudaError_t e = copy_in_chunks(h, dst, src, 2, bps);
+  cudaError_t e = copy_in_chunks(h, dst, src, 2, bps, frames);
   if (e != cudaSuccess) {
-    cudaStreamSynchronize(h->io_in);
+    sync_all(h);
     return h->cuda_fail(e);
   }
   // the conv of the evicted frames runs while the block is copied in; the ring append
-  // of each chunk of states waits for that chunk's copy
+  // of each chunk waits for that chunk's copy
   h->io_pending = true;
   const int rc = convkv_append_block(h, h->io_k, h->io_v, frames);
   h->io_pending = false;
+  h->io_frames = frames;
   // the caller may reuse its buffers once this returns
   e = cudaStreamSynchronize(h->io_in);
   if (rc != CONVKV_OK) return rc;
@@ -1139,25 +1175,22 @@ int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host) {
   const size_t bps = static_cast<size_t>(h->bcur) * h->frame_elems() * 2;
   void* const dst[1] = {h->io_q};
   const void* const src[1] = {q_host};
-  // queries in by chunks of states; each chunk's attention waits for its queries and
-  // its outputs go back on the second copy stream while later chunks compute
-  cudaError_t e = copy_in_chunks(h, dst, src, 1, bps);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, h->io_ev[0], 0);
+  // queries in by chunks; each chunk's attention waits for its queries and its
+  // outputs go back on the second copy stream while later chunks compute
+  cudaError_t e = copy_in_chunks(h, dst, src, 1, bps, h->bcur);
   int rc = CONVKV_OK;
   if (e == cudaSuccess) rc = attend_impl(h, h->io_q, h->io_out, nullptr, nullptr, static_cast<char*>(out_host));
-  const cudaError_t e1 = cudaStreamSynchronize(h->io_in);
-  const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
-  const cudaError_t e3 = cudaStreamSynchronize(h->stream);
+  h->io_frames = h->bcur;
+  const int rs = sync_all(h);
   if (e != cudaSuccess) return h->cuda_fail(e);
   if (rc != CONVKV_OK) return rc;
-  if (e1 != cudaSuccess) return h->cuda_fail(e1);
-  if (e2 != cudaSuccess) return h->cuda_fail(e2);
-  if (e3 != cudaSuccess) return h->cuda_fail(e3);
-  return CONVKV_OK;
+  return rs;
 }
 
-int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
-                     int frames) {
+// The enqueue of one host-buffer step (convkv_step_host_async); on failure everything
+// already queued is waited for, and the step is undone as a failed append.
+static int step_host_enqueue(convkv_t* h, const void* k_host, const void* v_host, const void* q_host,
+                             void* out_host, int frames) {
   if (!h || !k_host || !v_host || !q_host || !out_host || frames < 1 || frames > h->Bmax)
     return CONVKV_ERR_INVALID_ARG;
   if (!h->host_io || h->dry) return CONVKV_ERR_BAD_ORDER;
@@ -1165,10 +1198,9 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
   const size_t bps = static_cast<size_t>(frames) * h->frame_elems() * 2;
   void* const dst[3] = {h->io_k, h->io_v, h->io_q};
   const void* const src[3] = {k_host, v_host, q_host};
-  cudaError_t e = copy_in_chunks(h, dst, src, 3, bps);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->io_back, h->io_ev[0], 0);
+  cudaError_t e = copy_in_chunks(h, dst, src, 3, bps, frames);
   if (e != cudaSuccess) {
-    cudaStreamSynchronize(h->io_in);
+    sync_all(h);
     return h->cuda_fail(e);
   }
   // bookkeeping, conv, time table and key rotation for all states (while the block is
@@ -1197,14 +1229,31 @@ int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const 
     }
   }
   h->io_pending = false;
-  const cudaError_t e1 = cudaStreamSynchronize(h->io_in);
-  const cudaError_t e2 = cudaStreamSynchronize(h->io_back);
-  const cudaError_t e3 = cudaStreamSynchronize(h->stream);
+  h->io_frames = frames;
+  if (rc != CONVKV_OK) sync_all(h);
+  return rc;
+}
+
+int convkv_step_host_async(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
+                           int frames) {
+  return step_host_enqueue(h, k_host, v_host, q_host, out_host, frames);
+}
+
+int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
+                     int frames) {
+  const int rc = step_host_enqueue(h, k_host, v_host, q_host, out_host, frames);
   if (rc != CONVKV_OK) return rc;
-  if (e1 != cudaSuccess) return h->cuda_fail(e1);
-  if (e2 != cudaSuccess) return h->cuda_fail(e2);
-  if (e3 != cudaSuccess) return h->cuda_fail(e3);
-  return CONVKV_OK;
+  return sync_all(h);
+}
+
+int convkv_sync(convkv_t* h) {
+  if (!h) return CONVKV_ERR_INVALID_ARG;
+  if (h->dry) return CONVKV_OK;
+  if (!h->host_io) {
+    const cudaError_t e = cudaStreamSynchronize(h->stream);
+    return e == cudaSuccess ? CONVKV_OK : h->cuda_fail(e);
+  }
+  return sync_all(h);
 }
 
 int convkv_host_chunks(const convkv_t* h, int32_t* rec, int cap) {

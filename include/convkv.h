@@ -157,6 +157,22 @@ int convkv_attend_host(convkv_t* h, const void* q_host, void* out_host);
 int convkv_step_host(convkv_t* h, const void* k_host, const void* v_host, const void* q_host, void* out_host,
                      int frames);
 
+/* The same step, returned as soon as it is queued: the copies in of the next step's
+ * chunks then overlap this step's later kernels (a chunk's staging is refilled as soon
+ * as the previous step's kernels and copy back of that chunk are done), so a stream
+ * of steps runs at the rate of the slower of the kernels and the copies.  The host
+ * buffers of every queued step must stay valid, the inputs unchanged and the outputs
+ * unread, until convkv_sync returns.  Argument and order errors are returned at once
+ * with nothing queued; a failure while queueing is waited out and counts as a failed
+ * append, as for convkv_step_host; device-side errors show in convkv_sync.  Needs
+ * CONVKV_FLAG_HOST_IO. */
+int convkv_step_host_async(convkv_t* h, const void* k_host, const void* v_host, const void* q_host,
+                           void* out_host, int frames);
+
+/* Waits until every queued call of the handle has ended (its kernels, and with
+ * CONVKV_FLAG_HOST_IO its copies in both directions).  Errors: INVALID_ARG, CUDA. */
+int convkv_sync(convkv_t* h);
+
 /* Device bytes owned by the handle; constant from create to destroy. */
 size_t convkv_state_bytes(const convkv_t* h);
 

@@ -93,6 +93,10 @@ def test_call_order_and_argument_checks():
     assert lib.convkv_step_host(h._h, p, p, p, p, 2) == ckv.ERR_BAD_ORDER
     assert lib.convkv_step_host(h._h, p, p, p, p, 3) == ckv.ERR_INVALID_ARG   # > max block
     assert lib.convkv_append_block_host(h._h, p, p, 2) == ckv.ERR_BAD_ORDER
+    assert lib.convkv_step_host_async(h._h, p, p, p, p, 2) == ckv.ERR_BAD_ORDER
+    assert lib.convkv_step_host_async(h._h, None, p, p, p, 2) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_step_host_async(h._h, p, p, p, p, 0) == ckv.ERR_INVALID_ARG
+    assert lib.convkv_sync(h._h) == ckv.OK and lib.convkv_sync(None) == ckv.ERR_INVALID_ARG
     assert h.counters() == c1
     assert lib.convkv_state_bytes(h._h) == 0 and h.launch_count() == 0
     lib.convkv_destroy(None)

@@ -1,5 +1,5 @@
-"""The host-buffer entry points (convkv_append_block_host / convkv_attend_host) against
-the device-buffer ones, on the GPU.
+"""The host-buffer entry points (convkv_append_block_host / convkv_attend_host /
+convkv_step_host / convkv_step_host_async) against the device-buffer ones, on the GPU.
 
 The host forms copy their inputs in by chunks on a copy stream, start each chunk's
 kernels as soon as its copy lands, and copy each chunk's outputs back while later
@@ -120,6 +120,45 @@ def test_step_host_failure_rolls_back_and_recovers(torch, step):
         torch.cuda.synchronize()
         assert np.array_equal(o_dev.view(torch.int16).cpu().numpy(), oh.view(torch.int16).numpy()), (step, i)
         assert dev.counters() == hio.counters()
+    assert dev.status() == 0 and hio.status() == 0
+    dev.close()
+    hio.close()
+
+
+@pytest.mark.parametrize("name,states,blocks,kw", [
+    ("tiny", 3, 10, {}),
+    ("tiny", 1, 8, {"fp8": True}),
+    ("512x512", 1, 5, {}),
+    ("fp8_480x832", 4, 3, {}),
+])
+def test_queued_steps_match_device_buffers(torch, name, states, blocks, kw):
+    """Host-buffer steps queued back to back (convkv_step_host_async, one convkv_sync at
+    the end): each chunk's copy in waits only for the previous step's kernels and copy
+    back of that chunk, so steps overlap.  Every step's outputs must equal the device
+    path's bit for bit.  At 512x512 the first block has 6 frames and the others 8,
+    which moves every chunk's staging region: there the second step's copies must wait
+    for the whole first step."""
+    import compressed_kv_cache_convkv_b200 as ckv
+    w = replace(PRESETS[name], num_states=states, **kw)
+    weights = device_weights(w, torch)
+    dev = ckv.ConvKV(w.config(), weights)
+    hio = ckv.ConvKV(w.config(host_io=True), weights)
+    frame0 = 0
+    expected, queued = [], []
+    for frames in w.block_sizes()[:blocks]:
+        q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
+        frame0 += frames
+        dev.append(k, v)
+        expected.append(dev.attend(q))
+        qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        hio.step_host_async(kh, vh, qh, oh)
+        queued.append((qh, kh, vh, oh))   # every queued step's buffers stay alive
+    hio.sync()
+    torch.cuda.synchronize()
+    for i, (o_dev, (_, _, _, oh)) in enumerate(zip(expected, queued)):
+        assert np.array_equal(o_dev.view(torch.int16).cpu().numpy(), oh.view(torch.int16).numpy()), (name, i)
+    assert dev.counters() == hio.counters()
     assert dev.status() == 0 and hio.status() == 0
     dev.close()
     hio.close()
