@@ -89,7 +89,9 @@ struct convkv {
   uint8_t *ringBK = nullptr, *ringBV = nullptr, *memBK = nullptr, *memBV = nullptr;
   void *sinkK = nullptr, *sinkV = nullptr;    // bf16 reference frames, both formats
   void *scrK = nullptr, *scrV = nullptr;      // e4m3 / NVFP4: bf16 scratch [Sg][(C + W) * T][H][D]
-  int Sg = 0;                                 // states per dequantise-and-attend group
+  int Sg = 0;                                 // states the dequantisation scratch holds
+  int Sa = 0;                                 // states per dequantise-and-attend launch (<= Sg)
+  int sms = 148;                              // SMs of the device (148 for a dry-run handle)
   unsigned int* amax = nullptr;               // amax scratch of the quantisation passes
   float* convacc = nullptr;                   // e4m3 / NVFP4: fp32 conv outputs of one append
   int gmax = 0;                               // eviction groups one append can produce
@@ -142,6 +144,8 @@ struct convkv {
     return cudaSuccess;
   }
   int64_t frame_elems() const { return static_cast<int64_t>(T) * H * D; }
+  // attention CTAs per head and state of a steady block (one per 256 query rows)
+  int64_t ctas_per_head() const { return (static_cast<int64_t>(bn) * T + 255) / 256; }
   cudaEvent_t ev_in(int c) const { return io_ev[c]; }
   cudaEvent_t ev_done(int c) const { return io_ev[io_nchunks + c]; }
   cudaEvent_t ev_out(int c) const { return io_ev[2 * io_nchunks + c]; }
@@ -306,6 +310,21 @@ static double idle_share(int64_t ctas, int sms) {
   return static_cast<double>(full - ctas) / static_cast<double>(full);
 }
 
+// The group size in [1, cap] whose grid of ctas_per_state CTAs per state leaves the
+// smallest share of its last wave idle.
+static int wave_group(int64_t ctas_per_state, int cap, int sms) {
+  int c = 1;
+  double best = 2.0;
+  for (int n = 1; n <= cap; ++n) {
+    const double idle = idle_share(ctas_per_state * n, sms);
+    if (idle < best - 1e-12) {
+      best = idle;
+      c = n;
+    }
+  }
+  return c;
+}
+
 // Chunks of the host-buffer entry points.
 //
 // Several states: chunks of whole states.  The first chunk is one state, so the
@@ -353,16 +372,7 @@ static void plan_host_chunks(int S, int H, int D, int cap, int64_t ctas_per_head
     for (int h0 = 0; h0 < H; h0 += hg) out.push_back({0, 1, h0, H - h0 < hg ? H - h0 : hg});
     return;
   }
-  const int hi = cap < 6 ? (cap > 0 ? cap : 1) : 6;
-  int c = 1;
-  double best = 2.0;
-  for (int n = 1; n <= hi; ++n) {
-    const double idle = idle_share(ctas_per_head * H * n, sms);
-    if (idle < best - 1e-12) {
-      best = idle;
-      c = n;
-    }
-  }
+  const int c = wave_group(ctas_per_head * H, cap < 6 ? (cap > 0 ? cap : 1) : 6, sms);
   std::vector<int> tail;
   for (int t = c; t > 1;) {
     t = (t + 2) / 3;
@@ -387,13 +397,7 @@ static void plan_host_chunks(int S, int H, int D, int cap, int64_t ctas_per_head
 
 // Copy streams and events of the host-buffer entry points, and their chunk plan.
 static int create_host_io(convkv_t* h) {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
-    return CONVKV_ERR_CUDA;
-  // the attention launches one CTA per 256 query rows and head (steady blocks)
-  const int64_t ctas = (static_cast<int64_t>(h->bn) * h->T + 255) / 256;
-  plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, ctas, sms, h->io_chunks);
+  plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, h->ctas_per_head(), h->sms, h->io_chunks);
   h->io_nchunks = static_cast<int>(h->io_chunks.size());
   if (cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->io_back, cudaStreamNonBlocking) != cudaSuccess)
@@ -456,11 +460,19 @@ int convkv_create(const convkv_cfg* cfg, convkv_t** out) {
     const size_t budget = size_t(4) << 30;
     h->Sg = static_cast<int>(per_state * h->S <= budget ? h->S : (budget / per_state > 0 ? budget / per_state : 1));
   }
+  if (!h->dry) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || h->sms < 1) {
+      delete h;
+      return CONVKV_ERR_CUDA;
+    }
+  }
+  // the e4m3 / NVFP4 attend runs in launches of Sa states that fill the last wave best
+  h->Sa = h->fp8 ? wave_group(h->ctas_per_head() * h->H, h->Sg, h->sms) : h->S;
   if (h->dry) {
     // the host-buffer chunk plan only, for a B200's 148 SMs (no device is queried)
-    if (h->host_io)
-      plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, (static_cast<int64_t>(h->bn) * h->T + 255) / 256,
-                       148, h->io_chunks);
+    if (h->host_io) plan_host_chunks(h->S, h->H, h->D, h->fp8 ? h->Sg : h->S, h->ctas_per_head(), h->sms, h->io_chunks);
     *out = h;
     return CONVKV_OK;
   }
@@ -1021,7 +1033,8 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     return e;
   };
   // the launches: the host-buffer chunks [cbeg, cend) (index c), else all states at
-  // once (bf16) or groups of Sg states (the scratch's capacity), with every head
+  // once (bf16) or groups of Sa states (at most the scratch's capacity, sized so that
+  // the attention fills its last wave best), with every head
   struct Unit {
     IoChunk ck;
     int c;
@@ -1031,7 +1044,7 @@ static int attend_impl(convkv_t* h, const void* q, void* out, const void* const*
     if (cend < 0) cend = h->io_nchunks;
     for (int c = cbeg; c < cend; ++c) units.push_back({h->io_chunks[c], c});
   } else {
-    const int step = h->fp8 ? h->Sg : h->S;
+    const int step = h->fp8 ? h->Sa : h->S;
     for (int g0 = 0; g0 < h->S; g0 += step) units.push_back({{g0, h->S - g0 < step ? h->S - g0 : step, 0, h->H}, -1});
   }
   if (!h->fp8) {
