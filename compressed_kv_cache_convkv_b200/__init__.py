@@ -49,7 +49,7 @@ _SIGNATURES = {
     "convkv_state_bytes": (ctypes.c_size_t, [_P]),
     "convkv_destroy": (None, [_P]),
     "convkv_layout": (ctypes.c_int, [_P, _P, ctypes.c_int]),
-    "convkv_host_chunks": (ctypes.c_int, [_P, _P, ctypes.c_int]),
+    "convkv_host_chunks": (ctypes.c_int, [_P, ctypes.c_int, _P, ctypes.c_int]),
     "convkv_counters": (ctypes.c_int, [_P, _P]),
     "convkv_read_slot": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]),
     "convkv_read_ring": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]),
@@ -344,14 +344,15 @@ class ConvKV:
         _lib().convkv_layout(self._h, rec.ctypes.data, n)
         return rec[:n]
 
-    def host_chunks(self):
-        """The host-buffer chunk plan: rows of (first state, states, first head, heads)."""
+    def host_chunks(self, queued: bool = False):
+        """The host-buffer chunk plan: rows of (first state, states, first head, heads);
+        queued: the plan of a queued step that follows a queued step."""
         import numpy as np
-        n = _lib().convkv_host_chunks(self._h, None, 0)
+        n = _lib().convkv_host_chunks(self._h, int(queued), None, 0)
         if n < 0:
             raise ConvKVError(n, "convkv_host_chunks")
         rec = np.zeros((max(n, 1), 4), dtype=np.int32)
-        _lib().convkv_host_chunks(self._h, rec.ctypes.data, n)
+        _lib().convkv_host_chunks(self._h, int(queued), rec.ctypes.data, n)
         return rec[:n]
 
     def _read(self, fn, name: str, state: int, kv: int, idx: int):

@@ -232,10 +232,14 @@ int convkv_layout(const convkv_t* h, int32_t* rec, int cap);
 /* Chunk plan of the host-buffer entry points, in stream order, 4 int32 per chunk:
  * {first state, states, first head, heads}.  With several states the chunks are
  * whole states (all heads); with one state they are ranges of its heads (strided
- * copies of nh * D values per token).  A handle created with CONVKV_FLAG_HOST_IO has
- * the plan (a dry-run handle too, planned for 148 SMs); any other handle has none.
- * Returns the number of chunks, or a negative error; writes at most `cap` records. */
-int convkv_host_chunks(const convkv_t* h, int32_t* rec, int cap);
+ * copies of nh * D values per token).  queued = 0: the plan of a call that follows a
+ * synchronised one (it ramps up from one state and down to one); queued != 0: the
+ * plan of a queued step (convkv_step_host_async) that follows a queued step (steady
+ * chunks; its copies in ran during the previous step).  A handle created with
+ * CONVKV_FLAG_HOST_IO has the plans (a dry-run handle too, planned for 148 SMs); any
+ * other handle has none.  Returns the number of chunks, or a negative error; writes
+ * at most `cap` records. */
+int convkv_host_chunks(const convkv_t* h, int queued, int32_t* rec, int cap);
 
 /* Counters {P promoted frames, E evicted frames, S slots produced, m stored
  * slots, w window frames, b current frames, blocks appended, groups compressed

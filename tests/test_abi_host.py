@@ -268,8 +268,8 @@ def test_noalloc_quantiser_rejects_misaligned_pointers_before_any_work():
         assert lib.convkv_quantize_e4m3_noalloc(x, c, s, 1, 16, 2, 64, None) == ckv.ERR_INVALID_ARG
 
 
-def _plan(w, **kw):
-    return _dry(w, host_io=True, **kw).host_chunks().tolist()
+def _plan(w, queued=False, **kw):
+    return _dry(w, host_io=True, **kw).host_chunks(queued).tolist()
 
 
 def test_host_chunk_plan_covers_every_state_and_head_once():
@@ -280,8 +280,8 @@ def test_host_chunk_plan_covers_every_state_and_head_once():
     cases += [(replace(PRESETS["fp8_480x832"], num_states=s), {}) for s in (1, 2, 7, 8, 13)]
     cases += [(replace(PRESETS["tiny"], num_states=s), {}) for s in (1, 2, 3, 5)]
     cases += [(replace(PRESETS["512x512"], num_states=s), {}) for s in (2, 40)]
-    for w, kw in cases:
-        plan = _plan(w, **kw)
+    for (w, kw), queued in [(c, q) for c in cases for q in (False, True)]:
+        plan = _plan(w, queued, **kw)
         H, S = w.heads, w.num_states
         seen = np.zeros((S, H), dtype=int)
         for g0, n, h0, nh in plan:
@@ -295,7 +295,10 @@ def test_host_chunk_plan_covers_every_state_and_head_once():
         if S > 1:
             assert all(nh == H for _, _, _, nh in plan)
             sizes = [n for _, n, _, _ in plan]
-            assert sizes[0] == 1 and sizes[-1] == 1, sizes
+            if not queued:
+                assert sizes[0] == 1 and sizes[-1] == 1, sizes
+            else:
+                assert len(sizes) >= 2 and len(set(sizes[:-1])) <= 1 and sizes[-1] <= sizes[0], sizes
         elif H > 1:
             assert len(plan) >= 2
     # a handle without host buffers has no plan
@@ -310,6 +313,8 @@ def test_host_chunk_plan_fills_waves_at_the_bench_shapes():
     ranges are at least 512 bytes per token row."""
     fp8 = _plan(PRESETS["fp8_480x832"])
     assert [n for _, n, _, _ in fp8] == [1, 1, 1, 2, 2, 3, 4, 4, 4, 4, 4, 4, 3, 2, 1]
+    assert [n for _, n, _, _ in _plan(PRESETS["fp8_480x832"], True)] == [7] * 5 + [5]
+    assert _plan(PRESETS["512x512"], True) == _plan(PRESETS["512x512"])
     assert max(n for _, n, _, _ in fp8) <= 7        # the e4m3 dequantisation group
     assert _plan(PRESETS["512x512"]) == [[0, 1, h, 4] for h in range(0, 40, 4)]
     assert _plan(PRESETS["720x416"]) == [[0, 1, h, 4] for h in range(0, 40, 4)]
