@@ -18,7 +18,7 @@ import pytest
 
 import seeded_inputs as si
 from compressed_kv_cache_convkv_b200.configs import PRESETS
-from streams import device_weights
+from streams import device_frames, device_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -162,3 +162,41 @@ def test_queued_steps_match_device_buffers(torch, name, states, blocks, kw):
     assert dev.status() == 0 and hio.status() == 0
     dev.close()
     hio.close()
+
+
+@pytest.mark.parametrize("name,states", [("512x512", 1), ("tiny", 3)])
+def test_host_buffers_with_reference_frames(torch, name, states):
+    """With a reference-image partition (one frame, attended first and never evicted)
+    the host forms still equal the device form bit for bit: the reference keys enter
+    every chunk's attention through their own tensor maps, with head ranges (one
+    state) and whole-state chunks (three states), synchronous and queued."""
+    import compressed_kv_cache_convkv_b200 as ckv
+    w = replace(PRESETS[name], num_states=states)
+    weights = device_weights(w, torch)
+    hs = [ckv.ConvKV(w.config(sink_frames=1, **kw), weights) for kw in ({}, {"host_io": True}, {"host_io": True})]
+    rk, rv = device_frames(w, si.RK, 0, 1, torch), device_frames(w, si.RV, 0, 1, torch)
+    for h in hs:
+        h.set_sink(rk, rv)
+    dev, sync, queued = hs
+    frame0 = 0
+    expected, outs = [], []
+    for frames in w.block_sizes()[:5]:
+        q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
+        frame0 += frames
+        dev.append(k, v)
+        expected.append(dev.attend(q))
+        qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
+        o1 = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        o2 = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        sync.step_host(kh, vh, qh, o1)
+        queued.step_host_async(kh, vh, qh, o2)
+        outs.append((qh, kh, vh, o1, o2))
+    queued.sync()
+    torch.cuda.synchronize()
+    for i, (o_dev, (_, _, _, o1, o2)) in enumerate(zip(expected, outs)):
+        a = o_dev.view(torch.int16).cpu().numpy()
+        assert np.array_equal(a, o1.view(torch.int16).numpy()), (name, i, "step_host")
+        assert np.array_equal(a, o2.view(torch.int16).numpy()), (name, i, "step_host_async")
+    for h in hs:
+        assert h.status() == 0
+        h.close()
