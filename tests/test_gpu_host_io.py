@@ -200,3 +200,45 @@ def test_host_buffers_with_reference_frames(torch, name, states):
     for h in hs:
         assert h.status() == 0
         h.close()
+
+
+def test_queued_step_failure_rolls_back_and_recovers(torch):
+    """A launch failure injected on the host while a queued step is being queued (behind
+    two queued steps still in flight): the call waits everything out, restores the
+    counters and refuses attends; the earlier queued steps' outputs are complete and
+    correct, and queueing the same step again gives the device path's outputs."""
+    import compressed_kv_cache_convkv_b200 as ckv
+    w = replace(PRESETS["tiny"], fp8=True, num_states=3, name="tiny_fp8")
+    weights = device_weights(w, torch)
+    dev = ckv.ConvKV(w.config(), weights)
+    hio = ckv.ConvKV(w.config(host_io=True), weights)
+    lib = ckv.library()
+    frame0 = 0
+    expected, queued = [], []
+    for i, frames in enumerate(w.block_sizes()[:8]):
+        q, k, v = (_block(torch, w, tid, frame0, frames) for tid in (si.Q, si.K, si.V))
+        frame0 += frames
+        dev.append(k, v)
+        expected.append(dev.attend(q))
+        qh, kh, vh = (_pinned(torch, x) for x in (q, k, v))
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        if i == 5:
+            # block 5 evicts a group, so the conv runs: fail it
+            before = hio.counters()
+            assert lib.convkv_debug_fail_step(hio._h, 0) == ckv.OK
+            rc = lib.convkv_step_host_async(hio._h, kh.data_ptr(), vh.data_ptr(), qh.data_ptr(), oh.data_ptr(), frames)
+            assert rc == ckv.ERR_CUDA
+            assert hio.counters() == before
+            assert lib.convkv_attend_host(hio._h, qh.data_ptr(), oh.data_ptr()) == ckv.ERR_BAD_ORDER
+            for j, (o_dev, (_, _, _, o)) in enumerate(zip(expected[:-1], queued)):
+                assert np.array_equal(o_dev.view(torch.int16).cpu().numpy(), o.view(torch.int16).numpy()), j
+        hio.step_host_async(kh, vh, qh, oh)
+        queued.append((qh, kh, vh, oh))
+    hio.sync()
+    torch.cuda.synchronize()
+    for i, (o_dev, (_, _, _, oh)) in enumerate(zip(expected, queued)):
+        assert np.array_equal(o_dev.view(torch.int16).cpu().numpy(), oh.view(torch.int16).numpy()), i
+    assert dev.counters() == hio.counters()
+    assert dev.status() == 0 and hio.status() == 0
+    dev.close()
+    hio.close()
