@@ -46,12 +46,34 @@ def attend_sources(fmt: str):
     return ATTN_SOURCES if fmt == "bf16" else ATTN_SOURCES + DEQUANT_SOURCES
 
 
+def parse_peaks(d):
+    """The roofline denominators from the measured peaks' JSON object: hbm_gbs,
+    bf16_tflops and bf16_tflops_sustained found at any depth, each missing or unusable
+    one replaced by its fallback.  Returns (peaks, {key: "measured" | "fallback"})."""
+    out, src = dict(FALLBACK_PEAKS), {k: "fallback" for k in FALLBACK_PEAKS}
+
+    def walk(x):
+        if isinstance(x, dict):
+            for k, v in x.items():
+                if k in FALLBACK_PEAKS and src[k] == "fallback" and isinstance(v, (int, float)) \
+                        and not isinstance(v, bool) and v > 0:
+                    out[k], src[k] = float(v), "measured"
+                else:
+                    walk(v)
+        elif isinstance(x, list):
+            for v in x:
+                walk(v)
+    walk(d)
+    return out, src
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+    try:
+        d = json.load(open(p)) if os.path.exists(p) else None
+    except (OSError, ValueError):
+        d = None
+    return parse_peaks(d)
 
 
 def kv_format(w) -> str:
@@ -426,7 +448,8 @@ def run_ours(args, w):
     # a kernel timed alone against the burst peak; one timed inside a seconds-long loop
     # (the 40-state workloads) against the sustained one, reached under the power cap
     sustained = total_ms > 1000.0
-    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    pkey = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = pk[pkey]
     kvb = kv_bytes_per_value(w)
     att_bytes = attention_bytes(b * T, statistics.mean(nk_list), D, H, S, kv_bytes=kvb,
                                 Nk_bf16=(b + r) * T if kvb < 2 else None)
@@ -468,9 +491,10 @@ def run_ours(args, w):
                      "frac": att_achieved / peak, "traffic": traffic,
                      "algorithmic_bytes": att_bytes, "kernel": kernel,
                      "peak_source": (f"measured bf16 {'sustained' if sustained else 'burst'} (MEASURED_PEAKS.json)"
-                                     if kind == "measured" else
-                                     f"fallback bf16 {'sustained (1400 TF/s' if sustained else 'burst (1590 TF/s'}, "
-                                     "earlier measurement on this pool; no MEASURED_PEAKS.json on the box)"),
+                                     if kind[pkey] == "measured" else
+                                     f"fallback bf16 {'sustained' if sustained else 'burst'} ({peak:.0f} TF/s, "
+                                     "earlier measurement on this pool; no such figure in MEASURED_PEAKS.json "
+                                     "on the box)"),
                      "frac_of_burst": att_achieved / pk["bf16_tflops"],
                      "traffic_source": traffic_src},
         "e2e": e2e_line,

@@ -55,3 +55,21 @@ def test_reference_arm_prints_one_line(capsys):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["steps"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_peaks_fall_back_per_figure():
+    """The measured peaks file may be absent, flat, nested or partial: each roofline
+    denominator is the measured figure when one is found (any depth), else its
+    fallback, and the source of each is reported."""
+    fb = dict(bench.FALLBACK_PEAKS)
+    pk, src = bench.parse_peaks(None)
+    assert pk == fb and set(src.values()) == {"fallback"}
+    pk, src = bench.parse_peaks({"hbm_gbs": 6543.4, "bf16_tflops": 1637.0, "bf16_tflops_sustained": 1386.2})
+    assert pk == {"hbm_gbs": 6543.4, "bf16_tflops": 1637.0, "bf16_tflops_sustained": 1386.2}
+    assert set(src.values()) == {"measured"}
+    pk, src = bench.parse_peaks({"gpu": {"bf16_tflops": 1600}, "clocks": [1965], "hbm_gbs": "n/a"})
+    assert pk["bf16_tflops"] == 1600.0 and src["bf16_tflops"] == "measured"
+    assert pk["hbm_gbs"] == fb["hbm_gbs"] and src["hbm_gbs"] == "fallback"
+    assert pk["bf16_tflops_sustained"] == fb["bf16_tflops_sustained"]
+    pk, _ = bench.parse_peaks({"bf16_tflops": -1, "bf16_tflops_sustained": True})
+    assert pk == fb
