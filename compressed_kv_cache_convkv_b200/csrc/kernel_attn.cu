@@ -57,7 +57,9 @@ struct AttnCfg {
   // most 384 threads can have, 65536 / 384 rounded down to a multiple of 8); the
   // producer/MMA warpgroup gives registers to the two softmax warpgroups, and the
   // split must stay within the launch allocation or an increase waits forever
-  static constexpr int REG_LAUNCH = 168, REG_CTRL = 96, REG_SOFTMAX = 200;
+  // producer / MMA warps 112 and softmax warps 192 registers: both roles without
+  // spills (at 96 / 200 the MMA issuer's loop reloaded spilled values from local memory)
+  static constexpr int REG_LAUNCH = 168, REG_CTRL = 112, REG_SOFTMAX = 192;
   static_assert(128 * REG_CTRL + 256 * REG_SOFTMAX <= THREADS * REG_LAUNCH,
                 "register split must fit the launch allocation");
   static constexpr int NBARS = 1 + 1 + 2 * KST + 2 * VST + 3 * 2 + 1;
